@@ -1,0 +1,408 @@
+"""CPU oracle for the DeepSeekMoE layer forward with FP8 fine-grained scaling.
+
+TEST INFRASTRUCTURE ONLY. This module is the plain, slow, obviously-correct
+definition that the CUDA path is checked against. Only the tests, the smoke
+check and the CPU-baseline leg of the benchmark may import it; the library
+never does, and the oracle imports nothing from the library.
+
+Arithmetic is float64 except where the method itself fixes a narrower type:
+the E4M3 codes, the float32 tile scales and the float32 routing bias.
+
+Sources (web pages on the DeepSeek-V3 technical report), cited by tag:
+  [Explained]  "DeepSeek-V3, explained" (vibeengines.com), the numbered recipe
+               and the symbol notes under it.
+  [Dissection] "DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing,
+               Multi-Token Prediction, and FP8 Training at 671B Scale"
+               (trishampatil.com); section III (routing equations, bias
+               controller) and section V (FP8 details).
+  [Deepforge]  "DeepSeek-V3 Technical Report" (deepforge.srivtx.xyz);
+               "Per-tile FP8 scaling" and "Build it yourself".
+
+Readings taken where the pages are silent (each is listed in the design
+notes with its reason):
+  * E4M3 is the OCP E4M3FN format, round-to-nearest-even, saturating to
+    +-448; zero keeps its sign.
+  * Tile scale = fp32(448 / amax) with an IEEE divide; codes are
+    e4m3(fp32(x * scale)); an all-zero tile gets scale 1.
+  * Top-K ties go to the lower expert id; output order is biased score
+    descending.
+  * Load target is the mean T*K/N, compared in integers as T*K - N*c_i.
+  * Combine order: shared expert first, then routed experts by ascending id.
+  * No residual add; no routed scaling factor.
+
+parity pins: every function here is pinned by a test under tests/ against a
+closed form, a worked example, an invariant, a library routine or brute
+force; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+E4M3_MAX = 448.0
+TILE = 128
+
+
+# ---------------------------------------------------------------------------
+# E4M3 codec  ([Deepforge] "FP8 training, from first principles" and
+# "Per-tile FP8 scaling": 4 exponent bits, 3 mantissa bits, largest 448)
+# ---------------------------------------------------------------------------
+
+def _build_decode_table() -> np.ndarray:
+    """Value of each of the 256 byte codes, from the bit layout.
+
+    Layout s eeee mmm, exponent bias 7. Exponent field 0 is subnormal
+    (m/8 * 2^-6); field 15 with mantissa 7 is NaN (E4M3FN has no infinity).
+    """
+    table = np.empty(256, dtype=np.float64)
+    for code in range(256):
+        sign = -1.0 if (code >> 7) & 1 else 1.0
+        exp_field = (code >> 3) & 0xF
+        man_field = code & 0x7
+        if exp_field == 0xF and man_field == 0x7:
+            table[code] = np.nan
+        elif exp_field == 0:
+            table[code] = sign * (man_field / 8.0) * 2.0 ** (1 - 7)
+        else:
+            table[code] = sign * (1.0 + man_field / 8.0) * 2.0 ** (exp_field - 7)
+    return table
+
+
+E4M3_DECODE = _build_decode_table()
+# positive finite values, codes 0x00 .. 0x7E, ascending
+_E4M3_POS = E4M3_DECODE[:0x7F].copy()
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """uint8 codes -> float64 values."""
+    return E4M3_DECODE[np.asarray(codes, dtype=np.uint8)]
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """float values -> uint8 E4M3 codes: nearest value, ties to even, saturate.
+
+    The nearest representable magnitude is found by bracketing |v| between two
+    adjacent positive codes; on an exact midpoint the code with the even
+    mantissa (low bit 0) wins. Magnitudes above 448 (and +-inf) become 448.
+    NaN becomes 0x7F. The sign bit is copied, so -0.0 encodes to 0x80.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    nan = np.isnan(v)
+    neg = np.signbit(v)
+    a = np.minimum(np.abs(np.where(nan, 0.0, v)), E4M3_MAX)
+    hi = np.searchsorted(_E4M3_POS, a, side="left")  # first code with value >= a
+    hi = np.minimum(hi, 0x7E)
+    lo = np.maximum(hi - 1, 0)
+    d_lo = a - _E4M3_POS[lo]
+    d_hi = _E4M3_POS[hi] - a
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    mag = np.where(take_hi, hi, lo).astype(np.uint8)
+    codes = np.where(neg, mag | 0x80, mag).astype(np.uint8)
+    codes = np.where(nan, np.uint8(0x7F), codes).astype(np.uint8)
+    return codes
+
+
+# ---------------------------------------------------------------------------
+# Fine-grained quantisation ([Explained] recipe step 7; [Dissection] section V
+# "Four details", item 1; [Deepforge] "Per-tile FP8 scaling" formula:
+# scale = max_fp8 / amax, X_fp8 = round(X * scale), X_hat = X_fp8 / scale)
+# ---------------------------------------------------------------------------
+
+def _tile_scale(amax_f32: np.ndarray) -> np.ndarray:
+    """fp32(448 / amax) with IEEE float32 division; 1.0 for an all-zero tile."""
+    amax_f32 = np.asarray(amax_f32, dtype=np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        s = np.float32(E4M3_MAX) / amax_f32
+    return np.where(amax_f32 > 0, s, np.float32(1.0)).astype(np.float32)
+
+
+def quantize_1x128(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Online activation quantisation, one scale per row per 128 columns.
+
+    x: float array [rows, cols] (cols a multiple of 128), taken as float32.
+    Returns codes uint8 [rows, cols] and scales float32 [rows, cols/128]
+    (the multiplier 448/amax, as the per-tile formula stores it).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    assert cols % TILE == 0
+    xt = x.reshape(rows, cols // TILE, TILE)
+    amax = np.max(np.abs(xt), axis=2)
+    scale = _tile_scale(amax)
+    with np.errstate(invalid="ignore", over="ignore"):
+        prod = (xt * scale[:, :, None]).astype(np.float32)  # one float32 multiply
+    codes = e4m3_encode(prod).reshape(rows, cols)
+    return codes, scale
+
+
+def quantize_128x128(w: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Weight quantisation, one scale per 128x128 block.
+
+    w: float array [rows, cols], both multiples of 128, taken as float32.
+    Returns codes uint8 [rows, cols] and scales float32 [rows/128, cols/128].
+    """
+    w = np.asarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    assert rows % TILE == 0 and cols % TILE == 0
+    wb = w.reshape(rows // TILE, TILE, cols // TILE, TILE)
+    amax = np.max(np.abs(wb), axis=(1, 3))
+    scale = _tile_scale(amax)
+    with np.errstate(invalid="ignore", over="ignore"):
+        prod = (wb * scale[:, None, :, None]).astype(np.float32)
+    codes = e4m3_encode(prod).reshape(rows, cols)
+    return codes, scale
+
+
+def dequantize_1x128(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """X_hat = X_fp8 / scale, in float64."""
+    rows, cols = codes.shape
+    v = e4m3_decode(codes).reshape(rows, cols // TILE, TILE)
+    return (v / np.asarray(scales, np.float64)[:, :, None]).reshape(rows, cols)
+
+
+def dequantize_128x128(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    rows, cols = codes.shape
+    v = e4m3_decode(codes).reshape(rows // TILE, TILE, cols // TILE, TILE)
+    return (v / np.asarray(scales, np.float64)[:, None, :, None]).reshape(rows, cols)
+
+
+# ---------------------------------------------------------------------------
+# Routing ([Dissection] section III "The mechanism": s = Sigmoid(u^T e_i),
+# g' = s if s + b in TopK(s + b, K) else 0, g = g' / sum g';
+# [Explained] recipe step 4 and the notes on b_i and K_r)
+# ---------------------------------------------------------------------------
+
+def gate_logits(x: np.ndarray, gate_w: np.ndarray) -> np.ndarray:
+    """z[t, i] = u_t . e_i in float64 (gating stays in high precision,
+    [Explained] recipe step 7; [Dissection] section V item 4)."""
+    return np.asarray(x, np.float64) @ np.asarray(gate_w, np.float64).T
+
+
+def sigmoid(z: np.ndarray) -> np.ndarray:
+    return 1.0 / (1.0 + np.exp(-np.asarray(z, np.float64)))
+
+
+def route(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int):
+    """Sigmoid affinity, biased top-K selection, unbiased normalised gates.
+
+    Returns (ids int32 [T,K], gates float64 [T,K], s float64 [T,N],
+    score float64 [T,N]) with ids ordered by biased score descending and
+    ties broken toward the lower expert id.
+    """
+    s = sigmoid(gate_logits(x, gate_w))
+    score = s + np.asarray(bias, np.float32).astype(np.float64)
+    # stable sort of -score: equal scores keep ascending expert id
+    order = np.argsort(-score, axis=1, kind="stable")
+    ids = order[:, :k].astype(np.int32)
+    sel = np.take_along_axis(s, ids, axis=1)
+    gates = sel / np.sum(sel, axis=1, keepdims=True)
+    return ids, gates, s, score
+
+
+def expert_counts(ids: np.ndarray, n_experts: int) -> np.ndarray:
+    """c_i = number of tokens of this batch that selected expert i
+    ([Dissection] section III "Measure per-expert load this step")."""
+    return np.bincount(np.asarray(ids).ravel(), minlength=n_experts).astype(np.int32)
+
+
+def permutation(ids: np.ndarray, n_experts: int):
+    """Expert-major order of the (token, slot) pairs: expert ascending, then
+    token ascending. Every pair is kept (no token dropping, [Explained]
+    recipe step 5).
+
+    Returns offsets int32 [N+1] (exclusive scan of the counts), tokens int32
+    [T*K] (token of each position), rank int32 [T,K] (position of pair
+    (t, k) inside its expert's segment).
+    """
+    ids = np.asarray(ids)
+    t_count, k = ids.shape
+    counts = expert_counts(ids, n_experts)
+    offsets = np.zeros(n_experts + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    tokens = np.empty(t_count * k, dtype=np.int32)
+    rank = np.empty((t_count, k), dtype=np.int32)
+    fill = np.zeros(n_experts, dtype=np.int64)
+    for t in range(t_count):
+        for j in range(k):
+            e = ids[t, j]
+            tokens[offsets[e] + fill[e]] = t
+            rank[t, j] = fill[e]
+            fill[e] += 1
+    return offsets.astype(np.int32), tokens, rank
+
+
+# ---------------------------------------------------------------------------
+# Bias controller ([Dissection] section III "How the bias is set";
+# [Explained] recipe step 4: overloaded b_i -= gamma, underloaded b_i += gamma)
+# ---------------------------------------------------------------------------
+
+def update_bias(bias: np.ndarray, counts: np.ndarray, t_count: int, k: int,
+                gamma: float) -> np.ndarray:
+    """b_i <- fp32(b_i + gamma * sign(mean load - c_i)).
+
+    The mean load T*K/N is compared without division: sign(T*K - N*c_i).
+    Exactly at the mean the bias does not move. float32 arithmetic, as the
+    bias is stored.
+    """
+    bias = np.asarray(bias, np.float32)
+    n = bias.shape[0]
+    delta = np.sign(np.int64(t_count) * np.int64(k)
+                    - np.int64(n) * np.asarray(counts, np.int64))
+    step = (delta.astype(np.float32) * np.float32(gamma)).astype(np.float32)
+    return (bias + step).astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# Expert FFN (SwiGLU) and the combine ([Explained] recipe step 3 and the
+# note on K_r and the shared expert; [Dissection] section II, DeepSeekMoE)
+# ---------------------------------------------------------------------------
+
+def silu(a: np.ndarray) -> np.ndarray:
+    return a / (1.0 + np.exp(-a))
+
+
+def expert_ffn_q(xq: np.ndarray, xs: np.ndarray, wg_deq: np.ndarray,
+                 wu_deq: np.ndarray, wd_deq: np.ndarray):
+    """Quantisation-faithful expert FFN for a set of rows.
+
+    xq/xs: 1x128 codes and scales of the rows' input. w*_deq: float64
+    dequantised weights, gate [I,H], up [I,H], down [H,I].
+    h = silu(x_hat W_gate^T) * (x_hat W_up^T) in float64, re-quantised 1x128
+    from its float32 rounding, then Y = h_hat W_down^T in float64.
+    Returns (Y float64 [rows,H], hq uint8 [rows,I], hs float32 [rows,I/128]).
+    """
+    x_hat = dequantize_1x128(xq, xs)
+    g = x_hat @ wg_deq.T
+    u = x_hat @ wu_deq.T
+    h = silu(g) * u
+    hq, hs = quantize_1x128(h.astype(np.float32))
+    y = dequantize_1x128(hq, hs) @ wd_deq.T
+    return y, hq, hs
+
+
+def expert_ffn_r(x: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray):
+    """Unquantised float64 expert FFN (used only to measure FP8 error)."""
+    x = np.asarray(x, np.float64)
+    h = silu(x @ np.asarray(wg, np.float64).T) * (x @ np.asarray(wu, np.float64).T)
+    return h @ np.asarray(wd, np.float64).T
+
+
+def combine(y_shared: np.ndarray, y_routed: np.ndarray, ids: np.ndarray,
+            gates: np.ndarray) -> np.ndarray:
+    """y_t = FFN_shared(u_t) + sum_k g_{t,k} FFN_{id_k}(u_t).
+
+    y_routed[t, k] is expert ids[t, k]'s output for token t. Summed in
+    float64, shared first, then slots by ascending expert id.
+    """
+    out = np.array(y_shared, dtype=np.float64, copy=True)
+    order = np.argsort(ids, axis=1, kind="stable")
+    for t in range(out.shape[0]):
+        for j in order[t]:
+            out[t] += gates[t, j] * y_routed[t, j]
+    return out
+
+
+class ExpertWeights:
+    """Per-expert weights assembled from a pool of 128x128 blocks.
+
+    pool13/pool2: float32 blocks [P, 128, 128]; slot_gate/slot_up: [E, I/128,
+    H/128] pool indices; slot_down: [E, H/128, I/128]. Expert E-1 is the
+    shared expert. The oracle quantises the pool itself (128x128 blocks, so a
+    block of the pool is a block of the weight matrix).
+    """
+
+    def __init__(self, pool13, pool2, slot_gate, slot_up, slot_down):
+        self.pool13 = np.asarray(pool13, np.float32)
+        self.pool2 = np.asarray(pool2, np.float32)
+        self.slot_gate = np.asarray(slot_gate)
+        self.slot_up = np.asarray(slot_up)
+        self.slot_down = np.asarray(slot_down)
+        self._q13 = None
+        self._q2 = None
+
+    def _quantised_pools(self):
+        if self._q13 is None:
+            p = self.pool13.shape[0]
+            c13, s13 = quantize_128x128(self.pool13.reshape(p * TILE, TILE))
+            self._q13 = (c13.reshape(p, TILE, TILE), s13.reshape(p))
+            p = self.pool2.shape[0]
+            c2, s2 = quantize_128x128(self.pool2.reshape(p * TILE, TILE))
+            self._q2 = (c2.reshape(p, TILE, TILE), s2.reshape(p))
+        return self._q13, self._q2
+
+    def quantised_pools(self):
+        """((codes13 [P,128,128], scales13 [P]), (codes2, scales2))."""
+        return self._quantised_pools()
+
+    @staticmethod
+    def _assemble(blocks: np.ndarray, slots: np.ndarray) -> np.ndarray:
+        nb, kb = slots.shape
+        m = blocks[slots]  # [nb, kb, 128, 128]
+        return m.transpose(0, 2, 1, 3).reshape(nb * TILE, kb * TILE)
+
+    def dequantised(self, e: int):
+        """(gate [I,H], up [I,H], down [H,I]) float64, dequantised."""
+        (c13, s13), (c2, s2) = self._quantised_pools()
+        d13 = e4m3_decode(c13) / s13.astype(np.float64)[:, None, None]
+        d2 = e4m3_decode(c2) / s2.astype(np.float64)[:, None, None]
+        return (self._assemble(d13, self.slot_gate[e]),
+                self._assemble(d13, self.slot_up[e]),
+                self._assemble(d2, self.slot_down[e]))
+
+    def master(self, e: int):
+        """(gate, up, down) float32 master weights, unquantised."""
+        return (self._assemble(self.pool13, self.slot_gate[e]),
+                self._assemble(self.pool13, self.slot_up[e]),
+                self._assemble(self.pool2, self.slot_down[e]))
+
+
+def moe_forward(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int,
+                weights: ExpertWeights, mode: str = "Q", tokens=None,
+                ids=None):
+    """The MoE layer output for the rows `tokens` (all rows if None).
+
+    mode "Q": quantisation-faithful (1x128 x, 128x128 weights, 1x128 h).
+    mode "R": unquantised float64 reference (bf16 x and fp32 weights taken
+    exactly), used only to measure the FP8 error.
+    Routing always covers every token (the counts need them); `ids`, when
+    given, replaces the routing decision (used for near-tie tokens) and the
+    gates are recomputed from the unbiased affinities of those ids.
+    Returns dict with y [len(tokens), H] float64, ids, gates, counts.
+    """
+    x = np.asarray(x, np.float32)
+    t_count, h = x.shape
+    n = gate_w.shape[0]
+    r_ids, r_gates, s, _ = route(x, gate_w, bias, k)
+    if ids is None:
+        ids = r_ids
+        gates = r_gates
+    else:
+        ids = np.asarray(ids, np.int32)
+        sel = np.take_along_axis(s, ids, axis=1)
+        gates = sel / np.sum(sel, axis=1, keepdims=True)
+    counts = expert_counts(ids, n)
+    if tokens is None:
+        tokens = np.arange(t_count)
+    tokens = np.asarray(tokens)
+    xs_rows = x[tokens]
+    if mode == "Q":
+        xq, xsc = quantize_1x128(xs_rows)
+    y_routed = np.zeros((len(tokens), k, h), dtype=np.float64)
+    sub_ids = ids[tokens]
+    for e in np.unique(sub_ids):
+        rr, kk = np.nonzero(sub_ids == e)
+        if mode == "Q":
+            wg, wu, wd = weights.dequantised(int(e))
+            y_e, _, _ = expert_ffn_q(xq[rr], xsc[rr], wg, wu, wd)
+        else:
+            wg, wu, wd = weights.master(int(e))
+            y_e = expert_ffn_r(xs_rows[rr], wg, wu, wd)
+        y_routed[rr, kk] = y_e
+    shared = n  # expert index of the shared expert
+    if mode == "Q":
+        wg, wu, wd = weights.dequantised(shared)
+        y_shared, _, _ = expert_ffn_q(xq, xsc, wg, wu, wd)
+    else:
+        wg, wu, wd = weights.master(shared)
+        y_shared = expert_ffn_r(xs_rows, wg, wu, wd)
+    y = combine(y_shared, y_routed, sub_ids, gates[tokens])
+    return {"y": y, "ids": ids, "gates": gates, "counts": counts, "s": s}
