@@ -1,0 +1,232 @@
+/*
+ * moe_capi.h — C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ *
+ * The layer (sources: "DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing,
+ * Multi-Token Prediction, and FP8 Training at 671B Scale", trishampatil.com,
+ * section III "The mechanism" and "How the bias is set", section V "Four
+ * details"; "DeepSeek-V3, explained", vibeengines.com, recipe steps 3, 4, 5
+ * and 7; "DeepSeek-V3 Technical Report", deepforge.srivtx.xyz, "Per-tile FP8
+ * scaling"):
+ *
+ *   s[t,i]  = sigmoid(x_t . e_i)                          sigmoid affinity
+ *   ids_t   = TopK_i(s[t,i] + b_i, K)                     bias only selects
+ *   g[t,k]  = s[t,ids_k] / sum_k s[t,ids_k]               unbiased gates
+ *   y_t     = FFN_shared(x_t) + sum_k g[t,k] FFN_{ids_k}(x_t)
+ *   FFN(u)  = W_down (silu(W_gate u) * (W_up u))          SwiGLU, FP8 E4M3:
+ *             u and h in 1x128 tiles, weights in 128x128 blocks, fp32 sums
+ *   b_i    <- b_i + gamma * sign(T*K/N - c_i)             per step, c_i = load
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, row-major, owned by the caller;
+ *     the library never allocates or frees device memory.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
+ *     enqueued asynchronously; no call synchronises except moe_get_status.
+ *   - Return value: MOE_OK or a negative moe_status. Argument errors are
+ *     detected on the host before anything is enqueued. A launch failure
+ *     returns MOE_ERR_CUDA. Errors found on the device (a count or index
+ *     that fails its check, a bounded wait that gave up) are recorded in the
+ *     status word at the start of the workspace, read by moe_get_status;
+ *     device code never traps.
+ *   - bf16 tensors are passed as `const void*` holding IEEE bfloat16.
+ *   - E4M3 tensors hold OCP E4M3FN bytes (bias 7, max 448, NaN 0x7F).
+ *   - Scales are the multipliers 448 / amax (dequantised = code / scale).
+ *   - NaN or Inf in the layer input is outside the contract.
+ */
+#ifndef MOE_CAPI_H
+#define MOE_CAPI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_SHAPE = -1,      /* a size outside the supported range */
+  MOE_ERR_NULL = -2,       /* a required pointer is NULL */
+  MOE_ERR_CUDA = -3,       /* a CUDA call or kernel launch failed */
+  MOE_ERR_TIMEOUT = -4,    /* device status: a bounded wait gave up */
+  MOE_ERR_BOUNDS = -5,     /* device status: a count or index check failed */
+  MOE_ERR_WORKSPACE = -6,  /* workspace too small */
+  MOE_ERR_ALIGN = -7       /* a pointer is not aligned as required */
+} moe_status;
+
+/*
+ * Layer sizes. T tokens, H hidden, N routed experts, K routed experts per
+ * token, I intermediate size of every expert (routed and shared: the shared
+ * expert has the routed experts' shape, "DeepSeek-V3, explained", step 3).
+ * Supported: T >= 1; H a multiple of 256; I a multiple of 128; N a multiple
+ * of 16 with 16 <= N <= 1024; 1 <= K <= min(N, 16).
+ */
+typedef struct {
+  int32_t T, H, N, K, I;
+} moe_shape;
+
+/*
+ * Layer weights (device, caller-owned). Group N (the last) is the shared
+ * expert; groups 0..N-1 are the routed experts.
+ *   gate_w [N, H]              float32 centroids e_i (gating stays in high
+ *                              precision: "DeepSeek-V3, explained", step 7)
+ *   w13    [N+1, 2I, H]        E4M3: for each 128-channel block c of the
+ *                              intermediate size, 128 rows of W_gate
+ *                              (channels 128c..128c+127) then the 128 rows
+ *                              of W_up for the same channels
+ *   s13    [N+1, 2I/128, H/128] float32 block scales of w13 (same row order)
+ *   w2     [N+1, H, I]         E4M3 W_down
+ *   s2     [N+1, H/128, I/128] float32 block scales of w2
+ * w13 and w2 must be 16-byte aligned.
+ */
+typedef struct {
+  const float* gate_w;
+  const uint8_t* w13;
+  const float* s13;
+  const uint8_t* w2;
+  const float* s2;
+} moe_weights;
+
+/*
+ * Byte offsets of the intermediates inside the forward workspace, for
+ * inspection by tests and tools after moe_forward has completed. Rows of the
+ * expert GEMMs ("GEMM rows") are laid out expert-major: routed expert e owns
+ * rows [row_start[e], row_start[e] + counts[e]), row_start 128-aligned and
+ * increasing in e; the shared expert owns rows [routed_cap, routed_cap + T)
+ * in token order. Rows between segments are padding and hold no data.
+ */
+typedef struct {
+  int64_t routed_cap;   /* first GEMM row of the shared expert (multiple of 128) */
+  int64_t rows_total;   /* GEMM rows allocated (routed_cap + T rounded to 128) */
+  size_t status;        /* uint32 status word (also at offset 0) */
+  size_t counts;        /* int32 [N]: tokens routed to each expert (c_i) */
+  size_t offsets;       /* int32 [N+1]: exclusive scan of counts */
+  size_t group_rows;    /* int32 [N+1]: rows of each GEMM group (counts, then T) */
+  size_t row_start;     /* int32 [N+1]: first GEMM row of each group */
+  size_t row_token;     /* int32 [routed_cap]: token of each routed row, -1 on padding */
+  size_t token_row;     /* int32 [T, K]: GEMM row of (token t, slot k) */
+  size_t topk_ids;      /* int32 [T, K] (used when the caller passes none) */
+  size_t topk_gates;    /* float [T, K] (used when the caller passes none) */
+  size_t logits;        /* float [T, N] gate logits x . e_i */
+  size_t a_q;           /* E4M3 [rows_total, H]: GEMM1 input rows; x_q in the shared rows */
+  size_t a_s;           /* float [rows_total, H/128] */
+  size_t h_q;           /* E4M3 [rows_total, I]: SwiGLU output, 1x128 re-quantised */
+  size_t h_s;           /* float [rows_total, I/128] */
+  size_t y_rows;        /* bf16 [rows_total, H]: expert outputs before the combine */
+  size_t total;         /* workspace bytes required */
+} moe_ws_layout;
+
+/*
+ * Online 1x128 activation quantisation ("DeepSeek-V3 Technical Report",
+ * deepforge.srivtx.xyz, "Per-tile FP8 scaling"; "DeepSeek-V3, explained",
+ * step 7). For each row r and 128-column tile j:
+ *   amax = max |x[r, 128j .. 128j+127]|,  scale = fp32(448 / amax) (1 if 0),
+ *   q[r, c] = e4m3_rne_satfinite(fp32(x[r, c] * scale)).
+ * x: bf16 [rows, cols]; q: uint8 [rows, cols]; scales: float [rows, cols/128].
+ * cols must be a positive multiple of 128; x and q 16-byte aligned.
+ */
+int moe_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales,
+                       void* stream);
+
+/*
+ * 128x128 weight block quantisation (same pages, same rule per block), for
+ * preparing w13/w2 once at set-up. w: float [rows, cols]; q: uint8 [rows,
+ * cols]; scales: float [rows/128, cols/128]. rows and cols positive multiples
+ * of 128; w and q 16-byte aligned.
+ */
+int moe_quantize_128x128(const float* w, int64_t rows, int64_t cols, uint8_t* q, float* scales,
+                         void* stream);
+
+/* Workspace bytes needed by moe_route / moe_forward for `sh` (0 if invalid). */
+size_t moe_workspace_size(moe_shape sh);
+
+/* Fills *out with the workspace layout for `sh`. */
+int moe_workspace_layout(moe_shape sh, moe_ws_layout* out);
+
+/*
+ * Routing ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing, ...",
+ * section III equations for s, g' and g). Computes the fp32 gate logits,
+ * sigmoid affinities, top-K of s + b (ties to the lower expert id; output
+ * order biased score descending), the gates normalised from the unbiased
+ * affinities, and the per-expert counts.
+ *   gate_w: float [N, H]; x: bf16 [T, H]; bias: float [N]
+ *   topk_ids: int32 [T, K]; topk_gates: float [T, K]; counts: int32 [N]
+ *   ws: workspace of at least moe_workspace_size(sh) bytes, 256-byte aligned.
+ */
+int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bias,
+              int32_t* topk_ids, float* topk_gates, int32_t* counts, void* ws, size_t ws_bytes,
+              void* stream);
+
+/*
+ * The whole layer forward: quantise x (1x128), route, permute token rows by
+ * expert (expert ascending, token ascending; no token dropped), grouped FP8
+ * SwiGLU expert FFNs for the routed experts and the shared expert, and the
+ * weighted combine y_t = Y_shared[t] + sum_k g[t,k] Y[row(t,k)] accumulated in
+ * fp32 (shared first, then slots by ascending expert id) and rounded once to
+ * bf16. No residual is added.
+ *   w: weights (see moe_weights); x: bf16 [T, H]; bias: float [N]
+ *   y: bf16 [T, H], 16-byte aligned
+ *   topk_ids_opt, topk_gates_opt, counts_opt: optional outputs (may be NULL),
+ *   shapes as in moe_route; counts_opt feeds moe_update_bias.
+ *   ws: workspace of at least moe_workspace_size(sh) bytes, 256-byte aligned;
+ *   its contents are valid until the next call that uses it.
+ */
+int moe_forward(moe_shape sh, const moe_weights* w, const void* x, const float* bias, void* y,
+                int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt, void* ws,
+                size_t ws_bytes, void* stream);
+
+/*
+ * Aux-loss-free bias controller ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load
+ * Balancing, ...", section III "How the bias is set"; "DeepSeek-V3,
+ * explained", step 4): b_i <- fp32(b_i + gamma * sign(T*K - N*c_i)), i.e. an
+ * overloaded expert loses gamma, an underloaded one gains gamma, one exactly
+ * at the mean load T*K/N keeps its bias. bias: float [N], updated in place;
+ * counts: int32 [N]. gamma = 0 leaves the bias unchanged.
+ */
+int moe_update_bias(float* bias, const int32_t* counts, int32_t N, int32_t T, int32_t K,
+                    float gamma, void* stream);
+
+/*
+ * Stage entry points: the grouped FP8 expert GEMMs alone, on caller-laid-out
+ * rows ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing, ...", section
+ * V "Four details", items 1-2: E4M3 operands, one scale per 1x128 activation
+ * tile and 128x128 weight block, partial sums promoted to fp32 every 128
+ * products). Group g (0 <= g < n_groups) uses weight set g and owns GEMM rows
+ * [group_start[g], group_start[g] + group_rows[g]); group_start must be
+ * multiples of 128, the segments must not overlap and must lie inside
+ * [0, rows). group_rows and group_start are DEVICE int32 arrays [n_groups].
+ * status_ws: a device uint32 status word (may be the forward workspace).
+ *
+ * moe_expert_up: per group, G = A_hat W_gate^T, U = A_hat W_up^T in fp32,
+ *   h = silu(G) * U, h re-quantised 1x128.
+ *   a_q [rows, H] E4M3, a_s [rows, H/128]; w13/s13 as in moe_weights with
+ *   n_groups sets; h_q [rows, I] E4M3, h_s [rows, I/128].
+ * moe_expert_down: per group, Y = h_hat W_down^T, rounded to bf16.
+ *   h_q/h_s as above; w2/s2 as in moe_weights; y_rows bf16 [rows, H].
+ * Rows outside every segment are not written.
+ */
+int moe_expert_up(int32_t H, int32_t I, int32_t n_groups, const int32_t* group_rows,
+                  const int32_t* group_start, int64_t rows, const uint8_t* a_q, const float* a_s,
+                  const uint8_t* w13, const float* s13, uint8_t* h_q, float* h_s,
+                  uint32_t* status_ws, void* stream);
+
+int moe_expert_down(int32_t H, int32_t I, int32_t n_groups, const int32_t* group_rows,
+                    const int32_t* group_start, int64_t rows, const uint8_t* h_q,
+                    const float* h_s, const uint8_t* w2, const float* s2, void* y_rows,
+                    uint32_t* status_ws, void* stream);
+
+/*
+ * Synchronises `stream`, reads and clears the device status word at the
+ * start of `ws` (a forward workspace or a bare uint32 status word). Returns
+ * MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_BOUNDS (timeout reported first), or
+ * MOE_ERR_CUDA if the stream reports an error.
+ */
+int moe_get_status(void* ws, void* stream);
+
+/* Number of streaming multiprocessors of the current device (0 on error). */
+int moe_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_CAPI_H */

@@ -1,0 +1,187 @@
+"""ctypes binding of the C ABI in include/moe_capi.h (libmoe_b200.so).
+
+Argument marshalling only: every function takes torch tensors (device
+memory), checks dtype / contiguity / device, and passes raw pointers, sizes
+and the current CUDA stream to the library function of the same name. No
+computation happens here, and there is no fallback: if the library is
+missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_SHAPE", -2: "MOE_ERR_NULL", -3: "MOE_ERR_CUDA",
+                -4: "MOE_ERR_TIMEOUT", -5: "MOE_ERR_BOUNDS", -6: "MOE_ERR_WORKSPACE",
+                -7: "MOE_ERR_ALIGN"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("K", ctypes.c_int32), ("I", ctypes.c_int32)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [("gate_w", ctypes.c_void_p), ("w13", ctypes.c_void_p), ("s13", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("s2", ctypes.c_void_p)]
+
+
+_LAYOUT_FIELDS = ["status", "counts", "offsets", "group_rows", "row_start", "row_token",
+                  "token_row", "topk_ids", "topk_gates", "logits", "a_q", "a_s", "h_q", "h_s",
+                  "y_rows", "total"]
+
+
+class moe_ws_layout(ctypes.Structure):
+    _fields_ = ([("routed_cap", ctypes.c_int64), ("rows_total", ctypes.c_int64)]
+                + [(f, ctypes.c_size_t) for f in _LAYOUT_FIELDS])
+
+
+# name -> (restype, argtypes) of every function declared in the header
+_P = ctypes.c_void_p
+_I32, _I64, _F32, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "moe_quantize_1x128": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "moe_quantize_128x128": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "moe_workspace_size": (_SZ, [moe_shape]),
+    "moe_workspace_layout": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_ws_layout)]),
+    "moe_route": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_forward": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P, _P, _P,
+                                   _P, _SZ, _P]),
+    "moe_update_bias": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _F32, _P]),
+    "moe_expert_up": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_expert_down": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_get_status": (ctypes.c_int, [_P, _P]),
+    "moe_device_sm_count": (ctypes.c_int, []),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_40_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+def _check(name: str, code: int) -> None:
+    if code != MOE_OK:
+        raise MoeError(name, code)
+
+
+def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, name: str = "tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def shape_of(T: int, H: int, N: int, K: int, I: int) -> moe_shape:
+    return moe_shape(T, H, N, K, I)
+
+
+def moe_quantize_1x128(x: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, stream=None):
+    rows, cols = x.shape
+    _check("moe_quantize_1x128", LIB.moe_quantize_1x128(
+        _ptr(x, torch.bfloat16, "x"), rows, cols, _ptr(q, torch.uint8, "q"),
+        _ptr(scales, torch.float32, "scales"), _stream(stream)))
+
+
+def moe_quantize_128x128(w: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, stream=None):
+    rows, cols = w.shape
+    _check("moe_quantize_128x128", LIB.moe_quantize_128x128(
+        _ptr(w, torch.float32, "w"), rows, cols, _ptr(q, torch.uint8, "q"),
+        _ptr(scales, torch.float32, "scales"), _stream(stream)))
+
+
+def moe_workspace_size(sh: moe_shape) -> int:
+    return int(LIB.moe_workspace_size(sh))
+
+
+def moe_workspace_layout(sh: moe_shape) -> moe_ws_layout:
+    out = moe_ws_layout()
+    _check("moe_workspace_layout", LIB.moe_workspace_layout(sh, ctypes.byref(out)))
+    return out
+
+
+def moe_route(sh: moe_shape, gate_w, x, bias, topk_ids, topk_gates, counts, ws, stream=None):
+    _check("moe_route", LIB.moe_route(
+        sh, _ptr(gate_w, torch.float32, "gate_w"), _ptr(x, torch.bfloat16, "x"),
+        _ptr(bias, torch.float32, "bias"), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def make_weights(gate_w, w13, s13, w2, s2) -> moe_weights:
+    return moe_weights(_ptr(gate_w, torch.float32, "gate_w"), _ptr(w13, torch.uint8, "w13"),
+                       _ptr(s13, torch.float32, "s13"), _ptr(w2, torch.uint8, "w2"),
+                       _ptr(s2, torch.float32, "s2"))
+
+
+def moe_forward(sh: moe_shape, w: moe_weights, x, bias, y, topk_ids=None, topk_gates=None,
+                counts=None, ws=None, stream=None):
+    _check("moe_forward", LIB.moe_forward(
+        sh, ctypes.byref(w), _ptr(x, torch.bfloat16, "x"), _ptr(bias, torch.float32, "bias"),
+        _ptr(y, torch.bfloat16, "y"), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_update_bias(bias, counts, N: int, T: int, K: int, gamma: float, stream=None):
+    _check("moe_update_bias", LIB.moe_update_bias(
+        _ptr(bias, torch.float32, "bias"), _ptr(counts, torch.int32, "counts"), N, T, K,
+        float(gamma), _stream(stream)))
+
+
+def moe_expert_up(H, I, n_groups, group_rows, group_start, rows, a_q, a_s, w13, s13, h_q, h_s,
+                  status, stream=None):
+    _check("moe_expert_up", LIB.moe_expert_up(
+        H, I, n_groups, _ptr(group_rows, torch.int32), _ptr(group_start, torch.int32), rows,
+        _ptr(a_q, torch.uint8), _ptr(a_s, torch.float32), _ptr(w13, torch.uint8),
+        _ptr(s13, torch.float32), _ptr(h_q, torch.uint8), _ptr(h_s, torch.float32),
+        _ptr(status), _stream(stream)))
+
+
+def moe_expert_down(H, I, n_groups, group_rows, group_start, rows, h_q, h_s, w2, s2, y_rows,
+                    status, stream=None):
+    _check("moe_expert_down", LIB.moe_expert_down(
+        H, I, n_groups, _ptr(group_rows, torch.int32), _ptr(group_start, torch.int32), rows,
+        _ptr(h_q, torch.uint8), _ptr(h_s, torch.float32), _ptr(w2, torch.uint8),
+        _ptr(s2, torch.float32), _ptr(y_rows, torch.bfloat16), _ptr(status), _stream(stream)))
+
+
+def moe_get_status(ws, stream=None) -> int:
+    return int(LIB.moe_get_status(_ptr(ws), _stream(stream)))
+
+
+def moe_device_sm_count() -> int:
+    return int(LIB.moe_device_sm_count())

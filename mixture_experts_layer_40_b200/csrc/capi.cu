@@ -1,0 +1,274 @@
+// C ABI entry points (declared in include/moe_capi.h): argument checks,
+// workspace layout, tensor maps, and the launch sequence of the forward.
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+  });
+  return fn;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool shape_ok(const moe_shape& s) {
+  return s.T >= 1 && s.H >= 256 && s.H % 256 == 0 && s.I >= 128 && s.I % 128 == 0 && s.N >= 16 &&
+         s.N <= 1024 && s.N % 16 == 0 && s.K >= 1 && s.K <= s.N && s.K <= 16 &&
+         (int64_t)s.T * s.K < (1ll << 31) && (int64_t)s.T * s.N < (1ll << 31);
+}
+
+void layout_of(const moe_shape& s, moe_ws_layout* L) {
+  const int64_t T = s.T, H = s.H, N = s.N, K = s.K, I = s.I;
+  L->routed_cap = round_up(T * K + N * (kTile - 1), kTile);
+  L->rows_total = L->routed_cap + round_up(T, kTile);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = (size_t)round_up((int64_t)(off + bytes), 256);
+    return at;
+  };
+  L->status = take(16);
+  L->counts = take(N * 4);
+  L->offsets = take((N + 1) * 4);
+  L->group_rows = take((N + 1) * 4);
+  L->row_start = take((N + 1) * 4);
+  L->row_token = take((size_t)L->routed_cap * 4);
+  L->token_row = take((size_t)(T * K) * 4);
+  L->topk_ids = take((size_t)(T * K) * 4);
+  L->topk_gates = take((size_t)(T * K) * 4);
+  L->logits = take((size_t)(T * N) * 4);
+  L->a_q = take((size_t)L->rows_total * H);
+  L->a_s = take((size_t)L->rows_total * (H / kTile) * 4);
+  L->h_q = take((size_t)L->rows_total * I);
+  L->h_s = take((size_t)L->rows_total * (I / kTile) * 4);
+  L->y_rows = take((size_t)L->rows_total * H * 2);
+  L->total = off;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+
+cudaError_t make_tmap_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
+                         int box_inner, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)(rows > 0 ? rows : 1)};
+  const cuuint64_t strides[1] = {(cuuint64_t)inner};
+  const cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_device_sm_count(void) { return sm_count(); }
+
+int moe_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales,
+                       void* stream) {
+  if (x == nullptr || q == nullptr || scales == nullptr) return MOE_ERR_NULL;
+  if (rows < 0 || cols <= 0 || cols % kTile != 0) return MOE_ERR_SHAPE;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scales, 4)) return MOE_ERR_ALIGN;
+  return cuda_status(launch_quantize_1x128(x, rows, cols, q, scales,
+                                           static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+int moe_quantize_128x128(const float* w, int64_t rows, int64_t cols, uint8_t* q, float* scales,
+                         void* stream) {
+  if (w == nullptr || q == nullptr || scales == nullptr) return MOE_ERR_NULL;
+  if (rows <= 0 || cols <= 0 || rows % kTile != 0 || cols % kTile != 0) return MOE_ERR_SHAPE;
+  if (rows / kTile > 65535) return MOE_ERR_SHAPE;
+  if (!aligned(w, 16) || !aligned(q, 16) || !aligned(scales, 4)) return MOE_ERR_ALIGN;
+  return cuda_status(
+      launch_quantize_128x128(w, rows, cols, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_workspace_size(moe_shape sh) {
+  if (!shape_ok(sh)) return 0;
+  moe_ws_layout L;
+  layout_of(sh, &L);
+  return L.total;
+}
+
+int moe_workspace_layout(moe_shape sh, moe_ws_layout* out) {
+  if (out == nullptr) return MOE_ERR_NULL;
+  if (!shape_ok(sh)) return MOE_ERR_SHAPE;
+  layout_of(sh, out);
+  return MOE_OK;
+}
+
+int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bias,
+              int32_t* topk_ids, float* topk_gates, int32_t* counts, void* ws, size_t ws_bytes,
+              void* stream) {
+  if (!shape_ok(sh)) return MOE_ERR_SHAPE;
+  if (!gate_w || !x || !bias || !topk_ids || !topk_gates || !counts || !ws) return MOE_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(gate_w, 16) || !aligned(ws, 256)) return MOE_ERR_ALIGN;
+  moe_ws_layout L;
+  layout_of(sh, &L);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
+  if (e == cudaSuccess)
+    e = launch_router(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, at<float>(ws, L.logits), topk_ids,
+                      topk_gates, counts, status, s, sm_count());
+  return cuda_status(e);
+}
+
+int moe_forward(moe_shape sh, const moe_weights* w, const void* x, const float* bias, void* y,
+                int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt, void* ws,
+                size_t ws_bytes, void* stream) {
+  if (!shape_ok(sh)) return MOE_ERR_SHAPE;
+  if (!w || !x || !bias || !y || !ws) return MOE_ERR_NULL;
+  if (!w->gate_w || !w->w13 || !w->s13 || !w->w2 || !w->s2) return MOE_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(w->gate_w, 16) || !aligned(w->w13, 16) ||
+      !aligned(w->w2, 16) || !aligned(ws, 256))
+    return MOE_ERR_ALIGN;
+  moe_ws_layout L;
+  layout_of(sh, &L);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = sm_count();
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  int32_t* ids = topk_ids_opt ? topk_ids_opt : at<int32_t>(ws, L.topk_ids);
+  float* gates = topk_gates_opt ? topk_gates_opt : at<float>(ws, L.topk_gates);
+  int32_t* counts = counts_opt ? counts_opt : at<int32_t>(ws, L.counts);
+  uint8_t* a_q = at<uint8_t>(ws, L.a_q);
+  float* a_s = at<float>(ws, L.a_s);
+  const int64_t H = sh.H, I = sh.I;
+
+  cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
+  // a1: x -> 1x128 codes and scales, written into the shared-expert GEMM rows
+  if (e == cudaSuccess)
+    e = launch_quantize_1x128(x, sh.T, H, a_q + L.routed_cap * H, a_s + L.routed_cap * (H / kTile),
+                              s, sms);
+  // a2-a5: gate logits, sigmoid, biased top-K, gates, counts
+  if (e == cudaSuccess)
+    e = launch_router(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K, at<float>(ws, L.logits), ids,
+                      gates, counts, status, s, sms);
+  // a6-a7: offsets, stable expert-major scatter, gather of the quantised rows
+  if (e == cudaSuccess)
+    e = launch_permute(ids, counts, sh.T, sh.N, sh.K, sh.H, L.routed_cap,
+                       at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.group_rows),
+                       at<int32_t>(ws, L.row_start), at<int32_t>(ws, L.row_token),
+                       at<int32_t>(ws, L.token_row), a_q, a_s, status, s, sms);
+  GroupedGemm gg{sh.H, sh.I, sh.N + 1, at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
+                 L.rows_total, status};
+  // a8: up/gate GEMM + SwiGLU + 1x128 re-quantisation
+  if (e == cudaSuccess)
+    e = launch_expert_up(gg, a_q, a_s, w->w13, w->s13, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s),
+                         s, sms);
+  // a9: down GEMM -> bf16 expert outputs
+  if (e == cudaSuccess)
+    e = launch_expert_down(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w->w2, w->s2,
+                           at<__nv_bfloat16>(ws, L.y_rows), s, sms);
+  // a10: weighted combine with the shared expert
+  if (e == cudaSuccess)
+    e = launch_combine(at<__nv_bfloat16>(ws, L.y_rows), ids, gates, at<int32_t>(ws, L.token_row),
+                       sh.T, sh.H, sh.K, L.routed_cap, L.rows_total,
+                       static_cast<__nv_bfloat16*>(y), status, s);
+  (void)I;
+  return cuda_status(e);
+}
+
+int moe_update_bias(float* bias, const int32_t* counts, int32_t N, int32_t T, int32_t K,
+                    float gamma, void* stream) {
+  if (!bias || !counts) return MOE_ERR_NULL;
+  if (N < 1 || T < 0 || K < 1) return MOE_ERR_SHAPE;
+  return cuda_status(launch_update_bias(bias, counts, N, T, K, gamma, static_cast<cudaStream_t>(stream)));
+}
+
+static int expert_args_ok(int32_t H, int32_t I, int32_t n_groups, const int32_t* gr,
+                          const int32_t* gs, int64_t rows) {
+  if (H < 256 || H % 256 != 0 || I < 128 || I % 128 != 0) return MOE_ERR_SHAPE;
+  if (n_groups < 1 || n_groups > 1025 || rows < 0 || rows >= (1ll << 31)) return MOE_ERR_SHAPE;
+  if (!gr || !gs) return MOE_ERR_NULL;
+  return MOE_OK;
+}
+
+int moe_expert_up(int32_t H, int32_t I, int32_t n_groups, const int32_t* group_rows,
+                  const int32_t* group_start, int64_t rows, const uint8_t* a_q, const float* a_s,
+                  const uint8_t* w13, const float* s13, uint8_t* h_q, float* h_s,
+                  uint32_t* status_ws, void* stream) {
+  const int r = expert_args_ok(H, I, n_groups, group_rows, group_start, rows);
+  if (r != MOE_OK) return r;
+  if (!a_q || !a_s || !w13 || !s13 || !h_q || !h_s) return MOE_ERR_NULL;
+  if (!aligned(a_q, 16) || !aligned(w13, 16) || !aligned(h_q, 16)) return MOE_ERR_ALIGN;
+  GroupedGemm gg{H, I, n_groups, group_rows, group_start, rows, status_ws};
+  return cuda_status(launch_expert_up(gg, a_q, a_s, w13, s13, h_q, h_s,
+                                      static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+int moe_expert_down(int32_t H, int32_t I, int32_t n_groups, const int32_t* group_rows,
+                    const int32_t* group_start, int64_t rows, const uint8_t* h_q,
+                    const float* h_s, const uint8_t* w2, const float* s2, void* y_rows,
+                    uint32_t* status_ws, void* stream) {
+  const int r = expert_args_ok(H, I, n_groups, group_rows, group_start, rows);
+  if (r != MOE_OK) return r;
+  if (!h_q || !h_s || !w2 || !s2 || !y_rows) return MOE_ERR_NULL;
+  if (!aligned(h_q, 16) || !aligned(w2, 16) || !aligned(y_rows, 16)) return MOE_ERR_ALIGN;
+  GroupedGemm gg{H, I, n_groups, group_rows, group_start, rows, status_ws};
+  return cuda_status(launch_expert_down(gg, h_q, h_s, w2, s2, static_cast<__nv_bfloat16*>(y_rows),
+                                        static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+int moe_get_status(void* ws, void* stream) {
+  if (!ws) return MOE_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(ws, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word & kStatusTimeout) return MOE_ERR_TIMEOUT;
+  if (word & kStatusBounds) return MOE_ERR_BOUNDS;
+  return MOE_OK;
+}
+
+}  // extern "C"

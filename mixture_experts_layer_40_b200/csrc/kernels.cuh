@@ -1,0 +1,56 @@
+// Launchers of the MoE kernels (each defined in its own .cu file) and the
+// host helpers they share.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Rows of the grouped expert GEMMs (see moe_expert_up / moe_expert_down).
+struct GroupedGemm {
+  int32_t H, I, n_groups;
+  const int32_t* group_rows;   // device [n_groups]
+  const int32_t* group_start;  // device [n_groups]
+  int64_t rows;
+  uint32_t* status;
+};
+
+// 2-D uint8 tensor map over a row-major [rows, inner] buffer, box of
+// box_inner bytes x box_rows rows, 128-byte swizzle (host side).
+cudaError_t make_tmap_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
+                         int box_inner, int box_rows);
+
+cudaError_t launch_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q,
+                                  float* scales, cudaStream_t stream, int sm_count);
+cudaError_t launch_quantize_128x128(const float* w, int64_t rows, int64_t cols, uint8_t* q,
+                                    float* scales, cudaStream_t stream);
+
+// Router: gate logits (fp32 SIMT GEMM), then sigmoid, biased top-K, gates and
+// counts (counts must be zero on entry).
+cudaError_t launch_router(const void* x, const float* gate_w, const float* bias, int T, int H,
+                          int N, int K, float* logits, int32_t* ids, float* gates, int32_t* counts,
+                          uint32_t* status, cudaStream_t stream, int sm_count);
+
+// Permutation: scan of counts into group tables, stable scatter, row gather.
+cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K, int H,
+                           int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
+                           int32_t* row_start, int32_t* row_token, int32_t* token_row,
+                           uint8_t* a_q, float* a_s, uint32_t* status, cudaStream_t stream,
+                           int sm_count);
+
+cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const float* a_s,
+                             const uint8_t* w13, const float* s13, uint8_t* h_q, float* h_s,
+                             cudaStream_t stream, int sm_count);
+cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const float* h_s,
+                               const uint8_t* w2, const float* s2, __nv_bfloat16* y,
+                               cudaStream_t stream, int sm_count);
+
+cudaError_t launch_combine(const __nv_bfloat16* y_rows, const int32_t* ids, const float* gates,
+                           const int32_t* token_row, int T, int H, int K, int64_t routed_cap,
+                           int64_t rows_total, __nv_bfloat16* y, uint32_t* status,
+                           cudaStream_t stream);
+
+cudaError_t launch_update_bias(float* bias, const int32_t* counts, int N, int T, int K,
+                               float gamma, cudaStream_t stream);
+
+}  // namespace moe

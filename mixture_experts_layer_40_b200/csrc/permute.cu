@@ -1,0 +1,190 @@
+// Token permutation by expert. Every (token, slot) pair is kept ("no tokens
+// are dropped in training or at inference": "DeepSeek-V3, explained", recipe
+// step 5) and placed expert-major, tokens ascending inside each expert, so the
+// order is unique and the scatter needs no atomics on output positions.
+//   scan    : counts -> offsets, GEMM group rows and 128-aligned row starts
+//   scatter : one CTA per expert compacts the tokens that chose it, in token
+//             order, with a block-wide prefix sum over ballots
+//   gather  : copies the quantised input row (codes + scales) of each routed
+//             GEMM row from the shared-expert rows, where the quantiser put it
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+// Block-wide exclusive prefix sum of a 0/1 flag over up to 1024 threads.
+// Returns this thread's prefix; *total receives the block sum.
+MOE_DEV int block_scan_flag(bool flag, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const uint32_t ballot = __ballot_sync(0xffffffffu, flag);
+  const int in_warp = __popc(ballot & ((1u << lane) - 1u));
+  if (lane == 0) warp_sums[warp] = __popc(ballot);
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < nwarps ? warp_sums[lane] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane < nwarps) warp_sums[lane] = incl - v;
+    if (lane == 31) warp_sums[32] = incl;
+  }
+  __syncthreads();
+  const int res = warp_sums[warp] + in_warp;
+  *total = warp_sums[32];
+  __syncthreads();
+  return res;
+}
+
+// Exclusive scan of v over the block (up to 1024 threads, one value each).
+MOE_DEV int block_scan_int(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nwarps ? warp_sums[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    if (lane < nwarps) warp_sums[lane] = wi - w;
+    if (lane == 31) warp_sums[32] = wi;
+  }
+  __syncthreads();
+  const int res = warp_sums[warp] + incl - v;
+  *total = warp_sums[32];
+  __syncthreads();
+  return res;
+}
+
+// One CTA of 1024 threads; N <= 1024.
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ counts, int N,
+                                                    int T, int K, int64_t routed_cap,
+                                                    int32_t* __restrict__ offsets,
+                                                    int32_t* __restrict__ group_rows,
+                                                    int32_t* __restrict__ row_start,
+                                                    uint32_t* __restrict__ status) {
+  __shared__ int sums[33];
+  const int e = threadIdx.x;
+  const int c = e < N ? counts[e] : 0;
+  const int padded = (c + kTile - 1) / kTile * kTile;
+  int total_c, total_p;
+  const int off = block_scan_int(c, sums, &total_c);
+  const int start = block_scan_int(padded, sums, &total_p);
+  if (e < N) {
+    offsets[e] = off;
+    group_rows[e] = c;
+    row_start[e] = start;
+  }
+  if (e == 0) {
+    offsets[N] = total_c;
+    group_rows[N] = T;
+    row_start[N] = (int32_t)routed_cap;
+    if ((int64_t)total_c != (int64_t)T * K || (int64_t)total_p > routed_cap) {
+      flag_status(status, kStatusBounds);
+    }
+  }
+}
+
+// One CTA (1024 threads) per routed expert e: walks the tokens in order and
+// writes the GEMM rows of the pairs (t, k) with ids[t, k] == e.
+__global__ void __launch_bounds__(1024) scatter_kernel(const int32_t* __restrict__ ids, int T, int K,
+                                                       const int32_t* __restrict__ group_rows,
+                                                       const int32_t* __restrict__ row_start,
+                                                       int64_t routed_cap,
+                                                       int32_t* __restrict__ row_token,
+                                                       int32_t* __restrict__ token_row,
+                                                       uint32_t* __restrict__ status) {
+  __shared__ int sums[33];
+  const int e = blockIdx.x;
+  const int base = row_start[e];
+  const int count = group_rows[e];
+  int running = 0;
+  for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+    const int t = t0 + threadIdx.x;
+    int slot = -1;
+    if (t < T) {
+      for (int k = 0; k < K; ++k)
+        if (__ldg(ids + (int64_t)t * K + k) == e) slot = k;
+    }
+    int total;
+    const int pos = block_scan_flag(slot >= 0, sums, &total);
+    if (slot >= 0) {
+      const int64_t r = (int64_t)base + running + pos;
+      if (running + pos < count && r < routed_cap) {
+        row_token[r] = t;
+        token_row[(int64_t)t * K + slot] = (int32_t)r;
+      } else {
+        flag_status(status, kStatusBounds);
+      }
+    }
+    running += total;
+  }
+  if (threadIdx.x == 0 && running != count) flag_status(status, kStatusBounds);
+}
+
+// One warp per routed GEMM row: copies H code bytes and H/128 scales of the
+// token's quantised input (stored in the shared-expert rows) into the row.
+__global__ void __launch_bounds__(256) gather_kernel(const int32_t* __restrict__ row_token,
+                                                     int64_t routed_cap, int T, int H,
+                                                     uint8_t* __restrict__ a_q,
+                                                     float* __restrict__ a_s,
+                                                     uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int vec = H / 16;
+  const int nsc = H / kTile;
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < routed_cap;
+       r += warps) {
+    const int t = __ldg(row_token + r);
+    if (t < 0) continue;
+    if (t >= T) {
+      if (lane == 0) flag_status(status, kStatusBounds);
+      continue;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a_q + (routed_cap + t) * (int64_t)H);
+    uint4* dst = reinterpret_cast<uint4*>(a_q + r * (int64_t)H);
+    for (int i = lane; i < vec; i += 32) dst[i] = __ldg(src + i);
+    const float* ss = a_s + (routed_cap + t) * (int64_t)nsc;
+    float* ds = a_s + r * (int64_t)nsc;
+    for (int i = lane; i < nsc; i += 32) ds[i] = __ldg(ss + i);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K, int H,
+                           int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
+                           int32_t* row_start, int32_t* row_token, int32_t* token_row,
+                           uint8_t* a_q, float* a_s, uint32_t* status, cudaStream_t stream,
+                           int sm_count) {
+  scan_kernel<<<1, 1024, 0, stream>>>(counts, N, T, K, routed_cap, offsets, group_rows, row_start,
+                                      status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(row_token, 0xFF, (size_t)routed_cap * sizeof(int32_t), stream);
+  if (e != cudaSuccess) return e;
+  scatter_kernel<<<N, 1024, 0, stream>>>(ids, T, K, group_rows, row_start, routed_cap, row_token,
+                                         token_row, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int64_t blocks = (routed_cap + 7) / 8;
+  if (blocks > (int64_t)sm_count * 8) blocks = (int64_t)sm_count * 8;
+  gather_kernel<<<(unsigned)blocks, 256, 0, stream>>>(row_token, routed_cap, T, H, a_q, a_s, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,98 @@
+// FP8 E4M3 fine-grained quantisers: 1x128 activation tiles (online) and
+// 128x128 weight blocks (set-up). Rule of "DeepSeek-V3 Technical Report"
+// (deepforge.srivtx.xyz), "Per-tile FP8 scaling": scale = 448 / amax,
+// code = round_to_e4m3(x * scale).
+#include "kernels.cuh"
+
+namespace moe {
+
+// One 128-column tile per 16 threads; each thread owns 8 consecutive bf16
+// (one 128-bit load) and writes 8 codes (one 64-bit store). HBM-bound: reads
+// 2 bytes and writes 1 byte per element plus 4 bytes per 128 elements.
+__global__ void __launch_bounds__(256) quantize_1x128_kernel(const uint4* __restrict__ x,
+                                                             int64_t n_tiles,
+                                                             uint2* __restrict__ q,
+                                                             float* __restrict__ scales) {
+  const int sub = threadIdx.x & 15;
+  // the whole CTA iterates together so that every shuffle is warp-convergent
+  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_tiles; base += (int64_t)gridDim.x * 16) {
+    const int64_t tile = base + (threadIdx.x >> 4);
+    const bool live = tile < n_tiles;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (live) v = __ldcs(x + tile * 16 + sub);
+    float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                  bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = tile_scale(amax);
+    if (live) {
+      uint2 out;
+      out.x = e4m3x4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
+      out.y = e4m3x4(__fmul_rn(f[4], s), __fmul_rn(f[5], s), __fmul_rn(f[6], s), __fmul_rn(f[7], s));
+      q[tile * 16 + sub] = out;
+      if (sub == 0) scales[tile] = s;
+    }
+  }
+}
+
+// One CTA per 128x128 block: 256 threads hold 16 float4 each in registers,
+// reduce the block amax through shared memory, then write the codes.
+__global__ void __launch_bounds__(256) quantize_128x128_kernel(const float4* __restrict__ w,
+                                                               int64_t cols, int64_t col_blocks,
+                                                               uint32_t* __restrict__ q,
+                                                               float* __restrict__ scales) {
+  __shared__ float red[8];
+  const int64_t rb = blockIdx.y, cb = blockIdx.x;
+  const int64_t cols4 = cols >> 2;
+  float4 v[16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int f = threadIdx.x + 256 * i;  // float4 index inside the block
+    const int r = f >> 5, c4 = f & 31;
+    v[i] = __ldcs(w + (rb * kTile + r) * cols4 + cb * 32 + c4);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float s = tile_scale(amax);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int f = threadIdx.x + 256 * i;
+    const int r = f >> 5, c4 = f & 31;
+    q[(rb * kTile + r) * cols4 + cb * 32 + c4] =
+        e4m3x4(__fmul_rn(v[i].x, s), __fmul_rn(v[i].y, s), __fmul_rn(v[i].z, s), __fmul_rn(v[i].w, s));
+  }
+  if (threadIdx.x == 0) scales[rb * col_blocks + cb] = s;
+}
+
+cudaError_t launch_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q,
+                                  float* scales, cudaStream_t stream, int sm_count) {
+  const int64_t n_tiles = rows * (cols / kTile);
+  if (n_tiles == 0) return cudaSuccess;
+  int64_t blocks = (n_tiles + 15) / 16;
+  const int64_t cap = (int64_t)sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  quantize_1x128_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(x), n_tiles, reinterpret_cast<uint2*>(q), scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_128x128(const float* w, int64_t rows, int64_t cols, uint8_t* q,
+                                    float* scales, cudaStream_t stream) {
+  dim3 grid((unsigned)(cols / kTile), (unsigned)(rows / kTile));
+  quantize_128x128_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(w), cols,
+                                                    cols / kTile, reinterpret_cast<uint32_t*>(q),
+                                                    scales);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,113 @@
+"""A thin holder for one MoE layer on the GPU: shape, device weights and the
+workspace, with methods that call the C ABI. All compute is in the CUDA
+library; this module only owns memory and forwards pointers.
+
+Also builds a workload's device weights from its block pool: the pool is
+quantised on the GPU by moe_quantize_128x128 and the code/scale blocks are
+placed into the ABI layout (w13 interleaves W_gate and W_up per 128 rows) by
+indexing, which moves bytes and computes nothing.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+from . import capi
+from .inputs import WeightPool, Workload
+
+
+@dataclasses.dataclass
+class DeviceWeights:
+    gate_w: torch.Tensor  # [N, H] float32
+    w13: torch.Tensor     # [E, 2I, H] uint8
+    s13: torch.Tensor     # [E, 2I/128, H/128] float32
+    w2: torch.Tensor      # [E, H, I] uint8
+    s2: torch.Tensor      # [E, H/128, I/128] float32
+
+
+def quantise_pool(pool: np.ndarray, device) -> tuple[torch.Tensor, torch.Tensor]:
+    """[P,128,128] float32 blocks -> codes [P,128,128] uint8, scales [P]."""
+    p = pool.shape[0]
+    w = torch.from_numpy(np.ascontiguousarray(pool.reshape(p * 128, 128))).to(device)
+    q = torch.empty((p * 128, 128), dtype=torch.uint8, device=device)
+    s = torch.empty((p, 1), dtype=torch.float32, device=device)
+    capi.moe_quantize_128x128(w, q, s)
+    return q.view(p, 128, 128), s.view(p)
+
+
+def _place(codes: torch.Tensor, scales: torch.Tensor, slots: np.ndarray, out_q: torch.Tensor,
+           out_s: torch.Tensor, chunk: int = 16) -> None:
+    """out_q[e] = block matrix of codes[slots[e]]; out_s[e] = scales[slots[e]]."""
+    e_total, rb, cb = slots.shape
+    idx_all = torch.from_numpy(np.ascontiguousarray(slots)).to(codes.device)
+    for e0 in range(0, e_total, chunk):
+        idx = idx_all[e0:e0 + chunk]
+        blocks = codes[idx]  # [e, rb, cb, 128, 128]
+        out_q[e0:e0 + chunk] = blocks.permute(0, 1, 3, 2, 4).reshape(idx.shape[0], rb * 128, cb * 128)
+        out_s[e0:e0 + chunk] = scales[idx]
+
+
+def device_weights(w: Workload, pool: WeightPool, gate_w: np.ndarray, device) -> DeviceWeights:
+    q13, s13p = quantise_pool(pool.pool13, device)
+    q2, s2p = quantise_pool(pool.pool2, device)
+    e, ib, hb = w.E, w.I // 128, w.H // 128
+    # row-block order of w13: gate block c, then up block c, for c = 0 .. I/128-1
+    slots13 = np.stack([pool.slot_gate, pool.slot_up], axis=2).reshape(e, 2 * ib, hb)
+    w13 = torch.empty((e, 2 * w.I, w.H), dtype=torch.uint8, device=device)
+    s13 = torch.empty((e, 2 * ib, hb), dtype=torch.float32, device=device)
+    _place(q13, s13p, slots13, w13, s13)
+    w2 = torch.empty((e, w.H, w.I), dtype=torch.uint8, device=device)
+    s2 = torch.empty((e, hb, ib), dtype=torch.float32, device=device)
+    _place(q2, s2p, pool.slot_down, w2, s2)
+    del q13, s13p, q2, s2p
+    gw = torch.from_numpy(np.ascontiguousarray(gate_w, dtype=np.float32)).to(device)
+    return DeviceWeights(gw, w13, s13, w2, s2)
+
+
+class MoELayer:
+    """One layer: forward(x, bias) -> y through moe_forward."""
+
+    def __init__(self, T: int, H: int, N: int, K: int, I: int, weights: DeviceWeights,
+                 device="cuda"):
+        self.T, self.H, self.N, self.K, self.I = T, H, N, K, I
+        self.shape = capi.shape_of(T, H, N, K, I)
+        nbytes = capi.moe_workspace_size(self.shape)
+        if nbytes == 0:
+            raise ValueError(f"unsupported shape T={T} H={H} N={N} K={K} I={I}")
+        self.device = torch.device(device)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.ws[:16].zero_()
+        self.weights = weights
+        self._cw = capi.make_weights(weights.gate_w, weights.w13, weights.s13, weights.w2,
+                                     weights.s2)
+        self.layout = capi.moe_workspace_layout(self.shape)
+        self.ids = torch.empty((T, K), dtype=torch.int32, device=self.device)
+        self.gates = torch.empty((T, K), dtype=torch.float32, device=self.device)
+        self.counts = torch.empty((N,), dtype=torch.int32, device=self.device)
+
+    def forward(self, x: torch.Tensor, bias: torch.Tensor, y: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+        if y is None:
+            y = torch.empty((self.T, self.H), dtype=torch.bfloat16, device=self.device)
+        capi.moe_forward(self.shape, self._cw, x, bias, y, self.ids, self.gates, self.counts,
+                         self.ws, stream)
+        return y
+
+    def route(self, x: torch.Tensor, bias: torch.Tensor, stream=None):
+        capi.moe_route(self.shape, self.weights.gate_w, x, bias, self.ids, self.gates,
+                       self.counts, self.ws, stream)
+        return self.ids, self.gates, self.counts
+
+    def update_bias(self, bias: torch.Tensor, gamma: float, stream=None) -> None:
+        capi.moe_update_bias(bias, self.counts, self.N, self.T, self.K, gamma, stream)
+
+    def status(self, stream=None) -> int:
+        return capi.moe_get_status(self.ws, stream)
+
+    def view(self, name: str, dtype: torch.dtype, shape) -> torch.Tensor:
+        """A workspace intermediate (see moe_ws_layout) as a tensor view."""
+        off = getattr(self.layout, name)
+        n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+        return self.ws[off:off + n].view(dtype).view(*shape)

@@ -1,0 +1,74 @@
+"""CPU checks of the C ABI library: it loads without a GPU, exports every
+function that include/moe_capi.h declares, and rejects bad arguments on the
+host (before any device work) with the documented codes."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from __graft_entry__ import ROOT, build
+
+HEADER = os.path.join(ROOT, "include", "moe_capi.h")
+
+
+@pytest.fixture(scope="module")
+def capi():
+    build()
+    from mixture_experts_layer_40_b200 import capi as c
+    return c
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for required in ["moe_quantize_1x128", "moe_route", "moe_forward", "moe_update_bias",
+                     "moe_workspace_size", "moe_get_status"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(capi):
+    lib = ctypes.CDLL(capi.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(declared_functions()) == set(capi.SIGNATURES)
+
+
+def test_workspace_layout(capi):
+    sh = capi.shape_of(4096, 7168, 256, 8, 2048)
+    L = capi.moe_workspace_layout(sh)
+    assert L.routed_cap % 128 == 0 and L.routed_cap >= 4096 * 8 + 256 * 127
+    assert L.rows_total == L.routed_cap + 4096
+    offs = [getattr(L, f) for f in capi._LAYOUT_FIELDS]
+    assert all(o % 256 == 0 for o in offs)
+    assert offs == sorted(offs) and L.total == capi.moe_workspace_size(sh)
+    assert L.y_rows + L.rows_total * 7168 * 2 <= L.total
+
+
+@pytest.mark.parametrize("shape", [(0, 256, 16, 4, 128), (64, 200, 16, 4, 128), (64, 256, 16, 4, 100),
+                                   (64, 256, 15, 4, 128), (64, 256, 16, 17, 128), (64, 256, 16, 0, 128),
+                                   (64, 128, 16, 4, 128), (64, 256, 2048, 4, 128)])
+def test_bad_shapes_rejected(capi, shape):
+    sh = capi.shape_of(*shape)
+    assert capi.moe_workspace_size(sh) == 0
+    w = capi.moe_weights(1, 1, 1, 1, 1)
+    rc = capi.LIB.moe_forward(sh, ctypes.byref(w), 16, 16, 16, None, None, None, 256, 1 << 30, None)
+    assert rc == -1  # MOE_ERR_SHAPE
+
+
+def test_null_and_alignment_rejected(capi):
+    sh = capi.shape_of(64, 256, 16, 4, 128)
+    w = capi.moe_weights(16, 16, 16, 16, 16)
+    assert capi.LIB.moe_forward(sh, ctypes.byref(w), None, 16, 16, None, None, None, 256, 1 << 30, None) == -2
+    assert capi.LIB.moe_forward(sh, ctypes.byref(w), 16, 16, 16, None, None, None, 128, 1 << 30, None) == -7
+    assert capi.LIB.moe_forward(sh, ctypes.byref(w), 16, 16, 16, None, None, None, 256, 1024, None) == -6
+    assert capi.LIB.moe_quantize_1x128(16, 4, 100, 16, 16, None) == -1
+    assert capi.LIB.moe_quantize_1x128(8, 4, 128, 16, 16, None) == -7
+    assert capi.LIB.moe_quantize_128x128(16, 100, 128, 16, 16, None) == -1
+    assert capi.LIB.moe_update_bias(None, 16, 16, 4, 2, 0.001, None) == -2
+    assert capi.LIB.moe_expert_up(256, 128, 0, 16, 16, 128, 16, 16, 16, 16, 16, 16, None, None) == -1
