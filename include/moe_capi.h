@@ -122,7 +122,8 @@ typedef struct {
  *   amax = max |x[r, 128j .. 128j+127]|,  scale = fp32(448 / amax) (1 if 0),
  *   q[r, c] = e4m3_rne_satfinite(fp32(x[r, c] * scale)).
  * x: bf16 [rows, cols]; q: uint8 [rows, cols]; scales: float [rows, cols/128].
- * cols must be a positive multiple of 128; x and q 16-byte aligned.
+ * cols must be a positive multiple of 128; x and q 16-byte aligned. rows = 0
+ * is a no-op (the pointers may then be NULL).
  */
 int moe_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales,
                        void* stream);

@@ -111,8 +111,9 @@ int moe_device_sm_count(void) { return sm_count(); }
 
 int moe_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales,
                        void* stream) {
-  if (x == nullptr || q == nullptr || scales == nullptr) return MOE_ERR_NULL;
   if (rows < 0 || cols <= 0 || cols % kTile != 0) return MOE_ERR_SHAPE;
+  if (rows == 0) return MOE_OK;  // nothing to do; empty tensors may carry NULL
+  if (x == nullptr || q == nullptr || scales == nullptr) return MOE_ERR_NULL;
   if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scales, 4)) return MOE_ERR_ALIGN;
   return cuda_status(launch_quantize_1x128(x, rows, cols, q, scales,
                                            static_cast<cudaStream_t>(stream), sm_count()));

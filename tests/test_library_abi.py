@@ -68,6 +68,8 @@ def test_null_and_alignment_rejected(capi):
     assert capi.LIB.moe_forward(sh, ctypes.byref(w), 16, 16, 16, None, None, None, 128, 1 << 30, None) == -7
     assert capi.LIB.moe_forward(sh, ctypes.byref(w), 16, 16, 16, None, None, None, 256, 1024, None) == -6
     assert capi.LIB.moe_quantize_1x128(16, 4, 100, 16, 16, None) == -1
+    assert capi.LIB.moe_quantize_1x128(None, 0, 128, None, None, None) == 0
+    assert capi.LIB.moe_quantize_1x128(None, 2, 128, None, None, None) == -2
     assert capi.LIB.moe_quantize_1x128(8, 4, 128, 16, 16, None) == -7
     assert capi.LIB.moe_quantize_128x128(16, 100, 128, 16, 16, None) == -1
     assert capi.LIB.moe_update_bias(None, 16, 16, 4, 2, 0.001, None) == -2
