@@ -1,0 +1,422 @@
+"""Benchmark of the MoE layer forward (plus the per-step bias update) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3_prefill]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step = one pass of the whole hot path on one batch of synthetic input:
+quantise x, route, permute, up/gate GEMM + SwiGLU + re-quantisation, down
+GEMM, combine, and the aux-loss-free bias update. With N > 1 ranks (torchrun,
+one GPU each) every rank runs its own batch (weak scaling) and the per-expert
+counts are summed across ranks (NCCL all-reduce of N int32) before the bias
+update, since the controller balances the whole batch.
+
+Rank 0 prints one JSON line. `value` is tokens per second of the whole job
+with inputs resident in HBM; `e2e` is the same through the public API with
+the input copied from pinned host memory and the output copied back inside
+the timed region. `--impl reference` times the CPU oracle instead (a bounded
+sample of the same workload per step, scaled to the whole layer).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and grouped-GEMM FP8 TFLOP/s (% of B200 dense FP8 peak)"
+FP8_SPEC_TFLOPS = 4500.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="v3_prefill")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-fp8-peak", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.strip()]
+        os.unlink(self.out.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload
+
+def algorithmic_work(w, counts: np.ndarray):
+    """Bytes and FLOPs each expert GEMM launch must move / compute."""
+    rows = w.T * w.K + w.T
+    touched = int(np.count_nonzero(counts)) + 1  # + the shared expert
+    hb, ib = w.H // 128, w.I // 128
+    w13_bytes = touched * (2 * w.I * w.H + 2 * ib * hb * 4)
+    w2_bytes = touched * (w.H * w.I + hb * ib * 4)
+    a_bytes = rows * (w.H + hb * 4)
+    h_bytes = rows * (w.I + ib * 4)
+    y_bytes = rows * w.H * 2
+    return {
+        "expert_up": {"bytes": w13_bytes + a_bytes + h_bytes, "flops": 2.0 * rows * w.H * 2 * w.I},
+        "expert_down": {"bytes": w2_bytes + h_bytes + y_bytes, "flops": 2.0 * rows * w.I * w.H},
+        "quantize": {"bytes": w.T * w.H * 3 + w.T * hb * 4, "flops": 0.0},
+        "combine": {"bytes": (w.T * w.K + w.T) * w.H * 2 + w.T * w.H * 2, "flops": 0.0},
+        "permute": {"bytes": 2 * w.T * w.K * (w.H + hb * 4), "flops": 0.0},
+        "route": {"bytes": w.T * w.H * 2 + w.N * w.H * 4, "flops": 2.0 * w.T * w.N * w.H},
+    }
+
+
+def measure_fp8_peak(torch, device):
+    """Dense FP8 E4M3 GEMM throughput of the vendor library (torch._scaled_mm,
+    8192^3, per-tensor scales): the measured denominator for the FP8 fraction."""
+    n = 8192
+    a = torch.randn(n, n, device=device).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=device).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=device)
+    for _ in range(3):
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(10):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e.record()
+        e.synchronize()
+        best = min(best, s.elapsed_time(e))
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample_step(w, x, gate_w, bias, ew, step: int, groups: int = 2, shared_rows: int = 64):
+    """One bounded sample of the layer on the CPU oracle; returns the time
+    scaled to the whole layer (all T tokens, all N + 1 expert groups)."""
+    from oracle import moe_oracle as O
+    t0 = time.perf_counter()
+    xq, xs = O.quantize_1x128(x)
+    t_quant = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    ids, gates, _, _ = O.route(x, gate_w, bias, w.K)
+    O.permutation(ids, w.N)
+    t_route = time.perf_counter() - t0
+    y_routed = np.zeros((w.T, w.K, w.H))
+    t0 = time.perf_counter()
+    for j in range(groups):
+        e = (step * groups + j) % w.N
+        rr, kk = np.nonzero(ids == e)
+        if len(rr):
+            y_routed[rr, kk] = O.expert_ffn_q(xq[rr], xs[rr], *ew.dequantised(e))[0]
+    t_groups = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    r0 = (step * shared_rows) % max(1, w.T - shared_rows + 1)
+    rows = slice(r0, r0 + shared_rows)
+    y_shared = np.zeros((w.T, w.H))
+    y_shared[rows] = O.expert_ffn_q(xq[rows], xs[rows], *ew.dequantised(w.N))[0]
+    t_shared = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.combine(y_shared, y_routed, ids, gates)
+    t_combine = time.perf_counter() - t0
+    return (t_quant + t_route + t_combine + t_groups * w.N / groups
+            + t_shared * w.T / min(shared_rows, w.T))
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_setup(w, x_bits):
+    from mixture_experts_layer_40_b200 import inputs as I
+    from oracle import moe_oracle as O
+    pool = I.make_weight_pool(w)
+    ew = O.ExpertWeights(pool.pool13, pool.pool2, pool.slot_gate, pool.slot_up, pool.slot_down)
+    ew.quantised_pools()
+    return I.bf16_bits_to_f32(x_bits), I.make_gate_w(w), I.make_bias(w), ew
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    from mixture_experts_layer_40_b200 import inputs as I
+    x, gate_w, bias, ew = oracle_setup(w, I.make_x(w))
+    for s in range(args.warmup):
+        oracle_sample_step(w, x, gate_w, bias, ew, s)
+    times = [oracle_sample_step(w, x, gate_w, bias, ew, args.warmup + s) for s in range(args.steps)]
+    ms = 1e3 * float(np.mean(times))
+    value = w.T / (ms * 1e-3)
+    sample = (f"per step: the whole layer's routing, quantisation and combine on all {w.T} tokens, "
+              f"2 of {w.N} routed expert groups with all their tokens and the shared expert on 64 "
+              f"tokens; group and shared time scaled to all groups and tokens")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"{w.name}: T={w.T} H={w.H} N={w.N} K={w.K} I={w.I}"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from __graft_entry__ import build
+    build()
+    from mixture_experts_layer_40_b200 import capi
+    from mixture_experts_layer_40_b200 import inputs as I
+    from mixture_experts_layer_40_b200.layer import MoELayer, device_weights
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wr = dataclasses.replace(w, seed=w.seed + rank)  # own batch per rank
+    x_bits = I.make_x(wr)
+    pool = I.make_weight_pool(w)   # same weights on every rank
+    gate_w = I.make_gate_w(w)
+    bias0 = I.make_bias(w)
+    layer = MoELayer(w.T, w.H, w.N, w.K, w.I, device_weights(w, pool, gate_w, dev), dev)
+    del pool
+    x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    x = x_host.to(dev)
+    y = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+    y_host = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
+    bias = torch.from_numpy(bias0).to(dev)
+    stream = torch.cuda.current_stream()
+    t_total = w.T * world
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(capi.TRACE_EVENTS)]
+              for _ in range(args.steps)]
+    for evs in events:
+        for ev in evs:
+            ev.record(stream)
+    launches_per_step = 10  # quantise, logits, top-K, scan, scatter, gather, up, down, combine, bias
+
+    def step(traced_events=None, x_in=x):
+        if traced_events is None:
+            capi.moe_forward(layer.shape, layer._cw, x_in, bias, y, layer.ids, layer.gates,
+                             layer.counts, layer.ws)
+        else:
+            capi.moe_forward_traced(layer.shape, layer._cw, x_in, bias, y, traced_events,
+                                    layer.ids, layer.gates, layer.counts, layer.ws)
+        if world > 1:
+            dist.all_reduce(layer.counts)
+        capi.moe_update_bias(bias, layer.counts, w.N, t_total, w.K, w.gamma)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if layer.status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    # ------------------------------------------------ timed region (HBM-resident inputs)
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(events[k])
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
+    ms_step = ms_total / args.steps
+    stage_ms = {name: float(np.mean([evs[i].elapsed_time(evs[i + 1]) for evs in events]))
+                for i, name in enumerate(capi.TRACE_STAGES)}
+    if layer.status() != 0:
+        raise RuntimeError("device status error in the timed region")
+    counts = layer.counts.cpu().numpy()
+
+    # ------------------------------------------------ end to end (host buffers)
+    for _ in range(2):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    e_end.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    fp8_meas = None
+    if not args.no_fp8_peak:
+        try:
+            fp8_meas = measure_fp8_peak(torch, dev)
+        except Exception:
+            fp8_meas = None
+    work = algorithmic_work(w, counts)
+    dom = max(stage_ms, key=stage_ms.get)
+    gemm_ms = stage_ms["expert_up"] + stage_ms["expert_down"]
+    gemm_tflops = (work["expert_up"]["flops"] + work["expert_down"]["flops"]) / (gemm_ms * 1e-3) / 1e12
+    achieved_gbs = work[dom]["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
+    hbm_peak = float(peaks["hbm_gbs"])
+    value = w.T * world / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: T={w.T} per GPU, H={w.H}, N={w.N} routed top-{w.K} "
+                               f"+ 1 shared, I={w.I}, SwiGLU, FP8 E4M3 1x128/128x128",
+                   "tokens_per_gpu": w.T, "parallelism": f"dp{world} (weak: own batch per GPU)",
+                   "l2": "no flush: each step streams 11.3 GB of weights + ~1.9 GB of "
+                         "activations, 100x the 126 MB L2"},
+        "gemm": {"tflops": gemm_tflops, "fp8_spec_tflops": FP8_SPEC_TFLOPS,
+                 "frac_of_fp8_spec": gemm_tflops / FP8_SPEC_TFLOPS,
+                 "fp8_library_tflops_measured": fp8_meas,
+                 "frac_of_fp8_measured": (gemm_tflops / fp8_meas) if fp8_meas else None},
+        "stages_ms": stage_ms,
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved_gbs / hbm_peak, "traffic": None,
+                     "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                     "algorithmic_bytes": work[dom]["bytes"]},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": w.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2},
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        x32, gw, b0, ew = oracle_setup(w, x_bits)
+        t = [oracle_sample_step(w, x32, gw, b0, ew, s) for s in range(2)]
+        v = w.T / float(np.mean(t))
+        line["cpu_baseline"] = {
+            "value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"2 steps; each: quantisation, routing and combine of all {w.T} tokens, 2 of "
+                      f"{w.N} routed expert groups with all their tokens and the shared expert on "
+                      f"64 tokens, group and shared time scaled to the whole layer"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from mixture_experts_layer_40_b200 import inputs as I
+    w = I.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -176,6 +176,20 @@ int moe_forward(moe_shape sh, const moe_weights* w, const void* x, const float* 
                 size_t ws_bytes, void* stream);
 
 /*
+ * moe_forward with stage timing: identical work and results, and in addition
+ * records events[i] on `stream` before stage i and events[6] after the last:
+ *   0 quantise x, 1 route, 2 permute (scan, scatter, gather),
+ *   3 up/gate GEMM + SwiGLU + re-quantisation, 4 down GEMM, 5 combine.
+ * events: MOE_TRACE_EVENTS cudaEvent_t handles created by the caller
+ * (n_events >= MOE_TRACE_EVENTS, none NULL, else MOE_ERR_NULL).
+ */
+#define MOE_TRACE_EVENTS 7
+int moe_forward_traced(moe_shape sh, const moe_weights* w, const void* x, const float* bias,
+                       void* y, int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
+                       void* ws, size_t ws_bytes, void* stream, void* const* events,
+                       int32_t n_events);
+
+/*
  * Aux-loss-free bias controller ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load
  * Balancing, ...", section III "How the bias is set"; "DeepSeek-V3,
  * explained", step 4): b_i <- fp32(b_i + gamma * sign(T*K - N*c_i)), i.e. an

@@ -59,6 +59,8 @@ SIGNATURES = {
     "moe_route": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_forward": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P, _P, _P,
                                    _P, _SZ, _P]),
+    "moe_forward_traced": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P,
+                                          _P, _P, _P, _SZ, _P, ctypes.POINTER(_P), _I32]),
     "moe_update_bias": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _F32, _P]),
     "moe_expert_up": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_down": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P]),
@@ -154,6 +156,22 @@ def moe_forward(sh: moe_shape, w: moe_weights, x, bias, y, topk_ids=None, topk_g
         _ptr(y, torch.bfloat16, "y"), _ptr(topk_ids, torch.int32, "topk_ids"),
         _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+TRACE_EVENTS = 7
+TRACE_STAGES = ["quantize", "route", "permute", "expert_up", "expert_down", "combine"]
+
+
+def moe_forward_traced(sh: moe_shape, w: moe_weights, x, bias, y, events, topk_ids=None,
+                       topk_gates=None, counts=None, ws=None, stream=None):
+    """moe_forward that also records `events` (TRACE_EVENTS torch.cuda.Event
+    objects created with enable_timing=True) around its six stages."""
+    arr = (_P * len(events))(*[ev.cuda_event for ev in events])
+    _check("moe_forward_traced", LIB.moe_forward_traced(
+        sh, ctypes.byref(w), _ptr(x, torch.bfloat16, "x"), _ptr(bias, torch.float32, "bias"),
+        _ptr(y, torch.bfloat16, "y"), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream), arr, len(events)))
 
 
 def moe_update_bias(bias, counts, N: int, T: int, K: int, gamma: float, stream=None):

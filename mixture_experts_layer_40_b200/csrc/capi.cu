@@ -162,9 +162,9 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
   return cuda_status(e);
 }
 
-int moe_forward(moe_shape sh, const moe_weights* w, const void* x, const float* bias, void* y,
-                int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt, void* ws,
-                size_t ws_bytes, void* stream) {
+static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const float* bias,
+                        void* y, int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
+                        void* ws, size_t ws_bytes, void* stream, void* const* events) {
   if (!shape_ok(sh)) return MOE_ERR_SHAPE;
   if (!w || !x || !bias || !y || !ws) return MOE_ERR_NULL;
   if (!w->gate_w || !w->w13 || !w->s13 || !w->w2 || !w->s2) return MOE_ERR_NULL;
@@ -184,16 +184,25 @@ int moe_forward(moe_shape sh, const moe_weights* w, const void* x, const float* 
   float* a_s = at<float>(ws, L.a_s);
   const int64_t H = sh.H, I = sh.I;
 
-  cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
+  // optional stage events: recorded before each of the 6 stages and at the end
+  auto mark = [&](int i, cudaError_t e) {
+    if (events != nullptr && e == cudaSuccess)
+      return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+    return e;
+  };
+  cudaError_t e = mark(0, cudaSuccess);
+  if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
   // a1: x -> 1x128 codes and scales, written into the shared-expert GEMM rows
   if (e == cudaSuccess)
     e = launch_quantize_1x128(x, sh.T, H, a_q + L.routed_cap * H, a_s + L.routed_cap * (H / kTile),
                               s, sms);
+  e = mark(1, e);
   // a2-a5: gate logits, sigmoid, biased top-K, gates, counts
   if (e == cudaSuccess)
     e = launch_router(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K, at<float>(ws, L.logits), ids,
                       gates, counts, status, s, sms);
+  e = mark(2, e);
   // a6-a7: offsets, stable expert-major scatter, gather of the quantised rows
   if (e == cudaSuccess)
     e = launch_permute(ids, counts, sh.T, sh.N, sh.K, sh.H, L.routed_cap,
@@ -202,22 +211,45 @@ int moe_forward(moe_shape sh, const moe_weights* w, const void* x, const float* 
                        at<int32_t>(ws, L.token_row), a_q, a_s, status, s, sms);
   GroupedGemm gg{sh.H, sh.I, sh.N + 1, at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
                  L.rows_total, status};
+  e = mark(3, e);
   // a8: up/gate GEMM + SwiGLU + 1x128 re-quantisation
   if (e == cudaSuccess)
     e = launch_expert_up(gg, a_q, a_s, w->w13, w->s13, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s),
                          s, sms);
+  e = mark(4, e);
   // a9: down GEMM -> bf16 expert outputs
   if (e == cudaSuccess)
     e = launch_expert_down(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w->w2, w->s2,
                            at<__nv_bfloat16>(ws, L.y_rows), s, sms);
+  e = mark(5, e);
   // a10: weighted combine with the shared expert
   if (e == cudaSuccess)
     e = launch_combine(at<__nv_bfloat16>(ws, L.y_rows), ids, gates, at<int32_t>(ws, L.token_row),
                        sh.T, sh.H, sh.K, L.routed_cap, L.rows_total,
                        static_cast<__nv_bfloat16*>(y), status, s);
+  e = mark(6, e);
   (void)I;
   return cuda_status(e);
 }
+
+int moe_forward(moe_shape sh, const moe_weights* w, const void* x, const float* bias, void* y,
+                int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt, void* ws,
+                size_t ws_bytes, void* stream) {
+  return forward_impl(sh, w, x, bias, y, topk_ids_opt, topk_gates_opt, counts_opt, ws, ws_bytes,
+                      stream, nullptr);
+}
+
+int moe_forward_traced(moe_shape sh, const moe_weights* w, const void* x, const float* bias,
+                       void* y, int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
+                       void* ws, size_t ws_bytes, void* stream, void* const* events,
+                       int32_t n_events) {
+  if (events == nullptr || n_events < MOE_TRACE_EVENTS) return MOE_ERR_NULL;
+  for (int i = 0; i < MOE_TRACE_EVENTS; ++i)
+    if (events[i] == nullptr) return MOE_ERR_NULL;
+  return forward_impl(sh, w, x, bias, y, topk_ids_opt, topk_gates_opt, counts_opt, ws, ws_bytes,
+                      stream, events);
+}
+
 
 int moe_update_bias(float* bias, const int32_t* counts, int32_t N, int32_t T, int32_t K,
                     float gamma, void* stream) {

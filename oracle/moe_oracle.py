@@ -355,9 +355,12 @@ class ExpertWeights:
 
     def dequantised(self, e: int):
         """(gate [I,H], up [I,H], down [H,I]) float64, dequantised."""
-        (c13, s13), (c2, s2) = self._quantised_pools()
-        d13 = e4m3_decode(c13) / s13.astype(np.float64)[:, None, None]
-        d2 = e4m3_decode(c2) / s2.astype(np.float64)[:, None, None]
+        if getattr(self, "_deq", None) is None:
+            # dequantised pool blocks, kept: every expert is assembled from them
+            (c13, s13), (c2, s2) = self._quantised_pools()
+            self._deq = (e4m3_decode(c13) / s13.astype(np.float64)[:, None, None],
+                         e4m3_decode(c2) / s2.astype(np.float64)[:, None, None])
+        d13, d2 = self._deq
         return (self._assemble(d13, self.slot_gate[e]),
                 self._assemble(d13, self.slot_up[e]),
                 self._assemble(d2, self.slot_down[e]))
