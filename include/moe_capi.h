@@ -111,7 +111,7 @@ typedef struct {
   size_t a_s;           /* float [rows_total, H/128] */
   size_t h_q;           /* E4M3 [rows_total, I]: SwiGLU output, 1x128 re-quantised */
   size_t h_s;           /* float [rows_total, I/128] */
-  size_t y_rows;        /* bf16 [rows_total, H]: expert outputs before the combine */
+  size_t y_rows;        /* float [rows_total, H]: expert outputs before the combine */
   size_t total;         /* workspace bytes required */
 } moe_ws_layout;
 
@@ -215,8 +215,9 @@ int moe_update_bias(float* bias, const int32_t* counts, int32_t N, int32_t T, in
  *   h = silu(G) * U, h re-quantised 1x128.
  *   a_q [rows, H] E4M3, a_s [rows, H/128]; w13/s13 as in moe_weights with
  *   n_groups sets; h_q [rows, I] E4M3, h_s [rows, I/128].
- * moe_expert_down: per group, Y = h_hat W_down^T, rounded to bf16.
- *   h_q/h_s as above; w2/s2 as in moe_weights; y_rows bf16 [rows, H].
+ * moe_expert_down: per group, Y = h_hat W_down^T in fp32 (the expert outputs
+ *   stay at accumulation precision until the combine rounds y once to bf16).
+ *   h_q/h_s as above; w2/s2 as in moe_weights; y_rows float [rows, H].
  * Rows outside every segment are not written.
  */
 int moe_expert_up(int32_t H, int32_t I, int32_t n_groups, const int32_t* group_rows,

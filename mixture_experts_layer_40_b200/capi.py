@@ -194,7 +194,7 @@ def moe_expert_down(H, I, n_groups, group_rows, group_start, rows, h_q, h_s, w2,
     _check("moe_expert_down", LIB.moe_expert_down(
         H, I, n_groups, _ptr(group_rows, torch.int32), _ptr(group_start, torch.int32), rows,
         _ptr(h_q, torch.uint8), _ptr(h_s, torch.float32), _ptr(w2, torch.uint8),
-        _ptr(s2, torch.float32), _ptr(y_rows, torch.bfloat16), _ptr(status), _stream(stream)))
+        _ptr(s2, torch.float32), _ptr(y_rows, torch.float32), _ptr(status), _stream(stream)))
 
 
 def moe_get_status(ws, stream=None) -> int:

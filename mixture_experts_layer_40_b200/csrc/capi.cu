@@ -73,7 +73,7 @@ void layout_of(const moe_shape& s, moe_ws_layout* L) {
   L->a_s = take((size_t)L->rows_total * (H / kTile) * 4);
   L->h_q = take((size_t)L->rows_total * I);
   L->h_s = take((size_t)L->rows_total * (I / kTile) * 4);
-  L->y_rows = take((size_t)L->rows_total * H * 2);
+  L->y_rows = take((size_t)L->rows_total * H * 4);
   L->total = off;
 }
 
@@ -220,11 +220,11 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   // a9: down GEMM -> bf16 expert outputs
   if (e == cudaSuccess)
     e = launch_expert_down(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w->w2, w->s2,
-                           at<__nv_bfloat16>(ws, L.y_rows), s, sms);
+                           at<float>(ws, L.y_rows), s, sms);
   e = mark(5, e);
   // a10: weighted combine with the shared expert
   if (e == cudaSuccess)
-    e = launch_combine(at<__nv_bfloat16>(ws, L.y_rows), ids, gates, at<int32_t>(ws, L.token_row),
+    e = launch_combine(at<float>(ws, L.y_rows), ids, gates, at<int32_t>(ws, L.token_row),
                        sh.T, sh.H, sh.K, L.routed_cap, L.rows_total,
                        static_cast<__nv_bfloat16*>(y), status, s);
   e = mark(6, e);
@@ -288,7 +288,7 @@ int moe_expert_down(int32_t H, int32_t I, int32_t n_groups, const int32_t* group
   if (!h_q || !h_s || !w2 || !s2 || !y_rows) return MOE_ERR_NULL;
   if (!aligned(h_q, 16) || !aligned(w2, 16) || !aligned(y_rows, 16)) return MOE_ERR_ALIGN;
   GroupedGemm gg{H, I, n_groups, group_rows, group_start, rows, status_ws};
-  return cuda_status(launch_expert_down(gg, h_q, h_s, w2, s2, static_cast<__nv_bfloat16*>(y_rows),
+  return cuda_status(launch_expert_down(gg, h_q, h_s, w2, s2, static_cast<float*>(y_rows),
                                         static_cast<cudaStream_t>(stream), sm_count()));
 }
 

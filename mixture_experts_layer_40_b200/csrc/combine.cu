@@ -16,7 +16,7 @@ namespace {
 
 constexpr int kMaxK = 16;
 
-__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __restrict__ y_rows,
+__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ y_rows,
                                                       const int32_t* __restrict__ ids,
                                                       const float* __restrict__ gates,
                                                       const int32_t* __restrict__ token_row,
@@ -58,17 +58,16 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
   const int n = s_n;
   const int64_t shared_row = routed_cap + t;
   if (shared_row >= rows_total) return;
-  const uint4* ys = reinterpret_cast<const uint4*>(y_rows + shared_row * H);
+  const float4* ys = reinterpret_cast<const float4*>(y_rows + shared_row * H);
   uint4* out = reinterpret_cast<uint4*>(y + (int64_t)t * H);
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
-    const uint4 v = __ldcs(ys + c);
-    float acc[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                    bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    const float4 v0 = __ldcs(ys + 2 * c), v1 = __ldcs(ys + 2 * c + 1);
+    float acc[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     for (int k = 0; k < n; ++k) {
-      const uint4 u = __ldcs(reinterpret_cast<const uint4*>(y_rows + s_row[k] * H) + c);
+      const float4* yk = reinterpret_cast<const float4*>(y_rows + s_row[k] * H);
+      const float4 u0 = __ldcs(yk + 2 * c), u1 = __ldcs(yk + 2 * c + 1);
       const float g = s_gate[k];
-      const float f[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
-                          bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+      const float f[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, f[i], acc[i]);
     }
@@ -92,7 +91,7 @@ __global__ void update_bias_kernel(float* __restrict__ bias, const int32_t* __re
 
 }  // namespace
 
-cudaError_t launch_combine(const __nv_bfloat16* y_rows, const int32_t* ids, const float* gates,
+cudaError_t launch_combine(const float* y_rows, const int32_t* ids, const float* gates,
                            const int32_t* token_row, int T, int H, int K, int64_t routed_cap,
                            int64_t rows_total, __nv_bfloat16* y, uint32_t* status,
                            cudaStream_t stream) {

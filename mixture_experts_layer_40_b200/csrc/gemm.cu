@@ -65,7 +65,7 @@ struct GemmArgs {
   uint8_t* h_q;           // up: [rows, I]
   float* h_s;             // up: [rows, I / 128]
   int32_t I;
-  __nv_bfloat16* y;       // down: [rows, H]
+  float* y;               // down: [rows, H] fp32
   int32_t H;
   uint32_t* status;
 };
@@ -330,16 +330,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         if (live) {
-          uint4* dst = reinterpret_cast<uint4*>(p.y + grow * p.H + n * kBN + 128 * eg);
+          float4* dst = reinterpret_cast<float4*>(p.y + grow * p.H + n * kBN + 128 * eg);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            uint4 o;
-            o.x = pack_bf16x2(acc[8 * j + 0], acc[8 * j + 1]);
-            o.y = pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]);
-            o.z = pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]);
-            o.w = pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]);
-            dst[j] = o;
-          }
+          for (int j = 0; j < 32; ++j)
+            dst[j] = make_float4(acc[4 * j + 0], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
         }
       }
     }
@@ -403,7 +397,7 @@ cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const fl
 }
 
 cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const float* h_s,
-                               const uint8_t* w2, const float* s2, __nv_bfloat16* y,
+                               const uint8_t* w2, const float* s2, float* y,
                                cudaStream_t stream, int sm_count) {
   CUtensorMap ma, mb;
   cudaError_t e = make_tmap_u8(&ma, h_q, gg.I, gg.rows, kBK, kBM);

@@ -42,10 +42,10 @@ cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const fl
                              const uint8_t* w13, const float* s13, uint8_t* h_q, float* h_s,
                              cudaStream_t stream, int sm_count);
 cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const float* h_s,
-                               const uint8_t* w2, const float* s2, __nv_bfloat16* y,
+                               const uint8_t* w2, const float* s2, float* y,
                                cudaStream_t stream, int sm_count);
 
-cudaError_t launch_combine(const __nv_bfloat16* y_rows, const int32_t* ids, const float* gates,
+cudaError_t launch_combine(const float* y_rows, const int32_t* ids, const float* gates,
                            const int32_t* token_row, int T, int H, int K, int64_t routed_cap,
                            int64_t rows_total, __nv_bfloat16* y, uint32_t* status,
                            cudaStream_t stream);

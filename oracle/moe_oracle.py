@@ -27,9 +27,9 @@ notes with its reason):
   * Top-K ties go to the lower expert id; output order is biased score
     descending.
   * Load target is the mean T*K/N, compared in integers as T*K - N*c_i.
-  * Expert FFN outputs are bf16 (the FP8 GEMMs give BF16 outputs); the
-    combine sums them in float64, shared expert first, then routed experts
-    by ascending id.
+  * Expert FFN outputs stay at full precision; the layer output y is the
+    BF16 result. The combine sums in float64, shared expert first, then
+    routed experts by ascending id.
   * No residual add; no routed scaling factor.
 
 parity pins: every function here is pinned by a test under tests/ against a
@@ -262,15 +262,6 @@ def silu(a: np.ndarray) -> np.ndarray:
     return a / (1.0 + np.exp(-a))
 
 
-def round_bf16(a: np.ndarray) -> np.ndarray:
-    """Round float64 values to bfloat16 (8 significant bits), half to even,
-    in one step from the exact value. Values are assumed far from the bf16
-    overflow and subnormal ranges."""
-    a = np.asarray(a, np.float64)
-    m, e = np.frexp(a)                      # a = m * 2^e, 0.5 <= |m| < 1
-    return np.ldexp(np.round(m * 256.0) / 256.0, e)
-
-
 def expert_ffn_q(xq: np.ndarray, xs: np.ndarray, wg_deq: np.ndarray,
                  wu_deq: np.ndarray, wd_deq: np.ndarray):
     """Quantisation-faithful expert FFN for a set of rows.
@@ -278,18 +269,17 @@ def expert_ffn_q(xq: np.ndarray, xs: np.ndarray, wg_deq: np.ndarray,
     xq/xs: 1x128 codes and scales of the rows' input. w*_deq: float64
     dequantised weights, gate [I,H], up [I,H], down [H,I].
     h = silu(x_hat W_gate^T) * (x_hat W_up^T) in float64, re-quantised 1x128
-    from its float32 rounding, then Y = h_hat W_down^T summed in float64 and
-    rounded to bf16: the FP8 GEMMs take E4M3 inputs, accumulate in FP32 and
-    give BF16 outputs ([Dissection] section V, Figure 6).
-    Returns (Y [rows,H] float64 holding bf16 values, hq uint8 [rows,I],
-    hs float32 [rows,I/128]).
+    from its float32 rounding, then Y = h_hat W_down^T in float64. Y is not
+    rounded: the layer's BF16 output ([Dissection] section V, Figure 6) is y,
+    rounded once after the combine.
+    Returns (Y float64 [rows,H], hq uint8 [rows,I], hs float32 [rows,I/128]).
     """
     x_hat = dequantize_1x128(xq, xs)
     g = x_hat @ wg_deq.T
     u = x_hat @ wu_deq.T
     h = silu(g) * u
     hq, hs = quantize_1x128(h.astype(np.float32))
-    y = round_bf16(dequantize_1x128(hq, hs) @ wd_deq.T)
+    y = dequantize_1x128(hq, hs) @ wd_deq.T
     return y, hq, hs
 
 
