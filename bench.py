@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=40)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default="v3_prefill")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -63,7 +63,7 @@ def load_peaks():
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+    """nvidia-smi samples (every 50 ms) while the timed regions run."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -78,7 +78,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.out, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
@@ -314,7 +314,6 @@ def run_ours(args, w, rank, world, local_rank):
         step(events[k])
     t_end.record(stream)
     barrier()
-    clk = clocks.stop() if clocks else None
     ms_total = max_over_ranks(t_start.elapsed_time(t_end))
     ms_step = ms_total / args.steps
     stage_ms = {name: float(np.mean([evs[i].elapsed_time(evs[i + 1]) for evs in events]))
@@ -338,6 +337,7 @@ def run_ours(args, w, rank, world, local_rank):
         y_host.copy_(y, non_blocking=True)
     e_end.record(stream)
     barrier()
+    clk = clocks.stop() if clocks else None
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
 
     if rank != 0:
