@@ -158,6 +158,32 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
               void* stream);
 
 /*
+ * Routing without a workspace. The pages have no counterpart to this entry
+ * point: it exists for callers that cannot hand the library scratch memory,
+ * such as a host application that owns every device allocation through its
+ * own pool and does not let plug-in libraries allocate, or a latency-critical
+ * loop where a cudaMalloc (which may synchronise the device) is not allowed.
+ *
+ * Same work and outputs as moe_route (same kernels), but the T x N gate
+ * logits live in a fixed array inside the library's device memory: 4 MiB,
+ * MOE_ROUTE_NOALLOC_MAX_LOGITS floats, present on every GPU that loads the
+ * library until the process exits. Nothing is allocated; the caller passes
+ * only inputs and outputs, as for moe_route. Returns MOE_ERR_WORKSPACE, before
+ * enqueuing anything, when T * N exceeds MOE_ROUTE_NOALLOC_MAX_LOGITS.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call uses the same array: calls whose work overlaps on the GPU (other
+ * streams, other host threads on the same device) race on it, so the caller
+ * must serialise them. The logits are fully rewritten by each call and
+ * `counts` is zeroed by the call, so no earlier contents leak into a result.
+ * Device status is not recorded (routing has no device-side checks).
+ */
+#define MOE_ROUTE_NOALLOC_MAX_LOGITS 1048576
+int moe_route_noalloc(moe_shape sh, const float* gate_w, const void* x, const float* bias,
+                      int32_t* topk_ids, float* topk_gates, int32_t* counts, void* stream);
+
+/*
  * The whole layer forward: quantise x (1x128), route, permute token rows by
  * expert (expert ascending, token ascending; no token dropped), grouped FP8
  * SwiGLU expert FFNs for the routed experts and the shared expert, and the

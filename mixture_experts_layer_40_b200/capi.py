@@ -57,6 +57,7 @@ SIGNATURES = {
     "moe_workspace_size": (_SZ, [moe_shape]),
     "moe_workspace_layout": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_ws_layout)]),
     "moe_route": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_route_noalloc": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P, _P, _P,
                                    _P, _SZ, _P]),
     "moe_forward_traced": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P,
@@ -141,6 +142,20 @@ def moe_route(sh: moe_shape, gate_w, x, bias, topk_ids, topk_gates, counts, ws, 
         _ptr(bias, torch.float32, "bias"), _ptr(topk_ids, torch.int32, "topk_ids"),
         _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+ROUTE_NOALLOC_MAX_LOGITS = 1048576
+
+
+def moe_route_noalloc(sh: moe_shape, gate_w, x, bias, topk_ids, topk_gates, counts, stream=None):
+    """moe_route without a workspace: the logits scratch is a fixed 4 MiB array
+    inside the library (T * N <= ROUTE_NOALLOC_MAX_LOGITS). For callers that
+    cannot give the library device memory; calls must not overlap on the GPU."""
+    _check("moe_route_noalloc", LIB.moe_route_noalloc(
+        sh, _ptr(gate_w, torch.float32, "gate_w"), _ptr(x, torch.bfloat16, "x"),
+        _ptr(bias, torch.float32, "bias"), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
+        _stream(stream)))
 
 
 def make_weights(gate_w, w13, s13, w2, s2) -> moe_weights:
