@@ -58,6 +58,11 @@ WORKLOADS = {
                               outlier_scale=20.0, pool13=4096, pool2=2048),
     "decode": Workload("decode", T=128, H=7168, N=256, K=8, I=2048,
                        bias_range=0.05, pool13=4096, pool2=2048),
+    # profiler-sized case: V3 expert shape and ~128 tokens per expert as in
+    # v3_prefill, but 32 routed experts, so 1.45 GB of weights (> L2, small
+    # enough for multi-pass counter captures)
+    "profile_small": Workload("profile_small", T=512, H=7168, N=32, K=8, I=2048,
+                              pool13=4096, pool2=2048),
 }
 
 
