@@ -69,14 +69,11 @@ typedef struct {
  * expert; groups 0..N-1 are the routed experts.
  *   gate_w [N, H]              float32 centroids e_i (gating stays in high
  *                              precision: "DeepSeek-V3, explained", step 7)
- *   w13    [N+1, 2I, H]        E4M3 W_gate and W_up interleaved in 64-row
- *                              pieces: for each 128-channel block c, the
- *                              256 rows are W_gate rows 128c..128c+63,
- *                              W_up rows 128c..128c+63, W_gate rows
- *                              128c+64..128c+127, W_up rows 128c+64..128c+127
- *   s13    [N+1, 2I/128, H/128] float32 scales of the 128x128 blocks of the
- *                              original matrices: row 2c is W_gate block c,
- *                              row 2c+1 is W_up block c
+ *   w13    [N+1, 2I, H]        E4M3: for each 128-channel block c of the
+ *                              intermediate size, 128 rows of W_gate
+ *                              (channels 128c..128c+127) then the 128 rows
+ *                              of W_up for the same channels
+ *   s13    [N+1, 2I/128, H/128] float32 block scales of w13 (same row order)
  *   w2     [N+1, H, I]         E4M3 W_down
  *   s2     [N+1, H/128, I/128] float32 block scales of w2
  * w13 and w2 must be 16-byte aligned.

@@ -195,35 +195,6 @@ MOE_DEV void mma_commit(uint32_t bar) {
 
 MOE_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 16 consecutive fp32 columns of this thread's TMEM lane (asynchronous: the
-// registers are valid only after tmem_wait_ld_tied on them).
-MOE_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// tcgen05.wait::ld that also names the 32 destination registers of the loads
-// it completes, so that no use of them can be scheduled before the wait.
-MOE_DEV void tmem_wait_ld_tied(float (&a)[16], float (&b)[16]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]),
-                 "+f"(a[6]), "+f"(a[7]), "+f"(a[8]), "+f"(a[9]), "+f"(a[10]), "+f"(a[11]),
-                 "+f"(a[12]), "+f"(a[13]), "+f"(a[14]), "+f"(a[15]), "+f"(b[0]), "+f"(b[1]),
-                 "+f"(b[2]), "+f"(b[3]), "+f"(b[4]), "+f"(b[5]), "+f"(b[6]), "+f"(b[7]),
-                 "+f"(b[8]), "+f"(b[9]), "+f"(b[10]), "+f"(b[11]), "+f"(b[12]), "+f"(b[13]),
-                 "+f"(b[14]), "+f"(b[15])
-               :
-               : "memory");
-}
-
 // 32 consecutive fp32 columns of this thread's TMEM lane.
 MOE_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];

@@ -4,7 +4,7 @@ library; this module only owns memory and forwards pointers.
 
 Also builds a workload's device weights from its block pool: the pool is
 quantised on the GPU by moe_quantize_128x128 and the code/scale blocks are
-placed into the ABI layout (w13 interleaves W_gate and W_up in 64-row pieces) by
+placed into the ABI layout (w13 interleaves W_gate and W_up per 128 rows) by
 indexing, which moves bytes and computes nothing.
 """
 from __future__ import annotations
@@ -49,31 +49,15 @@ def _place(codes: torch.Tensor, scales: torch.Tensor, slots: np.ndarray, out_q: 
         out_s[e0:e0 + chunk] = scales[idx]
 
 
-def pack_w13(gate: torch.Tensor, up: torch.Tensor, s_gate: torch.Tensor, s_up: torch.Tensor):
-    """w13/s13 in the ABI layout from W_gate, W_up codes [E, I, H] and their
-    128x128 block scales [E, I/128, H/128]: per 128-channel block, 64 gate
-    rows, 64 up rows, the next 64 gate rows, the next 64 up rows; scale rows
-    alternate gate block, up block."""
-    e, i, h = gate.shape
-    g = gate.reshape(e, i // 128, 2, 64, h)
-    u = up.reshape(e, i // 128, 2, 64, h)
-    w13 = torch.stack([g, u], dim=3).reshape(e, 2 * i, h).contiguous()
-    s13 = torch.stack([s_gate, s_up], dim=2).reshape(e, 2 * (i // 128), h // 128).contiguous()
-    return w13, s13
-
-
 def device_weights(w: Workload, pool: WeightPool, gate_w: np.ndarray, device) -> DeviceWeights:
     q13, s13p = quantise_pool(pool.pool13, device)
     q2, s2p = quantise_pool(pool.pool2, device)
     e, ib, hb = w.E, w.I // 128, w.H // 128
-    gate = torch.empty((e, w.I, w.H), dtype=torch.uint8, device=device)
-    up = torch.empty((e, w.I, w.H), dtype=torch.uint8, device=device)
-    s_gate = torch.empty((e, ib, hb), dtype=torch.float32, device=device)
-    s_up = torch.empty((e, ib, hb), dtype=torch.float32, device=device)
-    _place(q13, s13p, pool.slot_gate, gate, s_gate)
-    _place(q13, s13p, pool.slot_up, up, s_up)
-    w13, s13 = pack_w13(gate, up, s_gate, s_up)
-    del gate, up
+    # row-block order of w13: gate block c, then up block c, for c = 0 .. I/128-1
+    slots13 = np.stack([pool.slot_gate, pool.slot_up], axis=2).reshape(e, 2 * ib, hb)
+    w13 = torch.empty((e, 2 * w.I, w.H), dtype=torch.uint8, device=device)
+    s13 = torch.empty((e, 2 * ib, hb), dtype=torch.float32, device=device)
+    _place(q13, s13p, slots13, w13, s13)
     w2 = torch.empty((e, w.H, w.I), dtype=torch.uint8, device=device)
     s2 = torch.empty((e, hb, ib), dtype=torch.float32, device=device)
     _place(q2, s2p, pool.slot_down, w2, s2)

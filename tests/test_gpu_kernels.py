@@ -139,27 +139,17 @@ def _gemm_case(h_dim, i_dim, group_rows, seed=0):
     a = rng.standard_normal((rows, h_dim)).astype(np.float32)
     a *= rng.uniform(0.1, 10, (rows, 1)).astype(np.float32)
     a_q, a_s = O.quantize_1x128(a)
-    wg = (rng.standard_normal((n_groups, i_dim, h_dim)) / np.sqrt(h_dim)).astype(np.float32)
-    wu = (rng.standard_normal((n_groups, i_dim, h_dim)) / np.sqrt(h_dim)).astype(np.float32)
+    w13 = (rng.standard_normal((n_groups, 2 * i_dim, h_dim)) / np.sqrt(h_dim)).astype(np.float32)
     w2 = (rng.standard_normal((n_groups, h_dim, i_dim)) / np.sqrt(i_dim)).astype(np.float32)
-    ib, hb = i_dim // 128, h_dim // 128
-    q13 = np.empty((n_groups, 2 * i_dim, h_dim), np.uint8)
-    s13 = np.empty((n_groups, 2 * ib, hb), np.float32)
+    q13 = np.empty(w13.shape, np.uint8)
+    s13 = np.empty((n_groups, 2 * i_dim // 128, h_dim // 128), np.float32)
     q2 = np.empty(w2.shape, np.uint8)
-    s2 = np.empty((n_groups, hb, ib), np.float32)
-    deq_gate, deq_up = [], []
+    s2 = np.empty((n_groups, h_dim // 128, i_dim // 128), np.float32)
     for g in range(n_groups):
-        qg, sg = O.quantize_128x128(wg[g])
-        qu, su = O.quantize_128x128(wu[g])
-        deq_gate.append(O.dequantize_128x128(qg, sg))
-        deq_up.append(O.dequantize_128x128(qu, su))
-        # ABI layout: per 128-channel block, 64 gate rows, 64 up rows, 64, 64
-        q13[g] = np.stack([qg.reshape(ib, 2, 64, h_dim), qu.reshape(ib, 2, 64, h_dim)],
-                          axis=2).reshape(2 * i_dim, h_dim)
-        s13[g] = np.stack([sg, su], axis=1).reshape(2 * ib, hb)
+        q13[g], s13[g] = O.quantize_128x128(w13[g])
         q2[g], s2[g] = O.quantize_128x128(w2[g])
     return dict(rows=rows, starts=np.array(starts, np.int32), counts=np.array(group_rows, np.int32),
-                a_q=a_q, a_s=a_s, q13=q13, s13=s13, q2=q2, s2=s2, gate=deq_gate, up=deq_up)
+                a_q=a_q, a_s=a_s, q13=q13, s13=s13, q2=q2, s2=s2)
 
 
 def _dev(a):
@@ -189,7 +179,9 @@ def test_expert_up_parity(capi, h_dim, i_dim, group_rows):
         written[st:st + n] = True
         if n == 0:
             continue
-        gate, up = c["gate"][g], c["up"][g]
+        w13 = O.dequantize_128x128(c["q13"][g], c["s13"][g])
+        gate = np.concatenate([w13[256 * j:256 * j + 128] for j in range(i_dim // 128)])
+        up = np.concatenate([w13[256 * j + 128:256 * j + 256] for j in range(i_dim // 128)])
         xr = x_hat[st:st + n]
         h = O.silu(xr @ gate.T) * (xr @ up.T)
         # the GPU code of every element is the E4M3 rounding of h * scale up to
