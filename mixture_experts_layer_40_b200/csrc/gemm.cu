@@ -1,64 +1,55 @@
-// Grouped FP8 E4M3 expert GEMMs on tcgen05 tensor cores (sm_100a), issued
-// as 2-SM pair MMAs (cta_group::2).
+// Grouped FP8 E4M3 expert GEMMs on tcgen05 tensor cores (sm_100a).
 //
 // Numerics follow "DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing,
 // Multi-Token Prediction, and FP8 Training at 671B Scale" (trishampatil.com),
 // section V "Four details", items 1-2: E4M3 operands with one scale per 1x128
 // activation tile and per 128x128 weight block, and partial sums promoted to
 // fp32 every N_C = 128 products. The pages' H800 design promotes on CUDA cores
-// while a second WGMMA group computes. Here every 128-deep k-block is summed
-// by the tensor core into its own TMEM buffer (two buffers, ping-pong) and
-// eight promotion warps per SM read it back with tcgen05.ld and add
+// while a second WGMMA group computes; here every 128-deep k-block is
+// accumulated by the tensor core into its own TMEM buffer (two buffers, ping-
+// pong) and eight epilogue warps read it back with tcgen05.ld and add
 // partial * 1/(s_a s_b) into fp32 register totals while the tensor core fills
 // the other buffer.
 //
-// A cluster of two CTAs (two SMs) computes one 256-row x 256-column tile:
-// each CTA loads its 128 rows of A and its 128 rows (half the columns) of B
-// into its own shared memory, the even CTA issues the pair MMA (M=256, N=256,
-// K=32) that reads both halves, and each CTA's TMEM receives the 128 x 256
-// accumulator of its own rows. Against a one-SM 128 x 256 tile this halves the
-// weight bytes every SM loads and reads per MMA, which is what bounds the
-// one-SM version (shared-memory and L2 traffic, not the tensor core).
-//
-// Per CTA, 384 threads (three warpgroups):
-//   warp 0     TMA producer for this CTA's halves; the completion of both
-//              CTAs' loads is counted on the even CTA's stage barrier
-//   warp 1     TMEM allocator (pair allocation) and, in the even CTA, the MMA
-//              issuer; the MMA commits arrive on both CTAs' barriers
+// One persistent CTA per SM, 384 threads (three warpgroups):
+//   warp 0     TMA producer: A (128 rows x 128 B) and B (256 rows x 128 B)
+//              k-block tiles into a 4-stage shared-memory ring
+//   warp 1     TMEM allocator and MMA issuer (one thread): 4 MMAs of
+//              M=128, N=256, K=32 per k-block into TMEM buffer (k-block & 1)
 //   warps 2-3  idle (they only complete the first warpgroup)
-//   warps 4-11 promotion + epilogue on this CTA's 128 rows; warp w reads TMEM
-//              lanes 32*(w%4)..+31; each warpgroup owns half of the 256 columns
+//   warps 4-11 promotion + epilogue; warp w reads TMEM lanes 32*(w%4)..+31,
+//              so each warpgroup covers the 128 rows of a tile and owns half
+//              of its 256 columns
 // The first warpgroup gives registers back (setmaxnreg) so that each epilogue
-// thread can hold 128 fp32 totals plus two 16-column chunks in flight.
-// Work units are (group, n-tile, m-tile) with m fastest, so the m-tiles of one
+// thread can hold 128 fp32 totals plus two 32-column partial chunks.
+// Tiles are (group, n-tile, m-tile) with m fastest, so the m-tiles of one
 // expert's weight tile run back to back and the weight tile is read from HBM
-// about once. Every wait is bounded; a time-out raises the status word, and
-// the CTAs drain their in-flight copies and MMAs before TMEM is released.
+// about once. Every wait is bounded; a time-out raises the status word and
+// the CTA drains its in-flight copies and MMAs before releasing TMEM.
 #include "kernels.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kBMc = 128;       // rows per CTA
-constexpr int kBMp = 256;       // rows per pair tile
-constexpr int kBN = 256;        // columns per tile
-constexpr int kBNc = kBN / 2;   // B rows held by each CTA
+constexpr int kBM = 128;
+constexpr int kBN = 256;
 constexpr int kBK = 128;
-constexpr int kStages = 6;
-constexpr int kABytes = kBMc * kBK;
-constexpr int kBBytes = kBNc * kBK;
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK;
+constexpr int kBBytes = kBN * kBK;
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 384;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 256;
 constexpr int kMaxGroups = 1025;
-constexpr uint32_t kIdesc = make_idesc(kBMp, kBN, 0u, 0u);  // E4M3 x E4M3 -> fp32
+constexpr uint32_t kIdesc = make_idesc(kBM, kBN, 0u, 0u);  // E4M3 x E4M3 -> fp32
 constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024;
 // Register split: launched at kLaunchRegs per thread (384 x 168 = 64512);
 // warpgroup 0 drops to kRegsCtl, the two epilogue warpgroups rise to kRegsEpi.
+// 128 * kRegsCtl + 256 * kRegsEpi must not exceed 384 * kLaunchRegs.
 constexpr int kLaunchRegs = 168;
-constexpr int kRegsCtl = 64;
-constexpr int kRegsEpi = 216;
+constexpr int kRegsCtl = 40;
+constexpr int kRegsEpi = 232;
 static_assert(128 * kRegsCtl + 256 * kRegsEpi <= kThreads * kLaunchRegs, "register split");
 
 struct GemmArgs {
@@ -80,15 +71,15 @@ struct GemmArgs {
 };
 
 struct alignas(8) GemmShared {
-  uint64_t full[kStages];   // even CTA: both CTAs' bytes of a stage have landed
-  uint64_t empty[kStages];  // the pair MMA has consumed a stage (both CTAs)
-  uint64_t tfull[2];        // a TMEM buffer holds a finished k-block (both CTAs)
-  uint64_t tempty[2];       // even CTA: both CTAs have read a TMEM buffer
-  uint64_t xchg;            // amax exchange between the two epilogue groups
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t xchg;           // amax exchange between the two epilogue groups
   uint32_t tmem_base;
   int abort;
   int prefix[kMaxGroups + 1];
-  float amax[2][2][kBMc];   // [tile parity][epilogue group][row]
+  float amax[2][2][kBM];   // [tile parity][epilogue group][row]
 };
 
 MOE_DEV void decode_tile(int tile, const int* prefix, int n_groups, int n_tiles, int& g, int& n,
@@ -107,15 +98,6 @@ MOE_DEV void decode_tile(int tile, const int* prefix, int n_groups, int n_tiles,
 
 MOE_DEV float silu(float a) { return a / (1.0f + expf(-a)); }
 
-MOE_DEV uint4 quant16(const float* v, float s) {
-  uint4 o;
-  o.x = e4m3x4(__fmul_rn(v[0], s), __fmul_rn(v[1], s), __fmul_rn(v[2], s), __fmul_rn(v[3], s));
-  o.y = e4m3x4(__fmul_rn(v[4], s), __fmul_rn(v[5], s), __fmul_rn(v[6], s), __fmul_rn(v[7], s));
-  o.z = e4m3x4(__fmul_rn(v[8], s), __fmul_rn(v[9], s), __fmul_rn(v[10], s), __fmul_rn(v[11], s));
-  o.w = e4m3x4(__fmul_rn(v[12], s), __fmul_rn(v[13], s), __fmul_rn(v[14], s), __fmul_rn(v[15], s));
-  return o;
-}
-
 template <bool kUp>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
@@ -125,9 +107,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t ring = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();   // 0: even CTA (issues the MMAs), 1: odd
-  const int pair = (int)cluster_id_x();
-  const int n_pairs = (int)cluster_count_x();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -136,9 +115,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&sh.tfull[b]), 1);
-      mbar_init(smem_u32(&sh.tempty[b]), 2 * kEpiWarps);
+      mbar_init(smem_u32(&sh.tempty[b]), kEpiThreads / 32);
     }
-    mbar_init(smem_u32(&sh.xchg), kEpiWarps * 32);
+    mbar_init(smem_u32(&sh.xchg), kEpiThreads);
     sh.abort = 0;
     fence_mbar_init();
   }
@@ -146,10 +125,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_b);
   }
-  if (warp == 1) tmem_alloc_pair(smem_u32(&sh.tmem_base), 512);
+  if (warp == 1) tmem_alloc(smem_u32(&sh.tmem_base), 512);
   if (warp == 2) {
-    // pair-tile (256-row) prefix over the groups; a group whose rows fall
-    // outside the buffers or whose start is not 128-aligned is flagged and skipped
+    // m-tile prefix over the groups; a group whose rows fall outside the
+    // buffers or whose start is not 128-aligned is flagged and skipped
     int carry = 0;
     if (lane == 0) sh.prefix[0] = 0;
     for (int base = 0; base < p.n_groups; base += 32) {
@@ -158,9 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g < p.n_groups) {
         const int r = p.group_rows[g];
         const int st = p.group_start[g];
-        const bool ok = r >= 0 && st >= 0 && (st % kBMc) == 0 && (int64_t)st + r <= p.rows;
+        const bool ok = r >= 0 && st >= 0 && (st % kBM) == 0 && (int64_t)st + r <= p.rows;
         if (!ok) flag_status(p.status, kStatusBounds);
-        mt = ok ? (r + kBMp - 1) / kBMp : 0;
+        mt = ok ? (r + kBM - 1) / kBM : 0;
       }
       int incl = mt;
 #pragma unroll
@@ -174,8 +153,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  // both CTAs' barriers are initialised before any cross-CTA arrival
-  cluster_sync();
   tc_fence_after();
 
   const uint32_t tmem_base = sh.tmem_base;
@@ -193,24 +170,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_b = policy_evict_first();
       int it = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         int g, n, m;
         decode_tile(tile, sh.prefix, p.n_groups, p.n_tiles, g, n, m);
-        const int a_row = p.group_start[g] + m * kBMp + (int)rank * kBMc;
-        const int b_row = g * p.b_rows + n * kBN + (int)rank * kBNc;
+        const int a_row = p.group_start[g] + m * kBM;
+        const int b_row = g * p.b_rows + n * kBN;
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
           if (!mbar_wait(smem_u32(&sh.empty[s]), ph ^ 1u, abort, p.status)) { ok = false; break; }
-          const uint32_t full_even = map_to_rank(smem_u32(&sh.full[s]), 0);
-          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&sh.full[s]), 2 * kStageBytes);
+          const uint32_t full = smem_u32(&sh.full[s]);
+          mbar_arrive_expect_tx(full, kStageBytes);
           const uint32_t sa = ring + s * kStageBytes;
-          tma_load_2d_pair(sa, &tm_a, kb * kBK, a_row, full_even, pol_a);
-          tma_load_2d_pair(sa + kABytes, &tm_b, kb * kBK, b_row, full_even, pol_b);
+          tma_load_2d_hint(sa, &tm_a, kb * kBK, a_row, full, pol_a);
+          tma_load_2d_hint(sa + kABytes, &tm_b, kb * kBK, b_row, full, pol_b);
         }
       }
-      if (!ok && rank == 0) {
-        // drain: every armed stage must land before the pair may exit
+      if (!ok) {
+        // drain: every armed stage must land before the CTA may exit
         for (int s = 0; s < kStages && s < it; ++s) {
           const int last = s + ((it - 1 - s) / kStages) * kStages;
           mbar_wait(smem_u32(&sh.full[s]), (uint32_t)(last / kStages) & 1u, nullptr, p.status);
@@ -218,11 +195,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       int it = 0, kbi = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         for (int kb = 0; kb < kb_n; ++kb, ++it, ++kbi) {
           const int buf = kbi & 1;
           const uint32_t use = (uint32_t)(kbi >> 1);
@@ -236,11 +213,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t d = tmem_base + (uint32_t)(buf * kBN);
 #pragma unroll
           for (int k4 = 0; k4 < kBK / 32; ++k4) {
-            mma_f8_pair(d, smem_desc_sw128(sa + k4 * 32), smem_desc_sw128(sa + kABytes + k4 * 32),
-                        kIdesc, k4 > 0 ? 1u : 0u);
+            mma_f8(d, smem_desc_sw128(sa + k4 * 32), smem_desc_sw128(sa + kABytes + k4 * 32), kIdesc,
+                   k4 > 0 ? 1u : 0u);
           }
-          mma_commit_pair(smem_u32(&sh.empty[s]), (uint16_t)0x3);
-          mma_commit_pair(smem_u32(&sh.tfull[buf]), (uint16_t)0x3);
+          mma_commit(smem_u32(&sh.empty[s]));
+          mma_commit(smem_u32(&sh.tfull[buf]));
         }
       }
       if (!ok && kbi > 0) {
@@ -256,24 +233,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const int b_blocks = p.b_rows / kBMc;
-    // columns owned by this thread: up -> gate [64eg, 64eg+64) and up
-    // [128+64eg, ...); down -> [128eg, 128eg+128)
-    const uint32_t c0 = kUp ? (uint32_t)(64 * eg) : (uint32_t)(128 * eg);
-    const uint32_t c2 = kUp ? (uint32_t)(128 + 64 * eg) : (uint32_t)(128 * eg + 64);
-    const uint32_t tempty_even0 = map_to_rank(smem_u32(&sh.tempty[0]), 0);
-    const uint32_t tempty_even1 = map_to_rank(smem_u32(&sh.tempty[1]), 0);
+    const int b_blocks = p.b_rows / kBM;
     int kbi = 0;
     uint32_t xchg_phase = 0;
     int tile_count = 0;
-    bool ok = true;
     float acc[128];
-    for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++tile_count) {
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tile_count) {
       int g, n, m;
       decode_tile(tile, sh.prefix, p.n_groups, p.n_tiles, g, n, m);
-      const int row0 = m * kBMp + (int)rank * kBMc;   // first row of this CTA inside the group
-      const int valid = p.group_rows[g] - row0;
-      const int64_t grow = (int64_t)p.group_start[g] + row0 + row;
+      const int valid = p.group_rows[g] - m * kBM;
+      const int64_t grow = (int64_t)p.group_start[g] + m * kBM + row;
       const bool live = row < valid;
       const float* sa_ptr = p.a_s + (live ? grow : 0) * kb_n;
       const float* sb0 = p.b_s + ((int64_t)g * b_blocks + 2 * n + (kUp ? 0 : eg)) * kb_n;
@@ -283,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sa_next = __ldg(sa_ptr);
       float sb0_next = __ldg(sb0);
       float sb1_next = kUp ? __ldg(sb1) : 0.0f;
+      bool ok = true;
       for (int kb = 0; kb < kb_n; ++kb, ++kbi) {
         const float sa = sa_next, s0 = sb0_next, s1 = sb1_next;
         if (kb + 1 < kb_n) {
@@ -290,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           sb0_next = __ldg(sb0 + kb + 1);
           if (kUp) sb1_next = __ldg(sb1 + kb + 1);
         }
-        const float inv0 = __frcp_rn(sa * s0);
-        const float inv1 = kUp ? __frcp_rn(sa * s1) : inv0;
+        const float inv0 = 1.0f / (sa * s0);
+        const float inv1 = kUp ? 1.0f / (sa * s1) : inv0;
         const int buf = kbi & 1;
         // the result is made warp-uniform: tcgen05.ld below is warp-collective
         ok = __all_sync(0xffffffffu,
@@ -299,44 +269,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t t0 = lane_addr + (uint32_t)(buf * kBN);
-        // four pairs of 16-column chunks; the next pair is in flight while the
-        // current one is folded into the totals
-        float pa[16], pb[16], qa[16], qb[16];
-        tmem_ld16(t0 + c0, pa);
-        tmem_ld16(t0 + c0 + 16, pb);
-        tmem_wait_ld_tied(pa, pb);
-        tmem_ld16(t0 + c0 + 32, qa);
-        tmem_ld16(t0 + c0 + 48, qb);
+        // columns owned by this thread: up -> gate [64eg, 64eg+64) and up
+        // [128+64eg, ...); down -> [128eg, 128eg+128)
+        const uint32_t c0 = kUp ? (uint32_t)(64 * eg) : (uint32_t)(128 * eg);
+        const uint32_t c2 = kUp ? (uint32_t)(128 + 64 * eg) : (uint32_t)(128 * eg + 64);
+        float v0[32], v1[32];
+        tmem_ld32(t0 + c0, v0);
+        tmem_ld32(t0 + c0 + 32, v1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          acc[i] = fmaf(pa[i], inv0, acc[i]);
-          acc[16 + i] = fmaf(pb[i], inv0, acc[16 + i]);
-        }
-        tmem_wait_ld_tied(qa, qb);
-        tmem_ld16(t0 + c2, pa);
-        tmem_ld16(t0 + c2 + 16, pb);
+        for (int i = 0; i < 32; ++i) acc[i] = fmaf(v0[i], inv0, acc[i]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          acc[32 + i] = fmaf(qa[i], inv0, acc[32 + i]);
-          acc[48 + i] = fmaf(qb[i], inv0, acc[48 + i]);
-        }
-        tmem_wait_ld_tied(pa, pb);
-        tmem_ld16(t0 + c2 + 32, qa);
-        tmem_ld16(t0 + c2 + 48, qb);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          acc[64 + i] = fmaf(pa[i], inv1, acc[64 + i]);
-          acc[80 + i] = fmaf(pb[i], inv1, acc[80 + i]);
-        }
-        tmem_wait_ld_tied(qa, qb);
+        for (int i = 0; i < 32; ++i) acc[32 + i] = fmaf(v1[i], inv0, acc[32 + i]);
+        tmem_ld32(t0 + c2, v0);
+        tmem_ld32(t0 + c2 + 32, v1);
+        tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(buf ? tempty_even1 : tempty_even0);
+        if (lane == 0) mbar_arrive(smem_u32(&sh.tempty[buf]));
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          acc[96 + i] = fmaf(qa[i], inv1, acc[96 + i]);
-          acc[112 + i] = fmaf(qb[i], inv1, acc[112 + i]);
-        }
+        for (int i = 0; i < 32; ++i) acc[64 + i] = fmaf(v0[i], inv1, acc[64 + i]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(v1[i], inv1, acc[96 + i]);
       }
       if (!ok) break;
 
@@ -353,16 +307,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int par = tile_count & 1;
         sh.amax[par][eg][row] = amax;
         mbar_arrive(smem_u32(&sh.xchg));
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh.xchg), xchg_phase, abort, p.status));
-        if (!ok) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sh.xchg), xchg_phase, abort, p.status))) break;
         xchg_phase ^= 1u;
         amax = fmaxf(sh.amax[par][0][row], sh.amax[par][1][row]);
         const float s = tile_scale(amax);
         if (live) {
-          uint4* dst = reinterpret_cast<uint4*>(p.h_q + grow * p.I + n * kBMc + 64 * eg);
+          uint4* dst = reinterpret_cast<uint4*>(p.h_q + grow * p.I + n * kBM + 64 * eg);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = quant16(acc + 16 * j, s);
-          if (eg == 0) p.h_s[grow * (p.I / kBMc) + n] = s;
+          for (int j = 0; j < 4; ++j) {
+            uint4 o;
+            o.x = e4m3x4(__fmul_rn(acc[16 * j + 0], s), __fmul_rn(acc[16 * j + 1], s),
+                         __fmul_rn(acc[16 * j + 2], s), __fmul_rn(acc[16 * j + 3], s));
+            o.y = e4m3x4(__fmul_rn(acc[16 * j + 4], s), __fmul_rn(acc[16 * j + 5], s),
+                         __fmul_rn(acc[16 * j + 6], s), __fmul_rn(acc[16 * j + 7], s));
+            o.z = e4m3x4(__fmul_rn(acc[16 * j + 8], s), __fmul_rn(acc[16 * j + 9], s),
+                         __fmul_rn(acc[16 * j + 10], s), __fmul_rn(acc[16 * j + 11], s));
+            o.w = e4m3x4(__fmul_rn(acc[16 * j + 12], s), __fmul_rn(acc[16 * j + 13], s),
+                         __fmul_rn(acc[16 * j + 14], s), __fmul_rn(acc[16 * j + 15], s));
+            dst[j] = o;
+          }
+          if (eg == 0) p.h_s[grow * (p.I / kBM) + n] = s;
         }
       } else {
         if (live) {
@@ -377,17 +341,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  // neither CTA releases the pair's TMEM while the other may still use it
-  cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
 }
 
 template <bool kUp>
 cudaError_t launch(const GemmArgs& a, const CUtensorMap& ma, const CUtensorMap& mb,
                    cudaStream_t stream, int sm_count, int64_t tile_bound) {
-  static int max_pairs = 0;
-  if (max_pairs == 0) {
+  static bool configured = false;
+  if (!configured) {
     // the register split above is only safe if the kernel really was built
     // with kLaunchRegs registers per thread
     cudaFuncAttributes fa;
@@ -397,37 +359,12 @@ cudaError_t launch(const GemmArgs& a, const CUtensorMap& ma, const CUtensorMap& 
     e = cudaFuncSetAttribute(grouped_gemm_kernel<kUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kDynSmem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t probe = {};
-    probe.gridDim = dim3((unsigned)(sm_count / 2 * 2));
-    probe.blockDim = dim3(kThreads);
-    probe.dynamicSmemBytes = kDynSmem;
-    cudaLaunchAttribute cl;
-    cl.id = cudaLaunchAttributeClusterDimension;
-    cl.val.clusterDim.x = 2;
-    cl.val.clusterDim.y = 1;
-    cl.val.clusterDim.z = 1;
-    probe.attrs = &cl;
-    probe.numAttrs = 1;
-    int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<kUp>, &probe);
-    if (e != cudaSuccess || clusters < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
-    max_pairs = clusters;
+    configured = true;
   }
-  int pairs = max_pairs;
-  if (tile_bound < pairs) pairs = (int)(tile_bound > 0 ? tile_bound : 1);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * pairs));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kDynSmem;
-  cfg.stream = stream;
-  cudaLaunchAttribute cl;
-  cl.id = cudaLaunchAttributeClusterDimension;
-  cl.val.clusterDim.x = 2;
-  cl.val.clusterDim.y = 1;
-  cl.val.clusterDim.z = 1;
-  cfg.attrs = &cl;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kUp>, ma, mb, a);
+  int grid = sm_count;
+  if (tile_bound < grid) grid = (int)(tile_bound > 0 ? tile_bound : 1);
+  grouped_gemm_kernel<kUp><<<grid, kThreads, kDynSmem, stream>>>(ma, mb, a);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -436,9 +373,9 @@ cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const fl
                              const uint8_t* w13, const float* s13, uint8_t* h_q, float* h_s,
                              cudaStream_t stream, int sm_count) {
   CUtensorMap ma, mb;
-  cudaError_t e = make_tmap_u8(&ma, a_q, gg.H, gg.rows, kBK, kBMc);
+  cudaError_t e = make_tmap_u8(&ma, a_q, gg.H, gg.rows, kBK, kBM);
   if (e != cudaSuccess) return e;
-  e = make_tmap_u8(&mb, w13, gg.H, (int64_t)gg.n_groups * 2 * gg.I, kBK, kBNc);
+  e = make_tmap_u8(&mb, w13, gg.H, (int64_t)gg.n_groups * 2 * gg.I, kBK, kBN);
   if (e != cudaSuccess) return e;
   GemmArgs a{};
   a.group_rows = gg.group_rows;
@@ -455,7 +392,7 @@ cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const fl
   a.I = gg.I;
   a.H = gg.H;
   a.status = gg.status;
-  const int64_t bound = (gg.rows / kBMp + gg.n_groups) * (int64_t)a.n_tiles;
+  const int64_t bound = (gg.rows / kBM + gg.n_groups) * (int64_t)a.n_tiles;
   return launch<true>(a, ma, mb, stream, sm_count, bound);
 }
 
@@ -463,9 +400,9 @@ cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const 
                                const uint8_t* w2, const float* s2, float* y,
                                cudaStream_t stream, int sm_count) {
   CUtensorMap ma, mb;
-  cudaError_t e = make_tmap_u8(&ma, h_q, gg.I, gg.rows, kBK, kBMc);
+  cudaError_t e = make_tmap_u8(&ma, h_q, gg.I, gg.rows, kBK, kBM);
   if (e != cudaSuccess) return e;
-  e = make_tmap_u8(&mb, w2, gg.I, (int64_t)gg.n_groups * gg.H, kBK, kBNc);
+  e = make_tmap_u8(&mb, w2, gg.I, (int64_t)gg.n_groups * gg.H, kBK, kBN);
   if (e != cudaSuccess) return e;
   GemmArgs a{};
   a.group_rows = gg.group_rows;
@@ -481,7 +418,7 @@ cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const 
   a.I = gg.I;
   a.H = gg.H;
   a.status = gg.status;
-  const int64_t bound = (gg.rows / kBMp + gg.n_groups) * (int64_t)a.n_tiles;
+  const int64_t bound = (gg.rows / kBM + gg.n_groups) * (int64_t)a.n_tiles;
   return launch<false>(a, ma, mb, stream, sm_count, bound);
 }
 
