@@ -112,6 +112,7 @@ typedef struct {
   size_t h_q;           /* E4M3 [rows_total, I]: SwiGLU output, 1x128 re-quantised */
   size_t h_s;           /* float [rows_total, I/128] */
   size_t y_rows;        /* float [rows_total, H]: expert outputs before the combine */
+  size_t gate_split;    /* bf16 [3, N, H]: the fp32 centroids as three bf16 terms */
   size_t total;         /* workspace bytes required */
 } moe_ws_layout;
 

@@ -40,7 +40,7 @@ class moe_weights(ctypes.Structure):
 
 _LAYOUT_FIELDS = ["status", "counts", "offsets", "group_rows", "row_start", "row_token",
                   "token_row", "topk_ids", "topk_gates", "logits", "a_q", "a_s", "h_q", "h_s",
-                  "y_rows", "total"]
+                  "y_rows", "gate_split", "total"]
 
 
 class moe_ws_layout(ctypes.Structure):

@@ -74,6 +74,7 @@ void layout_of(const moe_shape& s, moe_ws_layout* L) {
   L->h_q = take((size_t)L->rows_total * I);
   L->h_s = take((size_t)L->rows_total * (I / kTile) * 4);
   L->y_rows = take((size_t)L->rows_total * H * 4);
+  L->gate_split = take(router_split_bytes((int)N, (int)H));
   L->total = off;
 }
 
@@ -95,6 +96,23 @@ cudaError_t make_tmap_u8(CUtensorMap* map, const void* base, int64_t inner, int6
   const cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
+                           int64_t depth, int box_inner, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)(rows > 0 ? rows : 1),
+                              (cuuint64_t)(depth > 0 ? depth : 1)};
+  const cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)(inner * 2 * (rows > 0 ? rows : 1))};
+  const cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint32_t rank = depth > 1 ? 3 : 2;
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -157,8 +175,9 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
   cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
   if (e == cudaSuccess)
-    e = launch_router(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, at<float>(ws, L.logits), topk_ids,
-                      topk_gates, counts, status, s, sm_count());
+    e = launch_router_tc(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K,
+                         at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), topk_ids,
+                         topk_gates, counts, status, s, sm_count());
   return cuda_status(e);
 }
 
@@ -200,8 +219,9 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   e = mark(1, e);
   // a2-a5: gate logits, sigmoid, biased top-K, gates, counts
   if (e == cudaSuccess)
-    e = launch_router(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K, at<float>(ws, L.logits), ids,
-                      gates, counts, status, s, sms);
+    e = launch_router_tc(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K,
+                         at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
+                         counts, status, s, sms);
   e = mark(2, e);
   // a6-a7: offsets, stable expert-major scatter, gather of the quantised rows
   if (e == cudaSuccess)

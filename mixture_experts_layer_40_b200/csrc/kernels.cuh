@@ -19,6 +19,10 @@ struct GroupedGemm {
 // box_inner bytes x box_rows rows, 128-byte swizzle (host side).
 cudaError_t make_tmap_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
                          int box_inner, int box_rows);
+// bf16 tensor map over [depth, rows, inner] (depth 1: 2-D), box of box_inner
+// elements x box_rows rows x 1, 128-byte swizzle (host side).
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
+                           int64_t depth, int box_inner, int box_rows);
 
 cudaError_t launch_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q,
                                   float* scales, cudaStream_t stream, int sm_count);
@@ -30,6 +34,15 @@ cudaError_t launch_quantize_128x128(const float* w, int64_t rows, int64_t cols, 
 cudaError_t launch_router(const void* x, const float* gate_w, const float* bias, int T, int H,
                           int N, int K, float* logits, int32_t* ids, float* gates, int32_t* counts,
                           uint32_t* status, cudaStream_t stream, int sm_count);
+
+// Router on tensor cores: splits the fp32 centroids into three bf16 terms in
+// `wsplit` (router_split_bytes), computes the logits with BF16 tcgen05 MMAs
+// and fp32 accumulation, then the same top-K as launch_router.
+size_t router_split_bytes(int N, int H);
+cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
+                             int N, int K, __nv_bfloat16* wsplit, float* logits, int32_t* ids,
+                             float* gates, int32_t* counts, uint32_t* status, cudaStream_t stream,
+                             int sm_count);
 
 // Permutation: scan of counts into group tables, stable scatter, row gather.
 cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K, int H,

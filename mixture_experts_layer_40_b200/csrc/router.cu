@@ -5,6 +5,8 @@
 // the gate is the unbiased affinity normalised over the K chosen. Gating stays
 // in fp32 ("DeepSeek-V3, explained", recipe step 7), so the logits come from an
 // fp32 FMA GEMM of the bf16 input and the fp32 centroids.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -158,6 +160,207 @@ cudaError_t launch_router(const void* x, const float* gate_w, const float* bias,
   logits_kernel<<<g1, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), gate_w, T, H, N,
                                         logits);
   cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int blocks = (T + 7) / 8;
+  if (blocks > sm_count * 8) blocks = sm_count * 8;
+  topk_kernel<<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, ids, gates, counts);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Gate logits on tcgen05 tensor cores. The fp32 centroids are split exactly
+// into three bf16 terms (hi + mid + lo carries all 24 significand bits), so
+// x . e_i = sum over the terms of bf16 x bf16 products, each exact in fp32,
+// accumulated in fp32 in TMEM: fp32-accurate logits from BF16 MMAs.
+// One CTA computes a 128-token x 64-expert tile over the whole hidden size.
+// ---------------------------------------------------------------------------
+namespace moe {
+
+namespace {
+
+constexpr int kRM = 128;                  // tokens per tile
+constexpr int kRN = 64;                   // experts per tile
+constexpr int kRK = 64;                   // bf16 elements per k-block (128 bytes)
+constexpr int kRStages = 5;
+constexpr int kRABytes = kRM * kRK * 2;   // 16 KB
+constexpr int kRBBytes = kRN * kRK * 2;   // 8 KB per split term
+constexpr int kRStageBytes = kRABytes + 3 * kRBBytes;
+constexpr int kRThreads = 256;
+constexpr uint32_t kRIdesc = make_idesc(kRM, kRN, 1u, 1u);  // BF16 x BF16 -> fp32
+constexpr size_t kRDynSmem = (size_t)kRStages * kRStageBytes + 1024;
+
+__global__ void __launch_bounds__(256) split_gate_kernel(const float* __restrict__ w, int64_t n,
+                                                         __nv_bfloat16* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = w[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(hi);   // exact
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);  // exact
+    out[i] = hi;
+    out[n + i] = mid;
+    out[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
+struct alignas(8) RouterShared {
+  uint64_t full[kRStages];
+  uint64_t empty[kRStages];
+  uint64_t tfull;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(kRThreads, 1)
+    logits_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                     const __grid_constant__ CUtensorMap tm_w, int T, int H, int N,
+                     float* __restrict__ z, uint32_t* __restrict__ status) {
+  __shared__ RouterShared sh;
+  extern __shared__ uint8_t dyn_smem[];
+  const uint32_t ring = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kRM;
+  const int n0 = blockIdx.y * kRN;
+  const int kb_n = H / kRK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRStages; ++s) {
+      mbar_init(smem_u32(&sh.full[s]), 1);
+      mbar_init(smem_u32(&sh.empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sh.tfull), 1);
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tm_x);
+    prefetch_tensormap(&tm_w);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(&sh.tmem_base), kRN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sh.tmem_base;
+  volatile int* abort = &sh.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // producer: x tile and the three centroid terms of every k-block
+      int kb = 0;
+      for (; kb < kb_n; ++kb) {
+        const int s = kb % kRStages;
+        const uint32_t ph = (uint32_t)(kb / kRStages) & 1u;
+        if (!mbar_wait(smem_u32(&sh.empty[s]), ph ^ 1u, abort, status)) break;
+        const uint32_t full = smem_u32(&sh.full[s]);
+        mbar_arrive_expect_tx(full, kRStageBytes);
+        const uint32_t sa = ring + s * kRStageBytes;
+        tma_load_2d(sa, &tm_x, kb * kRK, m0, full);
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          asm volatile(
+              "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+              " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(sa + kRABytes + t * kRBBytes),
+              "l"(reinterpret_cast<uint64_t>(&tm_w)), "r"(kb * kRK), "r"(n0), "r"(t), "r"(full)
+              : "memory");
+        }
+      }
+      if (kb < kb_n) {
+        for (int s = 0; s < kRStages && s < kb; ++s) {
+          const int last = s + ((kb - 1 - s) / kRStages) * kRStages;
+          mbar_wait(smem_u32(&sh.full[s]), (uint32_t)(last / kRStages) & 1u, nullptr, status);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // MMA issuer: one fp32 accumulator over all of H and the three terms
+      bool ok = true;
+      bool issued = false;
+      for (int kb = 0; kb < kb_n; ++kb) {
+        const int s = kb % kRStages;
+        const uint32_t ph = (uint32_t)(kb / kRStages) & 1u;
+        if (!mbar_wait(smem_u32(&sh.full[s]), ph, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = ring + s * kRStageBytes;
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+#pragma unroll
+          for (int k = 0; k < kRK / 16; ++k) {
+            mma_bf16(tmem_base, smem_desc_sw128(sa + k * 32),
+                     smem_desc_sw128(sa + kRABytes + t * kRBBytes + k * 32), kRIdesc,
+                     (kb | t | k) != 0 ? 1u : 0u);
+          }
+        }
+        issued = true;
+        mma_commit(smem_u32(&sh.empty[s]));
+      }
+      if (issued) mma_commit(smem_u32(&sh.tfull));
+      if (!ok && issued) mbar_wait(smem_u32(&sh.tfull), 0u, nullptr, status);
+    }
+  } else if (warp >= 4) {
+    // epilogue: 128 rows x 64 columns of fp32 logits -> z
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh.tfull), 0u, abort, status));
+    if (ok) {
+      tc_fence_after();
+      const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      float v0[32], v1[32];
+      tmem_ld32(t0, v0);
+      tmem_ld32(t0 + 32, v1);
+      tmem_wait_ld();
+      const int t = m0 + row;
+      if (t < T) {
+        float* dst = z + (int64_t)t * N + n0;
+        const int cols = min(kRN, N - n0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (4 * j < cols) reinterpret_cast<float4*>(dst)[j] = make_float4(v0[4 * j], v0[4 * j + 1], v0[4 * j + 2], v0[4 * j + 3]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (32 + 4 * j < cols) reinterpret_cast<float4*>(dst + 32)[j] = make_float4(v1[4 * j], v1[4 * j + 1], v1[4 * j + 2], v1[4 * j + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kRN);
+}
+
+}  // namespace
+
+size_t router_split_bytes(int N, int H) { return (size_t)3 * N * H * sizeof(__nv_bfloat16); }
+
+cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
+                             int N, int K, __nv_bfloat16* wsplit, float* logits, int32_t* ids,
+                             float* gates, int32_t* counts, uint32_t* status, cudaStream_t stream,
+                             int sm_count) {
+  if (T == 0) return cudaSuccess;
+  const int64_t nw = (int64_t)N * H;
+  split_gate_kernel<<<(unsigned)std::min<int64_t>((nw + 255) / 256, (int64_t)sm_count * 8), 256, 0,
+                      stream>>>(gate_w, nw, wsplit);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mx, mw;
+  e = make_tmap_bf16(&mx, x, H, T, 1, kRK, kRM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16(&mw, wsplit, H, N, 3, kRK, kRN);
+  if (e != cudaSuccess) return e;
+  static bool configured = false;
+  if (!configured) {
+    e = cudaFuncSetAttribute(logits_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kRDynSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid((unsigned)((T + kRM - 1) / kRM), (unsigned)((N + kRN - 1) / kRN));
+  logits_tc_kernel<<<grid, kRThreads, kRDynSmem, stream>>>(mx, mw, T, H, N, logits, status);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   int blocks = (T + 7) / 8;
   if (blocks > sm_count * 8) blocks = sm_count * 8;

@@ -11,6 +11,7 @@ from mixture_experts_layer_40_b200 import inputs as I
 from tests import helpers as H
 
 pytestmark = pytest.mark.gpu
+GATE_TOL = 1e-5
 
 
 @pytest.fixture(scope="module")
@@ -105,11 +106,13 @@ def test_route_parity(capi, name):
     use_ids, ndiff, nnear = H.reconcile_ids(ids, r_ids, score, w.K)
     assert np.array_equal(counts, O.expert_counts(use_ids, w.N))
     assert counts.sum() == w.T * w.K
-    # gates of the GPU's ids from the oracle's unbiased affinities
+    # gates of the GPU's ids from the oracle's unbiased affinities; the fp32
+    # logits are within ~1e-6 of the float64 ones (|z| up to ~10 in the skewed
+    # workload), which moves a gate by at most a few 1e-6
     sel = np.take_along_axis(s, ids.astype(np.int64), axis=1)
     ref = sel / sel.sum(axis=1, keepdims=True)
-    assert np.max(np.abs(gates - ref)) < 2e-6
-    assert np.allclose(gates.sum(axis=1), 1.0, atol=2e-6)
+    assert np.max(np.abs(gates - ref)) < GATE_TOL
+    assert np.allclose(gates.sum(axis=1), 1.0, atol=GATE_TOL)
 
 
 def test_route_ragged_tokens_and_hot_expert(capi):

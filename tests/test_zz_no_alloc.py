@@ -16,6 +16,8 @@ import pytest
 import torch
 
 from mixture_experts_layer_40_b200 import inputs as I
+from oracle import moe_oracle as O
+from tests import helpers as H
 
 pytestmark = pytest.mark.gpu
 
@@ -72,9 +74,17 @@ def test_two_calls_match_the_workspace_entry_point(capi):
         torch.cuda.synchronize()
         ids, gates, counts = (t.cpu().numpy() for t in got)
         rids, rgates, rcounts = (t.cpu().numpy() for t in ref)
-        assert np.array_equal(ids, rids)
-        assert np.array_equal(counts, rcounts) and counts.sum() == w.T * w.K
-        assert np.max(np.abs(gates - rgates)) <= 2e-6
+        # the two entry points compute the fp32 logits differently (this one
+        # with fp32 FMAs, moe_route on tensor cores), so ids may differ only on
+        # tokens whose K-th and (K+1)-th scores are a near tie; then the same
+        # rule as every routing test applies
+        _, _, _, score = O.route(I.bf16_bits_to_f32(I.make_x(w)), I.make_gate_w(w), I.make_bias(w), w.K)
+        same = np.all(np.sort(ids, 1) == np.sort(rids, 1), axis=1)
+        assert np.all(same | H.near_tie_tokens(score, w.K))
+        assert counts.sum() == w.T * w.K
+        assert np.array_equal(counts, O.expert_counts(ids, w.N))
+        both = same & np.all(ids == rids, axis=1)
+        assert np.max(np.abs(gates[both] - rgates[both])) <= 1e-5
 
 
 def test_size_beyond_the_scratch_is_refused(capi):
