@@ -22,9 +22,12 @@
 //              of its 256 columns
 // The first warpgroup gives registers back (setmaxnreg) so that each epilogue
 // thread can hold 128 fp32 totals plus two 32-column partial chunks.
-// Tiles are (group, n-tile, m-tile) with m fastest, so the m-tiles of one
-// expert's weight tile run back to back and the weight tile is read from HBM
-// about once. Every wait is bounded; a time-out raises the status word and
+// Tiles are (group, m-tile, n-tile) with n fastest: the n-tiles of one row
+// tile run on neighbouring CTAs at the same time and share its A rows in L2.
+// Both operands load with the default L2 policy: with the weight stream
+// marked evict-first (and A evict-last) the HBM reads matched one full read
+// of an expert's weights per row tile, i.e. the expert's second row tile
+// never found them in L2, and the kernel was slower. Every wait is bounded; a time-out raises the status word and
 // the CTA drains its in-flight copies and MMAs before releasing TMEM.
 #include "kernels.cuh"
 
@@ -43,7 +46,11 @@ constexpr int kThreads = 384;
 constexpr int kEpiThreads = 256;
 constexpr int kMaxGroups = 1025;
 constexpr uint32_t kIdesc = make_idesc(kBM, kBN, 0u, 0u);  // E4M3 x E4M3 -> fp32
-constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024;
+// down epilogue: each epilogue warp stages 32 rows x 16 fp32 columns of its
+// output tile in shared memory (64-byte swizzle) for one TMA store at a time
+constexpr int kYCols = 16;
+constexpr int kYBufBytes = 32 * kYCols * 4;
+constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 8 * kYBufBytes + 1024;
 // Register split: launched at kLaunchRegs per thread (384 x 168 = 64512);
 // warpgroup 0 drops to kRegsCtl, the two epilogue warpgroups rise to kRegsEpi.
 // 128 * kRegsCtl + 256 * kRegsEpi must not exceed 384 * kLaunchRegs.
@@ -90,10 +97,9 @@ MOE_DEV void decode_tile(int tile, const int* prefix, int n_groups, int n_tiles,
     if (prefix[mid] * n_tiles <= tile) lo = mid; else hi = mid;
   }
   g = lo;
-  const int mt = prefix[g + 1] - prefix[g];
   const int local = tile - prefix[g] * n_tiles;
-  n = local / mt;
-  m = local - n * mt;
+  m = local / n_tiles;
+  n = local - m * n_tiles;
 }
 
 MOE_DEV float silu(float a) { return a / (1.0f + expf(-a)); }
@@ -101,7 +107,8 @@ MOE_DEV float silu(float a) { return a / (1.0f + expf(-a)); }
 template <bool kUp>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                        const __grid_constant__ CUtensorMap tm_b, const GemmArgs p) {
+                        const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
   __shared__ GemmShared sh;
   extern __shared__ uint8_t dyn_smem[];
   const uint32_t ring = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -124,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_b);
+    if (!kUp) prefetch_tensormap(&tm_y);
   }
   if (warp == 1) tmem_alloc(smem_u32(&sh.tmem_base), 512);
   if (warp == 2) {
@@ -166,8 +174,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      const uint64_t pol_a = policy_evict_last();
-      const uint64_t pol_b = policy_evict_first();
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
@@ -182,8 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t full = smem_u32(&sh.full[s]);
           mbar_arrive_expect_tx(full, kStageBytes);
           const uint32_t sa = ring + s * kStageBytes;
-          tma_load_2d_hint(sa, &tm_a, kb * kBK, a_row, full, pol_a);
-          tma_load_2d_hint(sa + kABytes, &tm_b, kb * kBK, b_row, full, pol_b);
+          tma_load_2d(sa, &tm_a, kb * kBK, a_row, full);
+          tma_load_2d(sa + kABytes, &tm_b, kb * kBK, b_row, full);
         }
       }
       if (!ok) {
@@ -233,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t ybuf = ring + (uint32_t)(kStages * kStageBytes + ew * kYBufBytes);
     const int b_blocks = p.b_rows / kBM;
     int kbi = 0;
     uint32_t xchg_phase = 0;
@@ -262,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float inv0 = 1.0f / (sa * s0);
         const float inv1 = kUp ? 1.0f / (sa * s1) : inv0;
+        const uint64_t inv0x2 = splat_f32x2(inv0), inv1x2 = splat_f32x2(inv1);
         const int buf = kbi & 1;
         // the result is made warp-uniform: tcgen05.ld below is warp-collective
         ok = __all_sync(0xffffffffu,
@@ -278,9 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(t0 + c0 + 32, v1);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = fmaf(v0[i], inv0, acc[i]);
+        for (int i = 0; i < 32; i += 2) fma_f32x2(acc[i], acc[i + 1], v0[i], v0[i + 1], inv0x2);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[32 + i] = fmaf(v1[i], inv0, acc[32 + i]);
+        for (int i = 0; i < 32; i += 2) fma_f32x2(acc[32 + i], acc[33 + i], v1[i], v1[i + 1], inv0x2);
         tmem_ld32(t0 + c2, v0);
         tmem_ld32(t0 + c2 + 32, v1);
         tmem_wait_ld();
@@ -288,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sh.tempty[buf]));
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[64 + i] = fmaf(v0[i], inv1, acc[64 + i]);
+        for (int i = 0; i < 32; i += 2) fma_f32x2(acc[64 + i], acc[65 + i], v0[i], v0[i + 1], inv1x2);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(v1[i], inv1, acc[96 + i]);
+        for (int i = 0; i < 32; i += 2) fma_f32x2(acc[96 + i], acc[97 + i], v1[i], v1[i + 1], inv1x2);
       }
       if (!ok) break;
 
@@ -329,14 +337,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (eg == 0) p.h_s[grow * (p.I / kBM) + n] = s;
         }
       } else {
-        if (live) {
-          float4* dst = reinterpret_cast<float4*>(p.y + grow * p.H + n * kBN + 128 * eg);
+        // fp32 rows out through shared memory and TMA stores, 16 columns of
+        // the warp's 32 rows at a time, when all 32 rows belong to the group;
+        // a group's last, partial 32 rows are stored directly, row by row,
+        // and padding rows are never written
+        const int q_live = valid - quarter * 32;
+        const int y0 = p.group_start[g] + m * kBM + quarter * 32;
+        const int x0 = n * kBN + 128 * eg;
+        const uint32_t swz = (uint32_t)((lane >> 1) & 3);
+        if (q_live < 32) {
+          if (live) {
+            float4* dst = reinterpret_cast<float4*>(p.y + grow * p.H + x0);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            dst[j] = make_float4(acc[4 * j + 0], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+            for (int j = 0; j < 32; ++j)
+              dst[j] = make_float4(acc[4 * j + 0], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+          }
+        } else {
+#pragma unroll
+        for (int j = 0; j < 128 / kYCols; ++j) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t dst = ybuf + (uint32_t)lane * (kYCols * 4) + (((uint32_t)c ^ swz) << 4);
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                         "f"(acc[kYCols * j + 4 * c]), "f"(acc[kYCols * j + 4 * c + 1]),
+                         "f"(acc[kYCols * j + 4 * c + 2]), "f"(acc[kYCols * j + 4 * c + 3])
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_y, ybuf, x0 + kYCols * j, y0);
+            bulk_commit();
+          }
+        }
         }
       }
     }
+    if (!kUp && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -347,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <bool kUp>
 cudaError_t launch(const GemmArgs& a, const CUtensorMap& ma, const CUtensorMap& mb,
+                   const CUtensorMap& my,
                    cudaStream_t stream, int sm_count, int64_t tile_bound) {
   static bool configured = false;
   if (!configured) {
@@ -363,7 +403,7 @@ cudaError_t launch(const GemmArgs& a, const CUtensorMap& ma, const CUtensorMap& 
   }
   int grid = sm_count;
   if (tile_bound < grid) grid = (int)(tile_bound > 0 ? tile_bound : 1);
-  grouped_gemm_kernel<kUp><<<grid, kThreads, kDynSmem, stream>>>(ma, mb, a);
+  grouped_gemm_kernel<kUp><<<grid, kThreads, kDynSmem, stream>>>(ma, mb, my, a);
   return cudaGetLastError();
 }
 
@@ -393,16 +433,18 @@ cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const fl
   a.H = gg.H;
   a.status = gg.status;
   const int64_t bound = (gg.rows / kBM + gg.n_groups) * (int64_t)a.n_tiles;
-  return launch<true>(a, ma, mb, stream, sm_count, bound);
+  return launch<true>(a, ma, mb, ma, stream, sm_count, bound);
 }
 
 cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const float* h_s,
                                const uint8_t* w2, const float* s2, float* y,
                                cudaStream_t stream, int sm_count) {
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, my;
   cudaError_t e = make_tmap_u8(&ma, h_q, gg.I, gg.rows, kBK, kBM);
   if (e != cudaSuccess) return e;
   e = make_tmap_u8(&mb, w2, gg.I, (int64_t)gg.n_groups * gg.H, kBK, kBN);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_f32(&my, y, gg.H, gg.rows, kYCols, 32);
   if (e != cudaSuccess) return e;
   GemmArgs a{};
   a.group_rows = gg.group_rows;
@@ -419,7 +461,7 @@ cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const 
   a.H = gg.H;
   a.status = gg.status;
   const int64_t bound = (gg.rows / kBM + gg.n_groups) * (int64_t)a.n_tiles;
-  return launch<false>(a, ma, mb, stream, sm_count, bound);
+  return launch<false>(a, ma, mb, my, stream, sm_count, bound);
 }
 
 }  // namespace moe
