@@ -139,6 +139,41 @@ def algorithmic_work(w, counts: np.ndarray):
     }
 
 
+GEMM_SOURCES = ["mixture_experts_layer_40_b200/csrc/gemm.cu",
+                "mixture_experts_layer_40_b200/csrc/common.cuh"]
+TRAFFIC_FILE = "profiles/grouped_gemm_v3_prefill_dram.md"
+
+
+def gemm_fingerprint() -> str:
+    """Hash of the grouped-GEMM sources: a recorded DRAM capture is only
+    reported while the kernel it measured is unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum of one launch of `kernel`
+    from the committed ncu summary, or None when there is none for this
+    workload or the GEMM sources changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, TRAFFIC_FILE)) as fh:
+            lines = fh.read().splitlines()
+        fp = gemm_fingerprint()
+    except OSError:
+        return None
+    for ln in lines:
+        f = ln.split()
+        if len(f) == 5 and f[0] == "traffic" and f[1] == kernel:
+            kv = dict(x.split("=", 1) for x in f[2:])
+            if kv.get("workload") == workload and kv.get("fingerprint") == fp:
+                return int(kv["bytes"])
+    return None
+
+
 def measure_fp8_peak(torch, device):
     """Dense FP8 E4M3 GEMM throughput of the vendor library (torch._scaled_mm,
     8192^3, per-tensor scales): the measured denominator for the FP8 fraction."""
@@ -271,7 +306,9 @@ def run_ours(args, w, rank, world, local_rank):
     for evs in events:
         for ev in evs:
             ev.record(stream)
-    launches_per_step = 10  # quantise, logits, top-K, scan, scatter, gather, up, down, combine, bias
+    # quantise, split gate, logits, top-K, scan, scatter, gather, up, down,
+    # combine, bias update
+    launches_per_step = 11
 
     def step(traced_events=None, x_in=x):
         if traced_events is None:
@@ -350,6 +387,7 @@ def run_ours(args, w, rank, world, local_rank):
         except Exception:
             fp8_meas = None
     work = algorithmic_work(w, counts)
+    weight_gb = (int(np.count_nonzero(counts)) + 1) * 3 * w.H * w.I / 1e9
     dom = max(stage_ms, key=stage_ms.get)
     gemm_ms = stage_ms["expert_up"] + stage_ms["expert_down"]
     gemm_tflops = (work["expert_up"]["flops"] + work["expert_down"]["flops"]) / (gemm_ms * 1e-3) / 1e12
@@ -364,15 +402,16 @@ def run_ours(args, w, rank, world, local_rank):
         "config": {"workload": f"{w.name}: T={w.T} per GPU, H={w.H}, N={w.N} routed top-{w.K} "
                                f"+ 1 shared, I={w.I}, SwiGLU, FP8 E4M3 1x128/128x128",
                    "tokens_per_gpu": w.T, "parallelism": f"dp{world} (weak: own batch per GPU)",
-                   "l2": "no flush: each step streams 11.3 GB of weights + ~1.9 GB of "
-                         "activations, 100x the 126 MB L2"},
+                   "l2": f"no flush: each step streams {weight_gb:.2f} GB of expert weights, "
+                         f"{weight_gb * 1e3 / 126:.0f}x the 126 MB L2"},
         "gemm": {"tflops": gemm_tflops, "fp8_spec_tflops": FP8_SPEC_TFLOPS,
                  "frac_of_fp8_spec": gemm_tflops / FP8_SPEC_TFLOPS,
                  "fp8_library_tflops_measured": fp8_meas,
                  "frac_of_fp8_measured": (gemm_tflops / fp8_meas) if fp8_meas else None},
         "stages_ms": stage_ms,
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": achieved_gbs / hbm_peak, "traffic": None,
+                     "unit": "GB/s", "frac": achieved_gbs / hbm_peak,
+                     "traffic": recorded_traffic(dom, w.name), "traffic_source": TRAFFIC_FILE,
                      "peak_source": f"{peak_kind} hbm_gbs (copy)",
                      "algorithmic_bytes": work[dom]["bytes"]},
         "gpu_launches": launches_per_step * args.steps,
