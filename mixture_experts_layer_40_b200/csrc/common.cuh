@@ -132,8 +132,9 @@ MOE_DEV void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32
                : "memory");
 }
 MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// the shared-memory sources of this thread's committed stores may be reused
-MOE_DEV void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the shared-memory sources of all but the most recent of this thread's
+// committed stores may be reused
+MOE_DEV void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // this thread's committed stores have completed
 MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 MOE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -154,6 +155,14 @@ MOE_DEV void fma_f32x2(float& a0, float& a1, float v0, float v1, uint64_t s2) {
       "mov.b64 {%0, %1}, rc;\n\t}"
       : "+f"(a0), "+f"(a1)
       : "f"(v0), "f"(v1), "l"(s2));
+}
+
+// Read-only global load issued exactly here: the compiler may not sink it
+// towards its use, so a value fetched one loop iteration ahead arrives in time.
+MOE_DEV float ldg_early(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
 }
 
 MOE_DEV void prefetch_tensormap(const CUtensorMap* map) {

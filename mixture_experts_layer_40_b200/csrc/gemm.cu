@@ -46,11 +46,12 @@ constexpr int kThreads = 384;
 constexpr int kEpiThreads = 256;
 constexpr int kMaxGroups = 1025;
 constexpr uint32_t kIdesc = make_idesc(kBM, kBN, 0u, 0u);  // E4M3 x E4M3 -> fp32
-// down epilogue: each epilogue warp stages 32 rows x 16 fp32 columns of its
-// output tile in shared memory (64-byte swizzle) for one TMA store at a time
-constexpr int kYCols = 16;
+// down epilogue: each epilogue warp stages 32 rows x 8 fp32 columns of its
+// output tile in shared memory (32-byte swizzle), two buffers so that one TMA
+// store is in flight while the next chunk is written
+constexpr int kYCols = 8;
 constexpr int kYBufBytes = 32 * kYCols * 4;
-constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 8 * kYBufBytes + 1024;
+constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 8 * 2 * kYBufBytes + 1024;
 // Register split: launched at kLaunchRegs per thread (384 x 168 = 64512);
 // warpgroup 0 drops to kRegsCtl, the two epilogue warpgroups rise to kRegsEpi.
 // 128 * kRegsCtl + 256 * kRegsEpi must not exceed 384 * kLaunchRegs.
@@ -102,7 +103,10 @@ MOE_DEV void decode_tile(int tile, const int* prefix, int n_groups, int n_tiles,
   n = local - m * n_tiles;
 }
 
-MOE_DEV float silu(float a) { return a / (1.0f + expf(-a)); }
+// silu(a) = a * sigmoid(a) with the hardware exp2 and reciprocal (a few ulp;
+// the accurate library forms made the up GEMM's tile epilogue 6x longer).
+// For a < -88, exp(-a) is +inf and the quotient is -0.
+MOE_DEV float silu(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
 template <bool kUp>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t ybuf = ring + (uint32_t)(kStages * kStageBytes + ew * kYBufBytes);
+    const uint32_t ybuf = ring + (uint32_t)(kStages * kStageBytes + ew * 2 * kYBufBytes);
     const int b_blocks = p.b_rows / kBM;
     int kbi = 0;
     uint32_t xchg_phase = 0;
@@ -256,19 +260,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* sb1 = p.b_s + ((int64_t)g * b_blocks + 2 * n + 1) * kb_n;
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-      float sa_next = __ldg(sa_ptr);
-      float sb0_next = __ldg(sb0);
-      float sb1_next = kUp ? __ldg(sb1) : 0.0f;
+      float sa_next = ldg_early(sa_ptr);
+      float sb0_next = ldg_early(sb0);
+      float sb1_next = kUp ? ldg_early(sb1) : 0.0f;
       bool ok = true;
       for (int kb = 0; kb < kb_n; ++kb, ++kbi) {
         const float sa = sa_next, s0 = sb0_next, s1 = sb1_next;
         if (kb + 1 < kb_n) {
-          sa_next = __ldg(sa_ptr + kb + 1);
-          sb0_next = __ldg(sb0 + kb + 1);
-          if (kUp) sb1_next = __ldg(sb1 + kb + 1);
+          sa_next = ldg_early(sa_ptr + kb + 1);
+          sb0_next = ldg_early(sb0 + kb + 1);
+          if (kUp) sb1_next = ldg_early(sb1 + kb + 1);
         }
-        const float inv0 = 1.0f / (sa * s0);
-        const float inv1 = kUp ? 1.0f / (sa * s1) : inv0;
+        // 1/(s_a s_b) with the hardware reciprocal (<= 2 ulp)
+        const float inv0 = __fdividef(1.0f, sa * s0);
+        const float inv1 = kUp ? __fdividef(1.0f, sa * s1) : inv0;
         const uint64_t inv0x2 = splat_f32x2(inv0), inv1x2 = splat_f32x2(inv1);
         const int buf = kbi & 1;
         // the result is made warp-uniform: tcgen05.ld below is warp-collective
@@ -337,14 +342,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (eg == 0) p.h_s[grow * (p.I / kBM) + n] = s;
         }
       } else {
-        // fp32 rows out through shared memory and TMA stores, 16 columns of
+        // fp32 rows out through shared memory and TMA stores, 8 columns of
         // the warp's 32 rows at a time, when all 32 rows belong to the group;
         // a group's last, partial 32 rows are stored directly, row by row,
         // and padding rows are never written
         const int q_live = valid - quarter * 32;
         const int y0 = p.group_start[g] + m * kBM + quarter * 32;
         const int x0 = n * kBN + 128 * eg;
-        const uint32_t swz = (uint32_t)((lane >> 1) & 3);
+        const uint32_t swz = (uint32_t)((lane >> 2) & 1);
         if (q_live < 32) {
           if (live) {
             float4* dst = reinterpret_cast<float4*>(p.y + grow * p.H + x0);
@@ -355,11 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
         for (int j = 0; j < 128 / kYCols; ++j) {
-          if (lane == 0) bulk_wait_read_all();
+          const uint32_t buf_j = ybuf + (uint32_t)((j & 1) * kYBufBytes);
+          // the store that last read this buffer (two chunks ago) is done
+          if (lane == 0) bulk_wait_read_1();
           __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t dst = ybuf + (uint32_t)lane * (kYCols * 4) + (((uint32_t)c ^ swz) << 4);
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t dst = buf_j + (uint32_t)lane * (kYCols * 4) + (((uint32_t)c ^ swz) << 4);
             asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
                          "f"(acc[kYCols * j + 4 * c]), "f"(acc[kYCols * j + 4 * c + 1]),
                          "f"(acc[kYCols * j + 4 * c + 2]), "f"(acc[kYCols * j + 4 * c + 3])
@@ -368,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tm_y, ybuf, x0 + kYCols * j, y0);
+            tma_store_2d(&tm_y, buf_j, x0 + kYCols * j, y0);
             bulk_commit();
           }
         }

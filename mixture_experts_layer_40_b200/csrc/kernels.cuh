@@ -21,7 +21,8 @@ cudaError_t make_tmap_u8(CUtensorMap* map, const void* base, int64_t inner, int6
                          int box_inner, int box_rows);
 // bf16 tensor map over [depth, rows, inner] (depth 1: 2-D), box of box_inner
 // elements x box_rows rows x 1, 128-byte swizzle (host side).
-// fp32 [rows, inner] row-major, 64-byte swizzle (box_inner * 4 must be 64)
+// fp32 [rows, inner] row-major; the swizzle span is the box row (box_inner * 4
+// bytes: 32, 64 or 128)
 cudaError_t make_tmap_f32(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
                           int box_inner, int box_rows);
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
