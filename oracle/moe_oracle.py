@@ -16,7 +16,8 @@ Sources (web pages on the DeepSeek-V3 technical report), cited by tag:
                (trishampatil.com); section III (routing equations, bias
                controller) and section V (FP8 details).
   [Deepforge]  "DeepSeek-V3 Technical Report" (deepforge.srivtx.xyz);
-               "Per-tile FP8 scaling" and "Build it yourself".
+               "Per-tile FP8 scaling", "Balancing without a balance loss"
+               and "Build it yourself".
 
 Readings taken where the pages are silent (each is listed in the design
 notes with its reason):
@@ -31,6 +32,11 @@ notes with its reason):
     BF16 result. The combine sums in float64, shared expert first, then
     routed experts by ascending id.
   * No residual add; no routed scaling factor.
+  * Node-limited routing ranks groups by the sum of their K/M highest
+    *biased* scores (the selection side, as [Deepforge] ranks experts by
+    s_i + b_i; [Explained] says "affinities"); group ties go to the lower id.
+  * Sequence balance statistics: f_i is the load normalised so a perfectly
+    even split gives 1; P_i averages s_i / sum_j s_j over the sequence.
 
 parity pins: every function here is pinned by a test under tests/ against a
 closed form, a worked example, an invariant, a library routine or brute
@@ -198,6 +204,65 @@ def route(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int):
     sel = np.take_along_axis(s, ids, axis=1)
     gates = sel / np.sum(sel, axis=1, keepdims=True)
     return ids, gates, s, score
+
+
+def route_grouped(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int,
+                  n_groups: int, topk_groups: int):
+    """Node-limited routing ([Explained] recipe step 5; [Deepforge]
+    "Balancing without a balance loss"): the N routed experts are split into
+    n_groups contiguous groups (the nodes that hold them); a group's score is
+    the sum of its k / topk_groups highest biased scores s_i + b_i; only the
+    topk_groups best groups are eligible (ties to the lower group id), and
+    the K experts are the biased top-K among the eligible ones, as in route().
+
+    Returns (ids, gates, s, score, group_score [T, n_groups]).
+    """
+    s = sigmoid(gate_logits(x, gate_w))
+    score = s + np.asarray(bias, np.float32).astype(np.float64)
+    t_count, n = score.shape
+    size, per_group = n // n_groups, k // topk_groups
+    assert size * n_groups == n and per_group * topk_groups == k and per_group <= size
+    grouped = score.reshape(t_count, n_groups, size)
+    best = -np.sort(-grouped, axis=2)[:, :, :per_group]
+    group_score = best.sum(axis=2)
+    chosen = np.argsort(-group_score, axis=1, kind="stable")[:, :topk_groups]
+    eligible = np.zeros((t_count, n_groups), dtype=bool)
+    np.put_along_axis(eligible, chosen, True, axis=1)
+    masked = np.where(np.repeat(eligible, size, axis=1), score, -np.inf)
+    order = np.argsort(-masked, axis=1, kind="stable")
+    ids = order[:, :k].astype(np.int32)
+    sel = np.take_along_axis(s, ids, axis=1)
+    gates = sel / np.sum(sel, axis=1, keepdims=True)
+    return ids, gates, s, score, group_score
+
+
+def balance_stats(s: np.ndarray, ids: np.ndarray, k: int, seq_len: int, alpha: float):
+    """Complementary sequence-wise balance statistics ([Dissection] section
+    III, "a complementary sequence-wise balance loss", and [Explained] recipe
+    step 4): over the tokens of each sequence (consecutive runs of seq_len
+    tokens; the last may be shorter),
+      f_i = N / (K * T_seq) * #{(t, k): ids[t, k] = i}   (normalised load)
+      P_i = (1 / T_seq) * sum_t s[t, i] / sum_j s[t, j]  (mean gate mass)
+      L   = alpha * sum_i f_i * P_i.
+    s are the unbiased affinities of all N routed experts.
+
+    Returns f [S, N], P [S, N], loss [S] in float64.
+    """
+    s = np.asarray(s, np.float64)
+    ids = np.asarray(ids)
+    t_count, n = s.shape
+    n_seq = -(-t_count // seq_len)
+    f = np.zeros((n_seq, n))
+    p = np.zeros((n_seq, n))
+    loss = np.zeros(n_seq)
+    for q in range(n_seq):
+        lo, hi = q * seq_len, min(t_count, (q + 1) * seq_len)
+        t_seq = hi - lo
+        counts = np.bincount(ids[lo:hi].ravel(), minlength=n)
+        f[q] = n * counts / (k * t_seq)
+        p[q] = np.sum(s[lo:hi] / np.sum(s[lo:hi], axis=1, keepdims=True), axis=0) / t_seq
+        loss[q] = alpha * np.sum(f[q] * p[q])
+    return f, p, loss
 
 
 def expert_counts(ids: np.ndarray, n_experts: int) -> np.ndarray:
