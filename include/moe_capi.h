@@ -59,9 +59,19 @@ typedef enum {
  * expert has the routed experts' shape, "DeepSeek-V3, explained", step 3).
  * Supported: T >= 1; H a multiple of 256; I a multiple of 128; N a multiple
  * of 16 with 16 <= N <= 1024; 1 <= K <= min(N, 16).
+ *
+ * G, M: node-limited routing ("DeepSeek-V3, explained", recipe step 5;
+ * "DeepSeek-V3 Technical Report" (deepforge.srivtx.xyz), "Balancing without
+ * a balance loss"). The routed experts form G contiguous groups of N/G (the
+ * nodes holding them); a token's group score is the sum of its K/M highest
+ * biased scores s_i + b_i inside the group, and its K experts are chosen only
+ * from its M best groups (ties to the lower group id). G = 0 (or G = M)
+ * routes over all N experts. Otherwise: 1 <= M <= G <= 32, N % G == 0,
+ * K % M == 0 and K/M <= N/G.
  */
 typedef struct {
   int32_t T, H, N, K, I;
+  int32_t G, M;
 } moe_shape;
 
 /*
@@ -183,6 +193,26 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
 #define MOE_ROUTE_NOALLOC_MAX_LOGITS 1048576
 int moe_route_noalloc(moe_shape sh, const float* gate_w, const void* x, const float* bias,
                       int32_t* topk_ids, float* topk_gates, int32_t* counts, void* stream);
+
+/*
+ * Complementary sequence-wise balance statistics ("DeepSeek-V3:
+ * Auxiliary-Loss-Free MoE Load Balancing, Multi-Token Prediction, and FP8
+ * Training at 671B Scale", section III; "DeepSeek-V3, explained", step 4),
+ * for the routing that the last moe_route or moe_forward call on `ws` made.
+ * The T tokens form S = ceil(T / seq_len) sequences of seq_len consecutive
+ * tokens (the last may be shorter, T_s tokens). For sequence s and expert i:
+ *   f[s, i] = N / (K * T_s) * #{(t, k) in s : topk_ids[t, k] = i}
+ *   P[s, i] = (1 / T_s) * sum_{t in s} s_ti / sum_j s_tj   (all N affinities)
+ *   loss[s] = alpha * sum_i f[s, i] * P[s, i]
+ * with s_ti the router's sigmoid affinities (recomputed from the logits the
+ * router left in ws). Sums run in a fixed order: results are reproducible.
+ *   topk_ids: int32 [T, K] of that call; f, P: float [S, N]; loss: float [S]
+ * Errors: MOE_ERR_SHAPE for a bad shape or seq_len < 1; MOE_ERR_NULL;
+ * MOE_ERR_WORKSPACE if ws_bytes < moe_workspace_size(sh).
+ */
+int moe_balance_stats(moe_shape sh, int32_t seq_len, float alpha, const void* ws,
+                      size_t ws_bytes, const int32_t* topk_ids, float* f, float* P, float* loss,
+                      void* stream);
 
 /*
  * The whole layer forward: quantise x (1x128), route, permute token rows by

@@ -30,7 +30,8 @@ class MoeError(RuntimeError):
 
 class moe_shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
-                ("K", ctypes.c_int32), ("I", ctypes.c_int32)]
+                ("K", ctypes.c_int32), ("I", ctypes.c_int32), ("G", ctypes.c_int32),
+                ("M", ctypes.c_int32)]
 
 
 class moe_weights(ctypes.Structure):
@@ -58,6 +59,8 @@ SIGNATURES = {
     "moe_workspace_layout": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_ws_layout)]),
     "moe_route": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_route_noalloc": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_balance_stats": (ctypes.c_int, [moe_shape, ctypes.c_int32, ctypes.c_float, _P, _SZ, _P,
+                                         _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P, _P, _P,
                                    _P, _SZ, _P]),
     "moe_forward_traced": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P,
@@ -108,8 +111,9 @@ def _stream(stream=None):
     return s.cuda_stream
 
 
-def shape_of(T: int, H: int, N: int, K: int, I: int) -> moe_shape:
-    return moe_shape(T, H, N, K, I)
+def shape_of(T: int, H: int, N: int, K: int, I: int, G: int = 0, M: int = 0) -> moe_shape:
+    """G, M: node-limited routing over G expert groups, M per token (G = 0: off)."""
+    return moe_shape(T, H, N, K, I, G, M)
 
 
 def moe_quantize_1x128(x: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, stream=None):
@@ -142,6 +146,16 @@ def moe_route(sh: moe_shape, gate_w, x, bias, topk_ids, topk_gates, counts, ws, 
         _ptr(bias, torch.float32, "bias"), _ptr(topk_ids, torch.int32, "topk_ids"),
         _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_balance_stats(sh: moe_shape, seq_len: int, alpha: float, ws, topk_ids, f, P, loss,
+                      stream=None):
+    """Sequence-wise balance statistics of the routing the last moe_route /
+    moe_forward on `ws` made: f, P float [S, N], loss float [S]."""
+    _check("moe_balance_stats", LIB.moe_balance_stats(
+        sh, seq_len, alpha, _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _ptr(topk_ids, torch.int32, "topk_ids"), _ptr(f, torch.float32, "f"),
+        _ptr(P, torch.float32, "P"), _ptr(loss, torch.float32, "loss"), _stream(stream)))
 
 
 ROUTE_NOALLOC_MAX_LOGITS = 1048576

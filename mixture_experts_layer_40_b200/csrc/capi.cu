@@ -43,11 +43,6 @@ int sm_count() {
 inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-bool shape_ok(const moe_shape& s) {
-  return s.T >= 1 && s.H >= 256 && s.H % 256 == 0 && s.I >= 128 && s.I % 128 == 0 && s.N >= 16 &&
-         s.N <= 1024 && s.N % 16 == 0 && s.K >= 1 && s.K <= s.N && s.K <= 16 &&
-         (int64_t)s.T * s.K < (1ll << 31) && (int64_t)s.T * s.N < (1ll << 31);
-}
 
 void layout_of(const moe_shape& s, moe_ws_layout* L) {
   const int64_t T = s.T, H = s.H, N = s.N, K = s.K, I = s.I;
@@ -86,6 +81,14 @@ T* at(void* ws, size_t off) {
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 }  // namespace
+
+bool shape_ok(const moe_shape& s) {
+  return s.T >= 1 && s.H >= 256 && s.H % 256 == 0 && s.I >= 128 && s.I % 128 == 0 && s.N >= 16 &&
+         s.N <= 1024 && s.N % 16 == 0 && s.K >= 1 && s.K <= s.N && s.K <= 16 &&
+         (int64_t)s.T * s.K < (1ll << 31) && (int64_t)s.T * s.N < (1ll << 31) &&
+         (s.G == 0 || (s.G >= 1 && s.G <= 32 && s.N % s.G == 0 && s.M >= 1 && s.M <= s.G &&
+                       s.K % s.M == 0 && s.K / s.M <= s.N / s.G));
+}
 
 cudaError_t make_tmap_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
                          int box_inner, int box_rows) {
@@ -193,10 +196,24 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
   cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
   if (e == cudaSuccess)
-    e = launch_router_tc(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K,
+    e = launch_router_tc(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                          at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), topk_ids,
                          topk_gates, counts, status, s, sm_count());
   return cuda_status(e);
+}
+
+int moe_balance_stats(moe_shape sh, int32_t seq_len, float alpha, const void* ws,
+                      size_t ws_bytes, const int32_t* topk_ids, float* f, float* P, float* loss,
+                      void* stream) {
+  if (!shape_ok(sh) || seq_len < 1) return MOE_ERR_SHAPE;
+  if (!ws || !topk_ids || !f || !P || !loss) return MOE_ERR_NULL;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
+  moe_ws_layout L;
+  layout_of(sh, &L);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_balance_stats(at<float>(const_cast<void*>(ws), L.logits), topk_ids,
+                                          sh.T, sh.N, sh.K, seq_len, alpha, f, P, loss,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const float* bias,
@@ -237,7 +254,7 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   e = mark(1, e);
   // a2-a5: gate logits, sigmoid, biased top-K, gates, counts
   if (e == cudaSuccess)
-    e = launch_router_tc(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K,
+    e = launch_router_tc(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                          at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
                          counts, status, s, sms);
   e = mark(2, e);

@@ -38,7 +38,7 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBK = 128;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;
 constexpr int kABytes = kBM * kBK;
 constexpr int kBBytes = kBN * kBK;
 constexpr int kStageBytes = kABytes + kBBytes;
@@ -46,12 +46,26 @@ constexpr int kThreads = 384;
 constexpr int kEpiThreads = 256;
 constexpr int kMaxGroups = 1025;
 constexpr uint32_t kIdesc = make_idesc(kBM, kBN, 0u, 0u);  // E4M3 x E4M3 -> fp32
-// down epilogue: each epilogue warp stages 32 rows x 8 fp32 columns of its
-// output tile in shared memory (32-byte swizzle), two buffers so that one TMA
-// store is in flight while the next chunk is written
-constexpr int kYCols = 8;
+// down epilogue: each epilogue warp stages 32 rows x kYCols fp32 columns of
+// its output tile in shared memory (swizzled over the 128-byte box row), two
+// buffers so that one TMA store is in flight while the next chunk is written
+#ifndef MOE_YCOLS
+#define MOE_YCOLS 32
+#endif
+#ifndef MOE_DOWN_STAGES
+#define MOE_DOWN_STAGES 3
+#endif
+constexpr int kYCols = MOE_YCOLS;
 constexpr int kYBufBytes = 32 * kYCols * 4;
-constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 8 * 2 * kYBufBytes + 1024;
+// the up GEMM (56 k-blocks per tile at H = 7168) keeps a 4-stage ring; the
+// down GEMM gives one stage to the output staging buffers
+template <bool kUp>
+struct Cfg {
+  static constexpr int stages = kUp ? kMaxStages : MOE_DOWN_STAGES;
+  static constexpr size_t dyn_smem =
+      (size_t)stages * kStageBytes + (kUp ? 0 : 8 * 2 * kYBufBytes) + 1024;
+};
+static_assert(Cfg<false>::dyn_smem + 8192 <= 232448, "shared memory");
 // Register split: launched at kLaunchRegs per thread (384 x 168 = 64512);
 // warpgroup 0 drops to kRegsCtl, the two epilogue warpgroups rise to kRegsEpi.
 // 128 * kRegsCtl + 256 * kRegsEpi must not exceed 384 * kLaunchRegs.
@@ -79,8 +93,8 @@ struct GemmArgs {
 };
 
 struct alignas(8) GemmShared {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t xchg;           // amax exchange between the two epilogue groups
@@ -113,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
+  constexpr int kSt = Cfg<kUp>::stages;
   __shared__ GemmShared sh;
   extern __shared__ uint8_t dyn_smem[];
   const uint32_t ring = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -120,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(smem_u32(&sh.full[s]), 1);
       mbar_init(smem_u32(&sh.empty[s]), 1);
     }
@@ -186,8 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int a_row = p.group_start[g] + m * kBM;
         const int b_row = g * p.b_rows + n * kBN;
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          const int s = it % kSt;
+          const uint32_t ph = (uint32_t)(it / kSt) & 1u;
           if (!mbar_wait(smem_u32(&sh.empty[s]), ph ^ 1u, abort, p.status)) { ok = false; break; }
           const uint32_t full = smem_u32(&sh.full[s]);
           mbar_arrive_expect_tx(full, kStageBytes);
@@ -198,9 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // drain: every armed stage must land before the CTA may exit
-        for (int s = 0; s < kStages && s < it; ++s) {
-          const int last = s + ((it - 1 - s) / kStages) * kStages;
-          mbar_wait(smem_u32(&sh.full[s]), (uint32_t)(last / kStages) & 1u, nullptr, p.status);
+        for (int s = 0; s < kSt && s < it; ++s) {
+          const int last = s + ((it - 1 - s) / kSt) * kSt;
+          mbar_wait(smem_u32(&sh.full[s]), (uint32_t)(last / kSt) & 1u, nullptr, p.status);
         }
       }
     }
@@ -215,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t use = (uint32_t)(kbi >> 1);
           if (!mbar_wait(smem_u32(&sh.tempty[buf]), (use & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
           tc_fence_after();
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          const int s = it % kSt;
+          const uint32_t ph = (uint32_t)(it / kSt) & 1u;
           if (!mbar_wait(smem_u32(&sh.full[s]), ph, abort, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = ring + s * kStageBytes;
@@ -243,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t ybuf = ring + (uint32_t)(kStages * kStageBytes + ew * 2 * kYBufBytes);
+    const uint32_t ybuf = ring + (uint32_t)(kSt * kStageBytes + ew * 2 * kYBufBytes);
     const int b_blocks = p.b_rows / kBM;
     int kbi = 0;
     uint32_t xchg_phase = 0;
@@ -349,7 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q_live = valid - quarter * 32;
         const int y0 = p.group_start[g] + m * kBM + quarter * 32;
         const int x0 = n * kBN + 128 * eg;
-        const uint32_t swz = (uint32_t)((lane >> 2) & 1);
+        // 128-byte-span swizzle: 16-byte chunk c of row r sits at c ^ (r / rows
+        // per 128 bytes) within the row (32-, 64- and 128-byte modes alike)
+        constexpr int kChunks = kYCols / 4;
+        const uint32_t swz = (uint32_t)((lane / (32 / kYCols)) & (kChunks - 1));
         if (q_live < 32) {
           if (live) {
             float4* dst = reinterpret_cast<float4*>(p.y + grow * p.H + x0);
@@ -365,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) bulk_wait_read_1();
           __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < kChunks; ++c) {
             const uint32_t dst = buf_j + (uint32_t)lane * (kYCols * 4) + (((uint32_t)c ^ swz) << 4);
             asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
                          "f"(acc[kYCols * j + 4 * c]), "f"(acc[kYCols * j + 4 * c + 1]),
@@ -404,13 +422,13 @@ cudaError_t launch(const GemmArgs& a, const CUtensorMap& ma, const CUtensorMap& 
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(grouped_gemm_kernel<kUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kDynSmem);
+                             (int)Cfg<kUp>::dyn_smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   int grid = sm_count;
   if (tile_bound < grid) grid = (int)(tile_bound > 0 ? tile_bound : 1);
-  grouped_gemm_kernel<kUp><<<grid, kThreads, kDynSmem, stream>>>(ma, mb, my, a);
+  grouped_gemm_kernel<kUp><<<grid, kThreads, Cfg<kUp>::dyn_smem, stream>>>(ma, mb, my, a);
   return cudaGetLastError();
 }
 

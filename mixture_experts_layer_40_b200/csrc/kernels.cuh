@@ -28,25 +28,35 @@ cudaError_t make_tmap_f32(CUtensorMap* map, const void* base, int64_t inner, int
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
                            int64_t depth, int box_inner, int box_rows);
 
+// The sizes every entry point accepts (see moe_shape in moe_capi.h).
+bool shape_ok(const moe_shape& s);
+
 cudaError_t launch_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q,
                                   float* scales, cudaStream_t stream, int sm_count);
 cudaError_t launch_quantize_128x128(const float* w, int64_t rows, int64_t cols, uint8_t* q,
                                     float* scales, cudaStream_t stream);
 
-// Router: gate logits (fp32 SIMT GEMM), then sigmoid, biased top-K, gates and
-// counts (counts must be zero on entry).
+// Router: gate logits (fp32 SIMT GEMM), then sigmoid, biased top-K (node-
+// limited to the M best of G expert groups when G > 1), gates and counts
+// (counts must be zero on entry).
 cudaError_t launch_router(const void* x, const float* gate_w, const float* bias, int T, int H,
-                          int N, int K, float* logits, int32_t* ids, float* gates, int32_t* counts,
-                          uint32_t* status, cudaStream_t stream, int sm_count);
+                          int N, int K, int G, int M, float* logits, int32_t* ids, float* gates,
+                          int32_t* counts, uint32_t* status, cudaStream_t stream, int sm_count);
 
 // Router on tensor cores: splits the fp32 centroids into three bf16 terms in
 // `wsplit` (router_split_bytes), computes the logits with BF16 tcgen05 MMAs
 // and fp32 accumulation, then the same top-K as launch_router.
 size_t router_split_bytes(int N, int H);
 cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
-                             int N, int K, __nv_bfloat16* wsplit, float* logits, int32_t* ids,
-                             float* gates, int32_t* counts, uint32_t* status, cudaStream_t stream,
-                             int sm_count);
+                             int N, int K, int G, int M, __nv_bfloat16* wsplit, float* logits,
+                             int32_t* ids, float* gates, int32_t* counts, uint32_t* status,
+                             cudaStream_t stream, int sm_count);
+
+// Sequence-wise balance statistics from the router's logits and top-K ids:
+// one CTA per sequence of seq_len tokens; f, P [S, N], loss [S].
+cudaError_t launch_balance_stats(const float* logits, const int32_t* ids, int T, int N, int K,
+                                 int seq_len, float alpha, float* f, float* P, float* loss,
+                                 cudaStream_t stream);
 
 // Permutation: scan of counts into group tables, stable scatter, row gather.
 cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K, int H,

@@ -51,11 +51,6 @@ int current_sm_count() {
   return n;
 }
 
-bool route_shape_ok(const moe_shape& s) {
-  return s.T >= 1 && s.H >= 256 && s.H % 256 == 0 && s.I >= 128 && s.I % 128 == 0 && s.N >= 16 &&
-         s.N <= 1024 && s.N % 16 == 0 && s.K >= 1 && s.K <= s.N && s.K <= 16;
-}
-
 }  // namespace
 }  // namespace moe
 
@@ -63,7 +58,7 @@ extern "C" int moe_route_noalloc(moe_shape sh, const float* gate_w, const void* 
                                  const float* bias, int32_t* topk_ids, float* topk_gates,
                                  int32_t* counts, void* stream) {
   using namespace moe;
-  if (!route_shape_ok(sh)) return MOE_ERR_SHAPE;
+  if (!shape_ok(sh)) return MOE_ERR_SHAPE;
   if ((int64_t)sh.T * sh.N > (int64_t)MOE_ROUTE_NOALLOC_MAX_LOGITS) return MOE_ERR_WORKSPACE;
   if (!gate_w || !x || !bias || !topk_ids || !topk_gates || !counts) return MOE_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(x) % 16) != 0 || (reinterpret_cast<uintptr_t>(gate_w) % 16) != 0)
@@ -73,7 +68,7 @@ extern "C" int moe_route_noalloc(moe_shape sh, const float* gate_w, const void* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)sh.N * sizeof(int32_t), s);
   if (e == cudaSuccess)
-    e = launch_router(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, scratch, topk_ids, topk_gates,
-                      counts, nullptr, s, current_sm_count());
+    e = launch_router(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M, scratch, topk_ids,
+                      topk_gates, counts, nullptr, s, current_sm_count());
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -81,12 +81,31 @@ __global__ void __launch_bounds__(256) logits_kernel(const __nv_bfloat16* __rest
 
 constexpr int kMaxPerLane = 32;  // N <= 1024
 
+// Warp arg-max of (score, id) pairs: the highest score, the lower id on ties.
+MOE_DEV void warp_argmax(float& best, int& bid) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bid, o);
+    if (ob > best || (ob == best && oi < bid)) {
+      best = ob;
+      bid = oi;
+    }
+  }
+}
+
 // One warp per token: sigmoid, biased scores, K rounds of a warp arg-max
 // (highest score, lower id on ties), gates from the unbiased affinities,
 // counts by integer atomics (exact, order-independent).
+// Node-limited routing (G > 1, "DeepSeek-V3, explained", recipe step 5):
+// before the K rounds, each of the G contiguous expert groups is scored by
+// the sum of its K/M highest biased scores (taken in descending order), the
+// M best groups are kept (lower group id on ties) and every expert outside
+// them is masked out of the selection.
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
                                                    const float* __restrict__ bias, int T, int N,
-                                                   int K, int32_t* __restrict__ ids,
+                                                   int K, int G, int M,
+                                                   int32_t* __restrict__ ids,
                                                    float* __restrict__ gates,
                                                    int32_t* __restrict__ counts) {
   const int lane = threadIdx.x & 31;
@@ -104,6 +123,46 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
         const float v = s + bias[e];
         sv[j] = s;
         sc[j] = (v == v) ? v : -INFINITY;
+      }
+    }
+    if (G > 1 && M < G) {
+      const int size = N / G, per_group = K / M;
+      float my_group_score = -INFINITY;  // lane g holds group g's score
+      for (int g = 0; g < G; ++g) {
+        uint32_t used = 0;
+        float gsum = 0.0f;
+        for (int r = 0; r < per_group; ++r) {
+          float best = -INFINITY;
+          int bid = N, bj = -1;
+#pragma unroll
+          for (int j = 0; j < kMaxPerLane; ++j) {
+            const int e = lane + 32 * j;
+            if (j < per_lane && e < N && e / size == g && !((used >> j) & 1u) &&
+                (sc[j] > best || (sc[j] == best && e < bid))) {
+              best = sc[j];
+              bid = e;
+              bj = j;
+            }
+          }
+          const int own = bid;
+          warp_argmax(best, bid);
+          if (bid == own && bj >= 0) used |= 1u << bj;
+          gsum += best;
+        }
+        if (lane == g) my_group_score = gsum;
+      }
+      uint32_t keep = 0;  // warp-uniform mask of the eligible groups
+      for (int r = 0; r < M; ++r) {
+        float best = (lane < G && !((keep >> lane) & 1u)) ? my_group_score : -INFINITY;
+        int bid = lane < G ? lane : 32;
+        if ((keep >> lane) & 1u) bid = 32;
+        warp_argmax(best, bid);
+        keep |= 1u << bid;
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxPerLane; ++j) {
+        const int e = lane + 32 * j;
+        if (j < per_lane && e < N && !((keep >> (e / size)) & 1u)) sc[j] = -INFINITY;
       }
     }
     uint32_t taken = 0;
@@ -149,11 +208,102 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
   }
 }
 
+// Sequence-wise balance statistics, one CTA of 16 warps per sequence. Warp w
+// takes the sequence's tokens w, w + 16, ...; for each, the lanes recompute
+// the affinities exactly as topk_kernel does, reduce their sum with a fixed
+// butterfly and add s_ti / sum_j s_tj into per-lane partials. The warps'
+// partials are then added in warp order, and the counts come from integer
+// atomics: every result is independent of scheduling.
+constexpr int kBalWarps = 16;
+__global__ void __launch_bounds__(kBalWarps * 32) balance_stats_kernel(const float* __restrict__ z,
+                                                             const int32_t* __restrict__ ids,
+                                                             int T, int N, int K, int seq_len,
+                                                             float alpha, float* __restrict__ f,
+                                                             float* __restrict__ P,
+                                                             float* __restrict__ loss) {
+  __shared__ int cnt[1024];
+  __shared__ float red[kBalWarps][33];
+  __shared__ float fp_part[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int q = blockIdx.x;
+  const int lo = q * seq_len;
+  const int hi = min(T, lo + seq_len);
+  const int t_seq = hi - lo;
+  const int per_lane = (N + 31) >> 5;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  for (int i = lo * K + threadIdx.x; i < hi * K; i += blockDim.x) {
+    const int e = ids[i];
+    if (e >= 0 && e < N) atomicAdd(&cnt[e], 1);
+  }
+  float acc[kMaxPerLane];
+#pragma unroll
+  for (int j = 0; j < kMaxPerLane; ++j) acc[j] = 0.0f;
+  for (int t = lo + warp; t < hi; t += kBalWarps) {
+    float sv[kMaxPerLane];
+    float part = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kMaxPerLane; ++j) {
+      const int e = lane + 32 * j;
+      sv[j] = 0.0f;
+      if (j < per_lane && e < N) {
+        sv[j] = 1.0f / (1.0f + expf(-z[(int64_t)t * N + e]));
+        part += sv[j];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+#pragma unroll
+    for (int j = 0; j < kMaxPerLane; ++j)
+      if (j < per_lane) acc[j] += sv[j] / part;
+  }
+  __syncthreads();
+  float fp_lane = 0.0f;  // lane's share of sum_i f_i P_i (warp 0)
+#pragma unroll
+  for (int j = 0; j < kMaxPerLane; ++j) {
+    if (j >= per_lane) break;  // CTA-uniform
+    red[warp][lane] = acc[j];
+    __syncthreads();
+    if (warp == 0) {
+      float sum = 0.0f;
+      for (int w = 0; w < kBalWarps; ++w) sum += red[w][lane];
+      const int e = lane + 32 * j;
+      if (e < N) {
+        const float pi = sum / (float)t_seq;
+        const float fi = (float)N * (float)cnt[e] / ((float)K * (float)t_seq);
+        P[(int64_t)q * N + e] = pi;
+        f[(int64_t)q * N + e] = fi;
+        fp_lane += fi * pi;
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    fp_part[lane] = fp_lane;
+    __syncwarp();
+    if (lane == 0) {
+      float sum = 0.0f;
+      for (int l = 0; l < 32; ++l) sum += fp_part[l];
+      loss[q] = alpha * sum;
+    }
+  }
+}
+
 }  // namespace
 
+cudaError_t launch_balance_stats(const float* logits, const int32_t* ids, int T, int N, int K,
+                                 int seq_len, float alpha, float* f, float* P, float* loss,
+                                 cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const int n_seq = (T + seq_len - 1) / seq_len;
+  balance_stats_kernel<<<n_seq, kBalWarps * 32, 0, stream>>>(logits, ids, T, N, K, seq_len, alpha, f, P,
+                                                   loss);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router(const void* x, const float* gate_w, const float* bias, int T, int H,
-                          int N, int K, float* logits, int32_t* ids, float* gates, int32_t* counts,
-                          uint32_t* status, cudaStream_t stream, int sm_count) {
+                          int N, int K, int G, int M, float* logits, int32_t* ids, float* gates,
+                          int32_t* counts, uint32_t* status, cudaStream_t stream, int sm_count) {
   (void)status;
   if (T == 0) return cudaSuccess;
   dim3 g1((T + kLT - 1) / kLT, (N + kLE - 1) / kLE);
@@ -163,7 +313,7 @@ cudaError_t launch_router(const void* x, const float* gate_w, const float* bias,
   if (e != cudaSuccess) return e;
   int blocks = (T + 7) / 8;
   if (blocks > sm_count * 8) blocks = sm_count * 8;
-  topk_kernel<<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, ids, gates, counts);
+  topk_kernel<<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, G, M, ids, gates, counts);
   return cudaGetLastError();
 }
 
@@ -337,9 +487,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
 size_t router_split_bytes(int N, int H) { return (size_t)3 * N * H * sizeof(__nv_bfloat16); }
 
 cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
-                             int N, int K, __nv_bfloat16* wsplit, float* logits, int32_t* ids,
-                             float* gates, int32_t* counts, uint32_t* status, cudaStream_t stream,
-                             int sm_count) {
+                             int N, int K, int G, int M, __nv_bfloat16* wsplit, float* logits,
+                             int32_t* ids, float* gates, int32_t* counts, uint32_t* status,
+                             cudaStream_t stream, int sm_count) {
   if (T == 0) return cudaSuccess;
   const int64_t nw = (int64_t)N * H;
   split_gate_kernel<<<(unsigned)std::min<int64_t>((nw + 255) / 256, (int64_t)sm_count * 8), 256, 0,
@@ -364,7 +514,7 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
   if (e != cudaSuccess) return e;
   int blocks = (T + 7) / 8;
   if (blocks > sm_count * 8) blocks = sm_count * 8;
-  topk_kernel<<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, ids, gates, counts);
+  topk_kernel<<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, G, M, ids, gates, counts);
   return cudaGetLastError();
 }
 

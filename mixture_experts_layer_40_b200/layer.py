@@ -70,12 +70,13 @@ class MoELayer:
     """One layer: forward(x, bias) -> y through moe_forward."""
 
     def __init__(self, T: int, H: int, N: int, K: int, I: int, weights: DeviceWeights,
-                 device="cuda"):
+                 device="cuda", groups: int = 0, topk_groups: int = 0):
         self.T, self.H, self.N, self.K, self.I = T, H, N, K, I
-        self.shape = capi.shape_of(T, H, N, K, I)
+        self.shape = capi.shape_of(T, H, N, K, I, groups, topk_groups)
         nbytes = capi.moe_workspace_size(self.shape)
         if nbytes == 0:
-            raise ValueError(f"unsupported shape T={T} H={H} N={N} K={K} I={I}")
+            raise ValueError(f"unsupported shape T={T} H={H} N={N} K={K} I={I} "
+                             f"G={groups} M={topk_groups}")
         self.device = torch.device(device)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.ws[:16].zero_()
@@ -99,6 +100,15 @@ class MoELayer:
         capi.moe_route(self.shape, self.weights.gate_w, x, bias, self.ids, self.gates,
                        self.counts, self.ws, stream)
         return self.ids, self.gates, self.counts
+
+    def balance_stats(self, seq_len: int, alpha: float, stream=None):
+        """f, P [S, N] and loss [S] of the last route/forward's routing."""
+        n_seq = -(-self.T // seq_len)
+        f = torch.empty((n_seq, self.N), dtype=torch.float32, device=self.device)
+        p = torch.empty_like(f)
+        loss = torch.empty((n_seq,), dtype=torch.float32, device=self.device)
+        capi.moe_balance_stats(self.shape, seq_len, alpha, self.ws, self.ids, f, p, loss, stream)
+        return f, p, loss
 
     def update_bias(self, bias: torch.Tensor, gamma: float, stream=None) -> None:
         capi.moe_update_bias(bias, self.counts, self.N, self.T, self.K, gamma, stream)

@@ -61,6 +61,36 @@ def test_bad_shapes_rejected(capi, shape):
     assert rc == -1  # MOE_ERR_SHAPE
 
 
+@pytest.mark.parametrize("groups,top", [(3, 1), (8, 3), (64, 4), (4, 8), (8, 0), (32, 2)])
+def test_bad_group_shapes_rejected(capi, groups, top):
+    # node-limited routing needs N % G == 0, 1 <= M <= G <= 32, K % M == 0 and
+    # K / M <= N / G (here N = 64, K = 8; G = 32 leaves 2 experts per group
+    # for K / M = 4)
+    assert capi.moe_workspace_size(capi.shape_of(64, 256, 64, 8, 128, groups, top)) == 0
+
+
+@pytest.mark.parametrize("groups,top", [(0, 0), (8, 4), (8, 8), (1, 1), (32, 8), (4, 1)])
+def test_group_shapes_accepted(capi, groups, top):
+    assert capi.moe_workspace_size(capi.shape_of(64, 256, 64, 8, 128, groups, top)) > 0
+
+
+def test_balance_stats_rejects_bad_arguments(capi):
+    import torch
+    sh = capi.shape_of(64, 256, 64, 8, 128)
+    need = capi.moe_workspace_size(sh)
+    buf = torch.empty(need + 256, dtype=torch.uint8)
+    ws = ctypes.c_void_p((buf.data_ptr() + 255) // 256 * 256)   # host memory: never touched
+    ids = torch.zeros((64, 8), dtype=torch.int32)
+    f = torch.empty((1, 64))
+    loss = torch.empty((1,))
+    lib = capi.LIB
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    # MOE_ERR_SHAPE = -1, MOE_ERR_NULL = -2, MOE_ERR_WORKSPACE = -6
+    assert lib.moe_balance_stats(sh, 0, 1e-4, ws, need, p(ids), p(f), p(f), p(loss), None) == -1
+    assert lib.moe_balance_stats(sh, 64, 1e-4, None, need, p(ids), p(f), p(f), p(loss), None) == -2
+    assert lib.moe_balance_stats(sh, 64, 1e-4, ws, 16, p(ids), p(f), p(f), p(loss), None) == -6
+
+
 def test_null_and_alignment_rejected(capi):
     sh = capi.shape_of(64, 256, 16, 4, 128)
     w = capi.moe_weights(16, 16, 16, 16, 16)
