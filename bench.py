@@ -48,6 +48,11 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-fp8-peak", action="store_true")
+    p.add_argument("--groups", type=int, default=0,
+                   help="node-limited routing: G expert groups (0: top-K over all N)")
+    p.add_argument("--topk-groups", type=int, default=0, help="node-limited routing: M groups")
+    p.add_argument("--seq-len", type=int, default=0,
+                   help="sequence length for the balance statistics (0: the whole batch)")
     return p.parse_args()
 
 
@@ -197,7 +202,8 @@ def measure_fp8_peak(torch, device):
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_sample_step(w, x, gate_w, bias, ew, step: int, groups: int = 2, shared_rows: int = 64):
+def oracle_sample_step(w, x, gate_w, bias, ew, step: int, groups: int = 2, shared_rows: int = 64,
+                       node_limit: tuple = (0, 0)):
     """One bounded sample of the layer on the CPU oracle; returns the time
     scaled to the whole layer (all T tokens, all N + 1 expert groups)."""
     from oracle import moe_oracle as O
@@ -205,7 +211,10 @@ def oracle_sample_step(w, x, gate_w, bias, ew, step: int, groups: int = 2, share
     xq, xs = O.quantize_1x128(x)
     t_quant = time.perf_counter() - t0
     t0 = time.perf_counter()
-    ids, gates, _, _ = O.route(x, gate_w, bias, w.K)
+    if node_limit[0] > 1 and node_limit[1] < node_limit[0]:
+        ids, gates, *_ = O.route_grouped(x, gate_w, bias, w.K, node_limit[0], node_limit[1])
+    else:
+        ids, gates, _, _ = O.route(x, gate_w, bias, w.K)
     O.permutation(ids, w.N)
     t_route = time.perf_counter() - t0
     y_routed = np.zeros((w.T, w.K, w.H))
@@ -253,8 +262,10 @@ def run_reference(args, w, rank):
     from mixture_experts_layer_40_b200 import inputs as I
     x, gate_w, bias, ew = oracle_setup(w, I.make_x(w))
     for s in range(args.warmup):
-        oracle_sample_step(w, x, gate_w, bias, ew, s)
-    times = [oracle_sample_step(w, x, gate_w, bias, ew, args.warmup + s) for s in range(args.steps)]
+        oracle_sample_step(w, x, gate_w, bias, ew, s, node_limit=(args.groups, args.topk_groups))
+    times = [oracle_sample_step(w, x, gate_w, bias, ew, args.warmup + s,
+                                node_limit=(args.groups, args.topk_groups))
+             for s in range(args.steps)]
     ms = 1e3 * float(np.mean(times))
     value = w.T / (ms * 1e-3)
     sample = (f"per step: the whole layer's routing, quantisation and combine on all {w.T} tokens, "
@@ -291,7 +302,8 @@ def run_ours(args, w, rank, world, local_rank):
     pool = I.make_weight_pool(w)   # same weights on every rank
     gate_w = I.make_gate_w(w)
     bias0 = I.make_bias(w)
-    layer = MoELayer(w.T, w.H, w.N, w.K, w.I, device_weights(w, pool, gate_w, dev), dev)
+    layer = MoELayer(w.T, w.H, w.N, w.K, w.I, device_weights(w, pool, gate_w, dev), dev,
+                     groups=args.groups, topk_groups=args.topk_groups)
     del pool
     x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     x = x_host.to(dev)
@@ -374,8 +386,18 @@ def run_ours(args, w, rank, world, local_rank):
         y_host.copy_(y, non_blocking=True)
     e_end.record(stream)
     barrier()
+    # ------------------------------------------------ balance statistics (not part of the step)
+    seq_len = args.seq_len or w.T
+    bal_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    layer.balance_stats(seq_len, 1e-4)
+    bal_ev[0].record(stream)
+    for _ in range(20):
+        layer.balance_stats(seq_len, 1e-4)
+    bal_ev[1].record(stream)
+    barrier()
     clk = clocks.stop() if clocks else None
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
+    bal_ms = bal_ev[0].elapsed_time(bal_ev[1]) / 20
 
     if rank != 0:
         return
@@ -402,6 +424,9 @@ def run_ours(args, w, rank, world, local_rank):
         "config": {"workload": f"{w.name}: T={w.T} per GPU, H={w.H}, N={w.N} routed top-{w.K} "
                                f"+ 1 shared, I={w.I}, SwiGLU, FP8 E4M3 1x128/128x128",
                    "tokens_per_gpu": w.T, "parallelism": f"dp{world} (weak: own batch per GPU)",
+                   "routing": (f"node-limited: {args.topk_groups} of {args.groups} expert groups"
+                               if args.groups > 1 and args.topk_groups < args.groups
+                               else f"top-{w.K} of all {w.N}"),
                    "l2": f"no flush: each step streams {weight_gb:.2f} GB of expert weights, "
                          f"{weight_gb * 1e3 / 126:.0f}x the 126 MB L2"},
         "gemm": {"tflops": gemm_tflops, "fp8_spec_tflops": FP8_SPEC_TFLOPS,
@@ -418,10 +443,13 @@ def run_ours(args, w, rank, world, local_rank):
         "e2e": {"value": w.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2},
         "clocks": clk,
+        "balance_stats": {"ms": bal_ms, "seq_len": seq_len,
+                          "note": "moe_balance_stats after the step, not part of it"},
     }
     if world == 1 and not args.no_cpu_baseline:
         x32, gw, b0, ew = oracle_setup(w, x_bits)
-        t = [oracle_sample_step(w, x32, gw, b0, ew, s) for s in range(2)]
+        t = [oracle_sample_step(w, x32, gw, b0, ew, s, node_limit=(args.groups, args.topk_groups))
+             for s in range(2)]
         v = w.T / float(np.mean(t))
         line["cpu_baseline"] = {
             "value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",

@@ -1,0 +1,63 @@
+"""Host-side checks of bench.py (no GPU): the reference arm's JSON line on the
+tiny workload, the algorithmic byte counts the roofline divides by, and the
+rule that a recorded DRAM capture is reported only for the GEMM sources it
+measured."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+import bench
+from mixture_experts_layer_40_b200 import inputs as I
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(*extra):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "1", "--warmup", "3", *extra],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    return json.loads(out.stdout.strip().splitlines()[-1])
+
+
+def test_reference_arm_line():
+    d = _run()
+    for key in ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"]:
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_node_limited():
+    d = _run("--groups", "4", "--topk-groups", "2")
+    assert d["value"] > 0
+
+
+def test_algorithmic_bytes_by_hand():
+    w = I.WORKLOADS["v3_prefill"]
+    work = bench.algorithmic_work(w, np.ones(256))
+    # up: 257 experts x (2 I H codes + 2 (I/128)(H/128) fp32 scales), plus
+    # 36864 rows x (H codes + H/128 scales) in and x (I codes + I/128 scales) out
+    up = 257 * (2 * 2048 * 7168 + 2 * 16 * 56 * 4) + 36864 * (7168 + 56 * 4) + 36864 * (2048 + 16 * 4)
+    assert work["expert_up"]["bytes"] == up
+    assert work["expert_up"]["flops"] == 2.0 * 36864 * 7168 * 4096
+    # down: weights, h rows in, bf16 rows out (2 bytes x H)
+    down = 257 * (7168 * 2048 + 56 * 16 * 4) + 36864 * (2048 + 16 * 4) + 36864 * 7168 * 2
+    assert work["expert_down"]["bytes"] == down
+
+
+def test_recorded_traffic_follows_the_sources(tmp_path, monkeypatch):
+    fp = bench.gemm_fingerprint()
+    assert len(fp) == 16
+    note = tmp_path / "t.md"
+    note.write_text(f"traffic expert_up bytes=123 workload=v3_prefill fingerprint={fp}\n"
+                    f"traffic expert_down bytes=456 workload=v3_prefill fingerprint=0000000000000000\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(note))
+    assert bench.recorded_traffic("expert_up", "v3_prefill") == 123
+    assert bench.recorded_traffic("expert_up", "decode") is None
+    assert bench.recorded_traffic("expert_down", "v3_prefill") is None   # stale capture
