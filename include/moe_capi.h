@@ -123,6 +123,8 @@ typedef struct {
   size_t h_s;           /* float [rows_total, I/128] */
   size_t y_rows;        /* float [rows_total, H]: expert outputs before the combine */
   size_t gate_split;    /* bf16 [3, N, H]: the fp32 centroids as three bf16 terms */
+  size_t bal_scratch;   /* moe_balance_stats scratch: float [T] token sums, then
+                           float and int32 [T + ceil(T/128), N] chunk partials */
   size_t total;         /* workspace bytes required */
 } moe_ws_layout;
 
@@ -205,14 +207,14 @@ int moe_route_noalloc(moe_shape sh, const float* gate_w, const void* x, const fl
  *   P[s, i] = (1 / T_s) * sum_{t in s} s_ti / sum_j s_tj   (all N affinities)
  *   loss[s] = alpha * sum_i f[s, i] * P[s, i]
  * with s_ti the router's sigmoid affinities (recomputed from the logits the
- * router left in ws). Sums run in a fixed order: results are reproducible.
+ * router left in ws; the call writes only the bal_scratch region of ws). Sums
+ * run in a fixed order: results are reproducible.
  *   topk_ids: int32 [T, K] of that call; f, P: float [S, N]; loss: float [S]
  * Errors: MOE_ERR_SHAPE for a bad shape or seq_len < 1; MOE_ERR_NULL;
  * MOE_ERR_WORKSPACE if ws_bytes < moe_workspace_size(sh).
  */
-int moe_balance_stats(moe_shape sh, int32_t seq_len, float alpha, const void* ws,
-                      size_t ws_bytes, const int32_t* topk_ids, float* f, float* P, float* loss,
-                      void* stream);
+int moe_balance_stats(moe_shape sh, int32_t seq_len, float alpha, void* ws, size_t ws_bytes,
+                      const int32_t* topk_ids, float* f, float* P, float* loss, void* stream);
 
 /*
  * The whole layer forward: quantise x (1x128), route, permute token rows by

@@ -41,7 +41,7 @@ class moe_weights(ctypes.Structure):
 
 _LAYOUT_FIELDS = ["status", "counts", "offsets", "group_rows", "row_start", "row_token",
                   "token_row", "topk_ids", "topk_gates", "logits", "a_q", "a_s", "h_q", "h_s",
-                  "y_rows", "gate_split", "total"]
+                  "y_rows", "gate_split", "bal_scratch", "total"]
 
 
 class moe_ws_layout(ctypes.Structure):

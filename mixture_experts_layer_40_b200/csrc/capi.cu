@@ -70,6 +70,7 @@ void layout_of(const moe_shape& s, moe_ws_layout* L) {
   L->h_s = take((size_t)L->rows_total * (I / kTile) * 4);
   L->y_rows = take((size_t)L->rows_total * H * 4);
   L->gate_split = take(router_split_bytes((int)N, (int)H));
+  L->bal_scratch = take(balance_scratch_bytes(T, N));
   L->total = off;
 }
 
@@ -202,18 +203,17 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
   return cuda_status(e);
 }
 
-int moe_balance_stats(moe_shape sh, int32_t seq_len, float alpha, const void* ws,
-                      size_t ws_bytes, const int32_t* topk_ids, float* f, float* P, float* loss,
-                      void* stream) {
+int moe_balance_stats(moe_shape sh, int32_t seq_len, float alpha, void* ws, size_t ws_bytes,
+                      const int32_t* topk_ids, float* f, float* P, float* loss, void* stream) {
   if (!shape_ok(sh) || seq_len < 1) return MOE_ERR_SHAPE;
   if (!ws || !topk_ids || !f || !P || !loss) return MOE_ERR_NULL;
   if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
   moe_ws_layout L;
   layout_of(sh, &L);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  return cuda_status(launch_balance_stats(at<float>(const_cast<void*>(ws), L.logits), topk_ids,
-                                          sh.T, sh.N, sh.K, seq_len, alpha, f, P, loss,
-                                          static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_balance_stats(at<float>(ws, L.logits), topk_ids, sh.T, sh.N, sh.K,
+                                          seq_len, alpha, at<uint8_t>(ws, L.bal_scratch), f, P,
+                                          loss, static_cast<cudaStream_t>(stream)));
 }
 
 static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const float* bias,

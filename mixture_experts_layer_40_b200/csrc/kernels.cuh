@@ -52,11 +52,12 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
                              int32_t* ids, float* gates, int32_t* counts, uint32_t* status,
                              cudaStream_t stream, int sm_count);
 
-// Sequence-wise balance statistics from the router's logits and top-K ids:
-// one CTA per sequence of seq_len tokens; f, P [S, N], loss [S].
+// Sequence-wise balance statistics from the router's logits and top-K ids
+// (f, P [S, N], loss [S]); scratch of balance_scratch_bytes(T, N) bytes.
+size_t balance_scratch_bytes(int64_t T, int64_t N);
 cudaError_t launch_balance_stats(const float* logits, const int32_t* ids, int T, int N, int K,
-                                 int seq_len, float alpha, float* f, float* P, float* loss,
-                                 cudaStream_t stream);
+                                 int seq_len, float alpha, uint8_t* scratch, float* f, float* P,
+                                 float* loss, cudaStream_t stream);
 
 // Permutation: scan of counts into group tables, stable scatter, row gather.
 cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K, int H,

@@ -208,96 +208,123 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
   }
 }
 
-// Sequence-wise balance statistics, one CTA of 16 warps per sequence. Warp w
-// takes the sequence's tokens w, w + 16, ...; for each, the lanes recompute
-// the affinities exactly as topk_kernel does, reduce their sum with a fixed
-// butterfly and add s_ti / sum_j s_tj into per-lane partials. The warps'
-// partials are then added in warp order, and the counts come from integer
-// atomics: every result is independent of scheduling.
-constexpr int kBalWarps = 16;
-__global__ void __launch_bounds__(kBalWarps * 32) balance_stats_kernel(const float* __restrict__ z,
-                                                             const int32_t* __restrict__ ids,
-                                                             int T, int N, int K, int seq_len,
-                                                             float alpha, float* __restrict__ f,
-                                                             float* __restrict__ P,
-                                                             float* __restrict__ loss) {
-  __shared__ int cnt[1024];
-  __shared__ float red[kBalWarps][33];
-  __shared__ float fp_part[32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int q = blockIdx.x;
-  const int lo = q * seq_len;
-  const int hi = min(T, lo + seq_len);
-  const int t_seq = hi - lo;
+// Sequence-wise balance statistics in three passes, every sum in a fixed
+// order so the results do not depend on scheduling:
+//   1. one warp per token: D_t = sum_j s_tj over all N affinities, recomputed
+//      from the logits exactly as topk_kernel computes them;
+//   2. one CTA per chunk of <= kBalChunk tokens of one sequence, one thread
+//      per expert: the chunk's sum of s_ti / D_t (token order) and its
+//      selection counts (integer atomics);
+//   3. one CTA per sequence: chunk partials added in chunk order, then f, P
+//      and alpha * sum_i f_i P_i (expert order).
+constexpr int kBalChunk = 128;
+
+MOE_DEV float affinity(float z) { return 1.0f / (1.0f + expf(-z)); }
+
+__global__ void __launch_bounds__(256) token_sum_kernel(const float* __restrict__ z, int T, int N,
+                                                        float* __restrict__ denom) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
   const int per_lane = (N + 31) >> 5;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+    float part = 0.0f;
+    for (int j = 0; j < per_lane; ++j) {
+      const int e = lane + 32 * j;
+      if (e < N) part += affinity(z[(int64_t)t * N + e]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) denom[t] = part;
+  }
+}
+
+__global__ void __launch_bounds__(1024) chunk_partial_kernel(
+    const float* __restrict__ z, const int32_t* __restrict__ ids, const float* __restrict__ denom,
+    int T, int N, int K, int seq_len, int chunks_per_seq, float* __restrict__ part_p,
+    int32_t* __restrict__ part_c) {
+  __shared__ int cnt[1024];
+  const int seq = blockIdx.x / chunks_per_seq, chunk = blockIdx.x % chunks_per_seq;
+  const int seq_end = min(T, (seq + 1) * seq_len);
+  const int lo = seq * seq_len + chunk * kBalChunk;
+  const int hi = min(seq_end, lo + kBalChunk);
   for (int i = threadIdx.x; i < N; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   for (int i = lo * K + threadIdx.x; i < hi * K; i += blockDim.x) {
     const int e = ids[i];
     if (e >= 0 && e < N) atomicAdd(&cnt[e], 1);
   }
-  float acc[kMaxPerLane];
-#pragma unroll
-  for (int j = 0; j < kMaxPerLane; ++j) acc[j] = 0.0f;
-  for (int t = lo + warp; t < hi; t += kBalWarps) {
-    float sv[kMaxPerLane];
-    float part = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kMaxPerLane; ++j) {
-      const int e = lane + 32 * j;
-      sv[j] = 0.0f;
-      if (j < per_lane && e < N) {
-        sv[j] = 1.0f / (1.0f + expf(-z[(int64_t)t * N + e]));
-        part += sv[j];
-      }
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    float acc = 0.0f;
+    for (int t = lo; t < hi; ++t) acc += affinity(z[(int64_t)t * N + e]) / denom[t];
+    part_p[(int64_t)blockIdx.x * N + e] = acc;
+    part_c[(int64_t)blockIdx.x * N + e] = cnt[e];
+  }
+}
+
+__global__ void __launch_bounds__(1024) seq_reduce_kernel(const float* __restrict__ part_p,
+                                                          const int32_t* __restrict__ part_c,
+                                                          int T, int N, int K, int seq_len,
+                                                          int chunks_per_seq, float alpha,
+                                                          float* __restrict__ f,
+                                                          float* __restrict__ P,
+                                                          float* __restrict__ loss) {
+  __shared__ float fp[1024];
+  const int q = blockIdx.x;
+  const int t_seq = min(T, (q + 1) * seq_len) - q * seq_len;
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    float ps = 0.0f;
+    int c = 0;
+    for (int k = 0; k < chunks_per_seq; ++k) {
+      const int64_t at = ((int64_t)q * chunks_per_seq + k) * N + e;
+      ps += part_p[at];
+      c += part_c[at];
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-#pragma unroll
-    for (int j = 0; j < kMaxPerLane; ++j)
-      if (j < per_lane) acc[j] += sv[j] / part;
+    const float pi = ps / (float)t_seq;
+    const float fi = (float)N * (float)c / ((float)K * (float)t_seq);
+    P[(int64_t)q * N + e] = pi;
+    f[(int64_t)q * N + e] = fi;
+    fp[e] = fi * pi;
   }
   __syncthreads();
-  float fp_lane = 0.0f;  // lane's share of sum_i f_i P_i (warp 0)
-#pragma unroll
-  for (int j = 0; j < kMaxPerLane; ++j) {
-    if (j >= per_lane) break;  // CTA-uniform
-    red[warp][lane] = acc[j];
-    __syncthreads();
-    if (warp == 0) {
-      float sum = 0.0f;
-      for (int w = 0; w < kBalWarps; ++w) sum += red[w][lane];
-      const int e = lane + 32 * j;
-      if (e < N) {
-        const float pi = sum / (float)t_seq;
-        const float fi = (float)N * (float)cnt[e] / ((float)K * (float)t_seq);
-        P[(int64_t)q * N + e] = pi;
-        f[(int64_t)q * N + e] = fi;
-        fp_lane += fi * pi;
-      }
-    }
-    __syncthreads();
-  }
-  if (warp == 0) {
-    fp_part[lane] = fp_lane;
-    __syncwarp();
-    if (lane == 0) {
-      float sum = 0.0f;
-      for (int l = 0; l < 32; ++l) sum += fp_part[l];
-      loss[q] = alpha * sum;
-    }
+  if (threadIdx.x == 0) {
+    float sum = 0.0f;
+    for (int e = 0; e < N; ++e) sum += fp[e];
+    loss[q] = alpha * sum;
   }
 }
 
 }  // namespace
 
+size_t balance_scratch_bytes(int64_t T, int64_t N) {
+  const int64_t parts = T + (T + kBalChunk - 1) / kBalChunk;
+  return (size_t)((T * 4 + 255) / 256 * 256 + 2 * parts * N * 4);
+}
+
 cudaError_t launch_balance_stats(const float* logits, const int32_t* ids, int T, int N, int K,
-                                 int seq_len, float alpha, float* f, float* P, float* loss,
-                                 cudaStream_t stream) {
+                                 int seq_len, float alpha, uint8_t* scratch, float* f, float* P,
+                                 float* loss, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int n_seq = (T + seq_len - 1) / seq_len;
-  balance_stats_kernel<<<n_seq, kBalWarps * 32, 0, stream>>>(logits, ids, T, N, K, seq_len, alpha, f, P,
-                                                   loss);
+  const int per_seq = (std::min(seq_len, T) + kBalChunk - 1) / kBalChunk;
+  // n_seq * per_seq <= T + ceil(T / kBalChunk): the scratch bound
+  float* denom = reinterpret_cast<float*>(scratch);
+  const int64_t parts = (int64_t)n_seq * per_seq;
+  if (parts > (int64_t)T + (T + kBalChunk - 1) / kBalChunk) return cudaErrorInvalidValue;
+  float* part_p = reinterpret_cast<float*>(scratch + ((int64_t)T * 4 + 255) / 256 * 256);
+  int32_t* part_c = reinterpret_cast<int32_t*>(part_p + parts * N);
+  int blocks = (T + 7) / 8;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  token_sum_kernel<<<blocks, 256, 0, stream>>>(logits, T, N, denom);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int threads = std::min(1024, (N + 31) / 32 * 32);
+  chunk_partial_kernel<<<(unsigned)parts, threads, 0, stream>>>(logits, ids, denom, T, N, K,
+                                                                seq_len, per_seq, part_p, part_c);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  seq_reduce_kernel<<<n_seq, threads, 0, stream>>>(part_p, part_c, T, N, K, seq_len, per_seq,
+                                                   alpha, f, P, loss);
   return cudaGetLastError();
 }
 
