@@ -322,12 +322,12 @@ def run_ours(args, w, rank, world, local_rank):
     # combine, bias update
     launches_per_step = 11
 
-    def step(traced_events=None, x_in=x):
+    def step(traced_events=None, x_in=x, y_out=y):
         if traced_events is None:
-            capi.moe_forward(layer.shape, layer._cw, x_in, bias, y, layer.ids, layer.gates,
+            capi.moe_forward(layer.shape, layer._cw, x_in, bias, y_out, layer.ids, layer.gates,
                              layer.counts, layer.ws)
         else:
-            capi.moe_forward_traced(layer.shape, layer._cw, x_in, bias, y, traced_events,
+            capi.moe_forward_traced(layer.shape, layer._cw, x_in, bias, y_out, traced_events,
                                     layer.ids, layer.gates, layer.counts, layer.ws)
         if world > 1:
             dist.all_reduce(layer.counts)
@@ -372,18 +372,45 @@ def run_ours(args, w, rank, world, local_rank):
     counts = layer.counts.cpu().numpy()
 
     # ------------------------------------------------ end to end (host buffers)
-    for _ in range(2):
-        x.copy_(x_host, non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
+    # Every step copies its input from pinned host memory and its output back.
+    # The copies run on their own streams with two device buffers each way, so
+    # step i+1's upload and step i-1's download overlap step i's kernels; the
+    # layer's steps themselves stay in order on the compute stream (each
+    # step's routing uses the bias the previous step updated).
+    up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
+    xs = [x, torch.empty_like(x)]
+    ys = [y, torch.empty_like(y)]
+    y_hosts = [y_host, torch.empty_like(y_host).pin_memory()]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(i):
+        b = i % 2
+        up_s.wait_event(ev_done[b])          # step i-2 no longer reads xs[b]
+        with torch.cuda.stream(up_s):
+            xs[b].copy_(x_host, non_blocking=True)
+        ev_in[b].record(up_s)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])         # ys[b] of step i-2 is downloaded
+        step(x_in=xs[b], y_out=ys[b])
+        ev_done[b].record(stream)
+        down_s.wait_event(ev_done[b])
+        with torch.cuda.stream(down_s):
+            y_hosts[b].copy_(ys[b], non_blocking=True)
+        ev_out[b].record(down_s)
+
+    for i in range(2):
+        e2e_step(i)
     barrier()
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
-    for _ in range(args.steps):
-        x.copy_(x_host, non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
+    up_s.wait_event(e_start)
+    for i in range(args.steps):
+        e2e_step(i)
+    stream.wait_event(ev_out[0])
+    stream.wait_event(ev_out[1])
     e_end.record(stream)
     barrier()
     # ------------------------------------------------ balance statistics (not part of the step)
@@ -441,7 +468,9 @@ def run_ours(args, w, rank, world, local_rank):
                      "algorithmic_bytes": work[dom]["bytes"]},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": w.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2},
+                "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2,
+                "copies": "pinned host buffers; upload and download on side streams, "
+                          "double-buffered, overlapping the neighbouring steps' kernels"},
         "clocks": clk,
         "balance_stats": {"ms": bal_ms, "seq_len": seq_len,
                           "note": "moe_balance_stats after the step, not part of it"},
