@@ -84,7 +84,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA
 }  // namespace
 
 bool shape_ok(const moe_shape& s) {
-  return s.T >= 1 && s.H >= 256 && s.H % 256 == 0 && s.I >= 128 && s.I % 128 == 0 && s.N >= 16 &&
+  return s.T >= 0 && s.H >= 256 && s.H % 256 == 0 && s.I >= 128 && s.I % 128 == 0 && s.N >= 16 &&
          s.N <= 1024 && s.N % 16 == 0 && s.K >= 1 && s.K <= s.N && s.K <= 16 &&
          (int64_t)s.T * s.K < (1ll << 31) && (int64_t)s.T * s.N < (1ll << 31) &&
          (s.G == 0 || (s.G >= 1 && s.G <= 32 && s.N % s.G == 0 && s.M >= 1 && s.M <= s.G &&
@@ -187,6 +187,11 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
               int32_t* topk_ids, float* topk_gates, int32_t* counts, void* ws, size_t ws_bytes,
               void* stream) {
   if (!shape_ok(sh)) return MOE_ERR_SHAPE;
+  if (sh.T == 0) {  // an empty batch: only the counts are cleared
+    if (!counts) return MOE_ERR_NULL;
+    return cuda_status(
+        cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, static_cast<cudaStream_t>(stream)));
+  }
   if (!gate_w || !x || !bias || !topk_ids || !topk_gates || !counts || !ws) return MOE_ERR_NULL;
   if (!aligned(x, 16) || !aligned(gate_w, 16) || !aligned(ws, 256)) return MOE_ERR_ALIGN;
   moe_ws_layout L;
@@ -206,6 +211,7 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
 int moe_balance_stats(moe_shape sh, int32_t seq_len, float alpha, void* ws, size_t ws_bytes,
                       const int32_t* topk_ids, float* f, float* P, float* loss, void* stream) {
   if (!shape_ok(sh) || seq_len < 1) return MOE_ERR_SHAPE;
+  if (sh.T == 0) return MOE_OK;  // no sequences
   if (!ws || !topk_ids || !f || !P || !loss) return MOE_ERR_NULL;
   if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
   moe_ws_layout L;
@@ -220,6 +226,22 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
                         void* y, int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
                         void* ws, size_t ws_bytes, void* stream, void* const* events) {
   if (!shape_ok(sh)) return MOE_ERR_SHAPE;
+  if (sh.T == 0) {
+    // an empty batch: nothing to compute; the status word and the counts
+    // (for moe_update_bias, which then leaves the bias unchanged) are cleared
+    if (!ws) return MOE_ERR_NULL;
+    if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
+    moe_ws_layout L;
+    layout_of(sh, &L);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, L.status), 0, 4, s);
+    int32_t* counts = counts_opt ? counts_opt : at<int32_t>(ws, L.counts);
+    if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
+    for (int i = 0; events != nullptr && i < MOE_TRACE_EVENTS && e == cudaSuccess; ++i)
+      e = cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+    return cuda_status(e);
+  }
   if (!w || !x || !bias || !y || !ws) return MOE_ERR_NULL;
   if (!w->gate_w || !w->w13 || !w->s13 || !w->w2 || !w->s2) return MOE_ERR_NULL;
   if (!aligned(x, 16) || !aligned(y, 16) || !aligned(w->gate_w, 16) || !aligned(w->w13, 16) ||

@@ -60,6 +60,13 @@ extern "C" int moe_route_noalloc(moe_shape sh, const float* gate_w, const void* 
   using namespace moe;
   if (!shape_ok(sh)) return MOE_ERR_SHAPE;
   if ((int64_t)sh.T * sh.N > (int64_t)MOE_ROUTE_NOALLOC_MAX_LOGITS) return MOE_ERR_WORKSPACE;
+  if (sh.T == 0) {  // an empty batch: only the counts are cleared
+    if (!counts) return MOE_ERR_NULL;
+    return cudaMemsetAsync(counts, 0, (size_t)sh.N * sizeof(int32_t),
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+  }
   if (!gate_w || !x || !bias || !topk_ids || !topk_gates || !counts) return MOE_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(x) % 16) != 0 || (reinterpret_cast<uintptr_t>(gate_w) % 16) != 0)
     return MOE_ERR_ALIGN;

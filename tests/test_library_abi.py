@@ -50,7 +50,7 @@ def test_workspace_layout(capi):
     assert L.y_rows + L.rows_total * 7168 * 2 <= L.total
 
 
-@pytest.mark.parametrize("shape", [(0, 256, 16, 4, 128), (64, 200, 16, 4, 128), (64, 256, 16, 4, 100),
+@pytest.mark.parametrize("shape", [(-1, 256, 16, 4, 128), (64, 200, 16, 4, 128), (64, 256, 16, 4, 100),
                                    (64, 256, 15, 4, 128), (64, 256, 16, 17, 128), (64, 256, 16, 0, 128),
                                    (64, 128, 16, 4, 128), (64, 256, 2048, 4, 128)])
 def test_bad_shapes_rejected(capi, shape):
@@ -89,6 +89,11 @@ def test_balance_stats_rejects_bad_arguments(capi):
     assert lib.moe_balance_stats(sh, 0, 1e-4, ws, need, p(ids), p(f), p(f), p(loss), None) == -1
     assert lib.moe_balance_stats(sh, 64, 1e-4, None, need, p(ids), p(f), p(f), p(loss), None) == -2
     assert lib.moe_balance_stats(sh, 64, 1e-4, ws, 16, p(ids), p(f), p(f), p(loss), None) == -6
+
+
+def test_empty_batch_shape_accepted(capi):
+    # T = 0 is an empty batch (no work; counts cleared), not a bad shape
+    assert capi.moe_workspace_size(capi.shape_of(0, 7168, 256, 8, 2048)) > 0
 
 
 def test_null_and_alignment_rejected(capi):
