@@ -137,9 +137,11 @@ def algorithmic_work(w, counts: np.ndarray):
     return {
         "expert_up": {"bytes": w13_bytes + a_bytes + h_bytes, "flops": 2.0 * rows * w.H * 2 * w.I},
         "expert_down": {"bytes": w2_bytes + h_bytes + y_bytes, "flops": 2.0 * rows * w.I * w.H},
-        "quantize": {"bytes": w.T * w.H * 3 + w.T * hb * 4, "flops": 0.0},
+        # x read once, codes + scales written to the shared row and K routed rows
+        "quantize": {"bytes": w.T * w.H * 2 + (w.K + 1) * w.T * (w.H + hb * 4), "flops": 0.0},
         "combine": {"bytes": (w.T * w.K + w.T) * w.H * 2 + w.T * w.H * 2, "flops": 0.0},
-        "permute": {"bytes": 2 * w.T * w.K * (w.H + hb * 4), "flops": 0.0},
+        # ids read, row_token and token_row written
+        "permute": {"bytes": 3 * w.T * w.K * 4, "flops": 0.0},
         "route": {"bytes": w.T * w.H * 2 + w.N * w.H * 4, "flops": 2.0 * w.T * w.N * w.H},
     }
 
@@ -318,9 +320,9 @@ def run_ours(args, w, rank, world, local_rank):
     for evs in events:
         for ev in evs:
             ev.record(stream)
-    # quantise, split gate, logits, top-K, scan, scatter, gather, up, down,
+    # split gate, logits, top-K, scan, scatter, quantise-and-scatter, up, down,
     # combine, bias update
-    launches_per_step = 11
+    launches_per_step = 10
 
     def step(traced_events=None, x_in=x, y_out=y):
         if traced_events is None:

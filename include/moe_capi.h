@@ -238,8 +238,9 @@ int moe_forward(moe_shape sh, const moe_weights* w, const void* x, const float* 
 /*
  * moe_forward with stage timing: identical work and results, and in addition
  * records events[i] on `stream` before stage i and events[6] after the last:
- *   0 quantise x, 1 route, 2 permute (scan, scatter, gather),
- *   3 up/gate GEMM + SwiGLU + re-quantisation, 4 down GEMM, 5 combine.
+ *   0 route, 1 permute (scan, scatter), 2 quantise x into the token's
+ *   shared-expert and routed GEMM rows, 3 up/gate GEMM + SwiGLU +
+ *   re-quantisation, 4 down GEMM, 5 combine.
  * events: MOE_TRACE_EVENTS cudaEvent_t handles created by the caller
  * (n_events >= MOE_TRACE_EVENTS, none NULL, else MOE_ERR_NULL).
  */

@@ -188,7 +188,7 @@ def moe_forward(sh: moe_shape, w: moe_weights, x, bias, y, topk_ids=None, topk_g
 
 
 TRACE_EVENTS = 7
-TRACE_STAGES = ["quantize", "route", "permute", "expert_up", "expert_down", "combine"]
+TRACE_STAGES = ["route", "permute", "quantize", "expert_up", "expert_down", "combine"]
 
 
 def moe_forward_traced(sh: moe_shape, w: moe_weights, x, bias, y, events, topk_ids=None,

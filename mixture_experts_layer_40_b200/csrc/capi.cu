@@ -258,7 +258,6 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   int32_t* counts = counts_opt ? counts_opt : at<int32_t>(ws, L.counts);
   uint8_t* a_q = at<uint8_t>(ws, L.a_q);
   float* a_s = at<float>(ws, L.a_s);
-  const int64_t H = sh.H, I = sh.I;
 
   // optional stage events: recorded before each of the 6 stages and at the end
   auto mark = [&](int i, cudaError_t e) {
@@ -269,23 +268,23 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   cudaError_t e = mark(0, cudaSuccess);
   if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
-  // a1: x -> 1x128 codes and scales, written into the shared-expert GEMM rows
-  if (e == cudaSuccess)
-    e = launch_quantize_1x128(x, sh.T, H, a_q + L.routed_cap * H, a_s + L.routed_cap * (H / kTile),
-                              s, sms);
-  e = mark(1, e);
-  // a2-a5: gate logits, sigmoid, biased top-K, gates, counts
+  // a2-a5: gate logits, sigmoid, biased top-K, gates, counts (from bf16 x)
   if (e == cudaSuccess)
     e = launch_router_tc(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                          at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
                          counts, status, s, sms);
-  e = mark(2, e);
-  // a6-a7: offsets, stable expert-major scatter, gather of the quantised rows
+  e = mark(1, e);
+  // a6-a7: offsets, stable expert-major scatter of the (token, slot) pairs
   if (e == cudaSuccess)
-    e = launch_permute(ids, counts, sh.T, sh.N, sh.K, sh.H, L.routed_cap,
-                       at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.group_rows),
-                       at<int32_t>(ws, L.row_start), at<int32_t>(ws, L.row_token),
-                       at<int32_t>(ws, L.token_row), a_q, a_s, status, s, sms);
+    e = launch_permute(ids, counts, sh.T, sh.N, sh.K, L.routed_cap, at<int32_t>(ws, L.offsets),
+                       at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
+                       at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.token_row), status, s);
+  e = mark(2, e);
+  // a1 (+ a7's row copies): x -> 1x128 codes and scales, written to the
+  // token's shared-expert row and its K routed rows
+  if (e == cudaSuccess)
+    e = launch_quantize_scatter(x, sh.T, sh.H, sh.K, at<int32_t>(ws, L.token_row), L.routed_cap,
+                                a_q, a_s, status, s, sms);
   GroupedGemm gg{sh.H, sh.I, sh.N + 1, at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
                  L.rows_total, status};
   e = mark(3, e);
@@ -305,7 +304,6 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
                        sh.T, sh.H, sh.K, L.routed_cap, L.rows_total,
                        static_cast<__nv_bfloat16*>(y), status, s);
   e = mark(6, e);
-  (void)I;
   return cuda_status(e);
 }
 

@@ -59,12 +59,17 @@ cudaError_t launch_balance_stats(const float* logits, const int32_t* ids, int T,
                                  int seq_len, float alpha, uint8_t* scratch, float* f, float* P,
                                  float* loss, cudaStream_t stream);
 
-// Permutation: scan of counts into group tables, stable scatter, row gather.
-cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K, int H,
+// Permutation: scan of counts into group tables, stable scatter of the
+// (token, slot) pairs into expert-major GEMM rows.
+cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K,
                            int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
                            int32_t* row_start, int32_t* row_token, int32_t* token_row,
-                           uint8_t* a_q, float* a_s, uint32_t* status, cudaStream_t stream,
-                           int sm_count);
+                           uint32_t* status, cudaStream_t stream);
+// 1x128 quantisation of x written to each token's shared-expert row
+// (routed_cap + t) and to its K routed rows token_row[t, k].
+cudaError_t launch_quantize_scatter(const void* x, int T, int H, int K, const int32_t* token_row,
+                                    int64_t routed_cap, uint8_t* a_q, float* a_s,
+                                    uint32_t* status, cudaStream_t stream, int sm_count);
 
 cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const float* a_s,
                              const uint8_t* w13, const float* s13, uint8_t* h_q, float* h_s,

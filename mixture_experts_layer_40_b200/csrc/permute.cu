@@ -4,9 +4,9 @@
 // order is unique and the scatter needs no atomics on output positions.
 //   scan    : counts -> offsets, GEMM group rows and 128-aligned row starts
 //   scatter : one CTA per expert compacts the tokens that chose it, in token
-//             order, with a block-wide prefix sum over ballots
-//   gather  : copies the quantised input row (codes + scales) of each routed
-//             GEMM row from the shared-expert rows, where the quantiser put it
+//             order, with a block-wide prefix sum over ballots, and records
+//             each (token, slot)'s GEMM row; the activation quantiser then
+//             writes every token's codes straight into its rows
 #include "kernels.cuh"
 
 namespace moe {
@@ -136,41 +136,12 @@ __global__ void __launch_bounds__(1024) scatter_kernel(const int32_t* __restrict
   if (threadIdx.x == 0 && running != count) flag_status(status, kStatusBounds);
 }
 
-// One warp per routed GEMM row: copies H code bytes and H/128 scales of the
-// token's quantised input (stored in the shared-expert rows) into the row.
-__global__ void __launch_bounds__(256) gather_kernel(const int32_t* __restrict__ row_token,
-                                                     int64_t routed_cap, int T, int H,
-                                                     uint8_t* __restrict__ a_q,
-                                                     float* __restrict__ a_s,
-                                                     uint32_t* __restrict__ status) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  const int vec = H / 16;
-  const int nsc = H / kTile;
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < routed_cap;
-       r += warps) {
-    const int t = __ldg(row_token + r);
-    if (t < 0) continue;
-    if (t >= T) {
-      if (lane == 0) flag_status(status, kStatusBounds);
-      continue;
-    }
-    const uint4* src = reinterpret_cast<const uint4*>(a_q + (routed_cap + t) * (int64_t)H);
-    uint4* dst = reinterpret_cast<uint4*>(a_q + r * (int64_t)H);
-    for (int i = lane; i < vec; i += 32) dst[i] = __ldg(src + i);
-    const float* ss = a_s + (routed_cap + t) * (int64_t)nsc;
-    float* ds = a_s + r * (int64_t)nsc;
-    for (int i = lane; i < nsc; i += 32) ds[i] = __ldg(ss + i);
-  }
-}
-
 }  // namespace
 
-cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K, int H,
+cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K,
                            int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
                            int32_t* row_start, int32_t* row_token, int32_t* token_row,
-                           uint8_t* a_q, float* a_s, uint32_t* status, cudaStream_t stream,
-                           int sm_count) {
+                           uint32_t* status, cudaStream_t stream) {
   scan_kernel<<<1, 1024, 0, stream>>>(counts, N, T, K, routed_cap, offsets, group_rows, row_start,
                                       status);
   cudaError_t e = cudaGetLastError();
@@ -179,11 +150,6 @@ cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int
   if (e != cudaSuccess) return e;
   scatter_kernel<<<N, 1024, 0, stream>>>(ids, T, K, group_rows, row_start, routed_cap, row_token,
                                          token_row, status);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  int64_t blocks = (routed_cap + 7) / 8;
-  if (blocks > (int64_t)sm_count * 8) blocks = (int64_t)sm_count * 8;
-  gather_kernel<<<(unsigned)blocks, 256, 0, stream>>>(row_token, routed_cap, T, H, a_q, a_s, status);
   return cudaGetLastError();
 }
 

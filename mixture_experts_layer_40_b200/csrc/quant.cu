@@ -74,6 +74,68 @@ __global__ void __launch_bounds__(256) quantize_128x128_kernel(const float4* __r
   if (threadIdx.x == 0) scales[rb * col_blocks + cb] = s;
 }
 
+// The layer's activation quantiser, fused with the permutation: the codes and
+// the scale of each 1x128 tile of token t go to the shared expert's GEMM row
+// routed_cap + t and to the token's K routed GEMM rows token_row[t, k], so x
+// is read once and no second pass copies rows. Same tiling as above; lane k
+// of a tile's 16 threads fetches the k-th destination row.
+__global__ void __launch_bounds__(256) quantize_scatter_kernel(
+    const uint4* __restrict__ x, int T, int H, int K, const int32_t* __restrict__ token_row,
+    int64_t routed_cap, uint8_t* __restrict__ a_q, float* __restrict__ a_s,
+    uint32_t* __restrict__ status) {
+  const int sub = threadIdx.x & 15;
+  const int tiles_per_row = H / kTile;
+  const int64_t n_tiles = (int64_t)T * tiles_per_row;
+  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_tiles; base += (int64_t)gridDim.x * 16) {
+    const int64_t tile = base + (threadIdx.x >> 4);
+    const bool live = tile < n_tiles;
+    const int64_t t = live ? tile / tiles_per_row : 0;
+    const int c = live ? (int)(tile - t * tiles_per_row) : 0;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (live) v = __ldcs(x + tile * 16 + sub);
+    int my_row = -1;
+    if (live && sub < K) my_row = __ldg(token_row + t * K + sub);
+    float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                  bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = tile_scale(amax);
+    uint2 out;
+    out.x = e4m3x4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
+    out.y = e4m3x4(__fmul_rn(f[4], s), __fmul_rn(f[5], s), __fmul_rn(f[6], s), __fmul_rn(f[7], s));
+    for (int k = -1; k < K; ++k) {
+      int64_t r = routed_cap + t;
+      if (k >= 0) {
+        r = __shfl_sync(0xffffffffu, my_row, k, 16);
+        if (live && (r < 0 || r >= routed_cap)) {
+          if (sub == 0) flag_status(status, kStatusBounds);
+          continue;
+        }
+      }
+      if (live) {
+        reinterpret_cast<uint2*>(a_q + r * H + (int64_t)c * kTile)[sub] = out;
+        if (sub == 0) a_s[r * tiles_per_row + c] = s;
+      }
+    }
+  }
+}
+
+cudaError_t launch_quantize_scatter(const void* x, int T, int H, int K, const int32_t* token_row,
+                                    int64_t routed_cap, uint8_t* a_q, float* a_s,
+                                    uint32_t* status, cudaStream_t stream, int sm_count) {
+  const int64_t n_tiles = (int64_t)T * (H / kTile);
+  if (n_tiles == 0) return cudaSuccess;
+  int64_t blocks = (n_tiles + 15) / 16;
+  const int64_t cap = (int64_t)sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  quantize_scatter_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(x), T, H, K, token_row, routed_cap, a_q, a_s, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q,
                                   float* scales, cudaStream_t stream, int sm_count) {
   const int64_t n_tiles = rows * (cols / kTile);
