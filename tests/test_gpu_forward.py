@@ -67,7 +67,7 @@ def check_intermediates(w, case, layer, bias, sample_rows=None):
     assert np.array_equal(row_token, expect_rt)
     expect_tr = st[use_ids] + rank
     assert np.array_equal(token_row, expect_tr)
-    # routed GEMM rows hold the token's codes (gather)
+    # routed GEMM rows hold the token's codes
     some = np.nonzero(row_token >= 0)[0][:: max(1, (row_token >= 0).sum() // 64)]
     got = a_q[torch.from_numpy(some).cuda()].cpu().numpy()
     want = a_q[torch.from_numpy(L.routed_cap + row_token[some]).cuda()].cpu().numpy()
