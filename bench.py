@@ -258,6 +258,48 @@ def oracle_setup(w, x_bits):
     return I.bf16_bits_to_f32(x_bits), I.make_gate_w(w), I.make_bias(w), ew
 
 
+# ---------------------------------------------------------------- ranks
+
+def rank_batch(w, rank: int):
+    """Weak scaling: every rank routes its own batch of T tokens (its own
+    seed); the weights, centroids and starting bias are the same on all."""
+    return dataclasses.replace(w, seed=w.seed + rank)
+
+
+def batch_counts(counts, world: int):
+    """The bias controller balances the whole batch: per-expert counts are
+    summed over the ranks (one all-reduce of N int32) before the update,
+    which then uses T_total = world * T."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(counts)
+    return counts
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    """A multi-rank time is the slowest rank's."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_config(args, w, world: int) -> dict:
+    """The `config` object of both arms' lines."""
+    weight_gb = (w.N + 1) * 3 * w.H * w.I / 1e9
+    return {"workload": f"{w.name}: T={w.T} per GPU, H={w.H}, N={w.N} routed top-{w.K} "
+                        f"+ 1 shared, I={w.I}, SwiGLU, FP8 E4M3 1x128/128x128",
+            "tokens_per_gpu": w.T, "parallelism": f"dp{world} (weak: own batch per GPU)",
+            "routing": (f"node-limited: {args.topk_groups} of {args.groups} expert groups"
+                        if args.groups > 1 and args.topk_groups < args.groups
+                        else f"top-{w.K} of all {w.N}"),
+            "l2": f"no flush: each step streams {weight_gb:.2f} GB of expert weights, "
+                  f"{weight_gb * 1e3 / 126:.0f}x the 126 MB L2"}
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return
@@ -277,7 +319,7 @@ def run_reference(args, w, rank):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": f"{w.name}: T={w.T} H={w.H} N={w.N} K={w.K} I={w.I}"},
+            "config": run_config(args, w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -299,7 +341,7 @@ def run_ours(args, w, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wr = dataclasses.replace(w, seed=w.seed + rank)  # own batch per rank
+    wr = rank_batch(w, rank)
     x_bits = I.make_x(wr)
     pool = I.make_weight_pool(w)   # same weights on every rank
     gate_w = I.make_gate_w(w)
@@ -331,21 +373,13 @@ def run_ours(args, w, rank, world, local_rank):
         else:
             capi.moe_forward_traced(layer.shape, layer._cw, x_in, bias, y_out, traced_events,
                                     layer.ids, layer.gates, layer.counts, layer.ws)
-        if world > 1:
-            dist.all_reduce(layer.counts)
+        batch_counts(layer.counts, world)
         capi.moe_update_bias(bias, layer.counts, w.N, t_total, w.K, w.gamma)
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     for _ in range(args.warmup):
         step()
@@ -365,7 +399,7 @@ def run_ours(args, w, rank, world, local_rank):
         step(events[k])
     t_end.record(stream)
     barrier()
-    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     ms_step = ms_total / args.steps
     stage_ms = {name: float(np.mean([evs[i].elapsed_time(evs[i + 1]) for evs in events]))
                 for i, name in enumerate(capi.TRACE_STAGES)}
@@ -425,7 +459,7 @@ def run_ours(args, w, rank, world, local_rank):
     bal_ev[1].record(stream)
     barrier()
     clk = clocks.stop() if clocks else None
-    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev) / args.steps
     bal_ms = bal_ev[0].elapsed_time(bal_ev[1]) / 20
 
     if rank != 0:
@@ -438,7 +472,6 @@ def run_ours(args, w, rank, world, local_rank):
         except Exception:
             fp8_meas = None
     work = algorithmic_work(w, counts)
-    weight_gb = (int(np.count_nonzero(counts)) + 1) * 3 * w.H * w.I / 1e9
     dom = max(stage_ms, key=stage_ms.get)
     gemm_ms = stage_ms["expert_up"] + stage_ms["expert_down"]
     gemm_tflops = (work["expert_up"]["flops"] + work["expert_down"]["flops"]) / (gemm_ms * 1e-3) / 1e12
@@ -450,14 +483,7 @@ def run_ours(args, w, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: T={w.T} per GPU, H={w.H}, N={w.N} routed top-{w.K} "
-                               f"+ 1 shared, I={w.I}, SwiGLU, FP8 E4M3 1x128/128x128",
-                   "tokens_per_gpu": w.T, "parallelism": f"dp{world} (weak: own batch per GPU)",
-                   "routing": (f"node-limited: {args.topk_groups} of {args.groups} expert groups"
-                               if args.groups > 1 and args.topk_groups < args.groups
-                               else f"top-{w.K} of all {w.N}"),
-                   "l2": f"no flush: each step streams {weight_gb:.2f} GB of expert weights, "
-                         f"{weight_gb * 1e3 / 126:.0f}x the 126 MB L2"},
+        "config": run_config(args, w, world),
         "gemm": {"tflops": gemm_tflops, "fp8_spec_tflops": FP8_SPEC_TFLOPS,
                  "frac_of_fp8_spec": gemm_tflops / FP8_SPEC_TFLOPS,
                  "fp8_library_tflops_measured": fp8_meas,
