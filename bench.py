@@ -449,6 +449,20 @@ def run_ours(args, w, rank, world, local_rank):
     stream.wait_event(ev_out[1])
     e_end.record(stream)
     barrier()
+    # ------------------------------------------------ controller trace (untimed)
+    # workloads with several steps (the skewed one: 50) replay forward + bias
+    # update from the starting bias and record each step's max/mean load
+    trace = None
+    if w.steps > 1:
+        bias.copy_(torch.from_numpy(bias0).to(dev))
+        ratios = []
+        for _ in range(w.steps):
+            step()
+            c = layer.counts.cpu().numpy().astype(np.float64)
+            ratios.append(float(c.max() / c.mean()))
+        trace = {"steps": w.steps, "gamma": w.gamma, "load_max_over_mean": ratios,
+                 "bias_abs_max": float(bias.abs().max().item())}
+    barrier()
     # ------------------------------------------------ balance statistics (not part of the step)
     seq_len = args.seq_len or w.T
     bal_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -500,6 +514,7 @@ def run_ours(args, w, rank, world, local_rank):
                 "copies": "pinned host buffers; upload and download on side streams, "
                           "double-buffered, overlapping the neighbouring steps' kernels"},
         "clocks": clk,
+        "controller": trace,
         "balance_stats": {"ms": bal_ms, "seq_len": seq_len,
                           "note": "moe_balance_stats after the step, not part of it"},
     }

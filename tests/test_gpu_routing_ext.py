@@ -130,3 +130,32 @@ def test_balance_stats(t_count, seq_len):
     f2, p2, l2 = torch.empty_like(f), torch.empty_like(p), torch.empty_like(loss)
     capi.moe_balance_stats(sh, seq_len, 1e-4, ws, ids, f2, p2, l2)
     assert torch.equal(f, f2) and torch.equal(p, p2) and torch.equal(loss, l2)
+
+
+def test_bias_controller_trajectory():
+    """Forward + bias update repeated on a skewed router: at every step the
+    GPU counts are those of its routing (checked against the oracle's up to
+    near ties), the GPU bias equals the oracle's fp32 update of the previous
+    bias with those counts bit for bit, and the max/mean load falls."""
+    w = I.Workload("ctl", T=1024, H=512, N=32, K=4, I=128, bias_range=0.0, seed=31, zipf_s=1.2,
+                   zipf_alpha=4.0)
+    case = H.make_case(w)
+    layer = MoELayer(w.T, w.H, w.N, w.K, w.I, device_weights(w, case.pool, case.gate_w, "cuda"))
+    xd = H.x_to_device(case.x_bits)
+    bias = np.zeros(w.N, np.float32)
+    bd = torch.from_numpy(bias).cuda()
+    gamma = 5e-3
+    ratios = []
+    for step in range(30):
+        layer.route(xd, bd)
+        gid = layer.ids.cpu().numpy()
+        o_ids, _, _, score = O.route(case.x, case.gate_w, bias, w.K)
+        use, _, _ = H.reconcile_ids(gid, o_ids, score, w.K)
+        counts = layer.counts.cpu().numpy()
+        assert np.array_equal(counts, O.expert_counts(use, w.N))
+        ratios.append(counts.max() / counts.mean())
+        layer.update_bias(bd, gamma)
+        bias = O.update_bias(bias, counts, w.T, w.K, gamma)
+        assert np.array_equal(bd.cpu().numpy(), bias), step
+    # the oracle alone on this router goes from 5.8 to 1.1 in 30 steps
+    assert ratios[0] > 3.0 and ratios[-1] < 0.4 * ratios[0], ratios
