@@ -83,41 +83,52 @@ __global__ void __launch_bounds__(256) quantize_scatter_kernel(
     const uint4* __restrict__ x, int T, int H, int K, const int32_t* __restrict__ token_row,
     int64_t routed_cap, uint8_t* __restrict__ a_q, float* __restrict__ a_s,
     uint32_t* __restrict__ status) {
+  constexpr int kPerThread = 2;  // tiles in flight per thread (both loads issued first)
   const int sub = threadIdx.x & 15;
   const int tiles_per_row = H / kTile;
   const int64_t n_tiles = (int64_t)T * tiles_per_row;
-  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_tiles; base += (int64_t)gridDim.x * 16) {
-    const int64_t tile = base + (threadIdx.x >> 4);
-    const bool live = tile < n_tiles;
-    const int64_t t = live ? tile / tiles_per_row : 0;
-    const int c = live ? (int)(tile - t * tiles_per_row) : 0;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (live) v = __ldcs(x + tile * 16 + sub);
-    int my_row = -1;
-    if (live && sub < K) my_row = __ldg(token_row + t * K + sub);
-    float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                  bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-    float amax = 0.0f;
+  const int64_t step = (int64_t)gridDim.x * 16;
+  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_tiles; base += step * kPerThread) {
+    uint4 v[kPerThread];
+    int my_row[kPerThread];
+    int64_t tile[kPerThread];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    for (int u = 0; u < kPerThread; ++u) {
+      tile[u] = base + u * step + (threadIdx.x >> 4);
+      const bool live = tile[u] < n_tiles;
+      const int64_t t = live ? tile[u] / tiles_per_row : 0;
+      v[u] = live ? __ldcs(x + tile[u] * 16 + sub) : make_uint4(0, 0, 0, 0);
+      my_row[u] = (live && sub < K) ? __ldg(token_row + t * K + sub) : -1;
+    }
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = tile_scale(amax);
-    uint2 out;
-    out.x = e4m3x4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
-    out.y = e4m3x4(__fmul_rn(f[4], s), __fmul_rn(f[5], s), __fmul_rn(f[6], s), __fmul_rn(f[7], s));
-    for (int k = -1; k < K; ++k) {
-      int64_t r = routed_cap + t;
-      if (k >= 0) {
-        r = __shfl_sync(0xffffffffu, my_row, k, 16);
-        if (live && (r < 0 || r >= routed_cap)) {
-          if (sub == 0) flag_status(status, kStatusBounds);
-          continue;
+    for (int u = 0; u < kPerThread; ++u) {
+      const bool live = tile[u] < n_tiles;
+      const int64_t t = live ? tile[u] / tiles_per_row : 0;
+      const int c = live ? (int)(tile[u] - t * tiles_per_row) : 0;
+      float f[8] = {bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y),
+                    bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w)};
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float s = tile_scale(amax);
+      uint2 out;
+      out.x = e4m3x4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
+      out.y = e4m3x4(__fmul_rn(f[4], s), __fmul_rn(f[5], s), __fmul_rn(f[6], s), __fmul_rn(f[7], s));
+      for (int k = -1; k < K; ++k) {
+        int64_t r = routed_cap + t;
+        if (k >= 0) {
+          r = __shfl_sync(0xffffffffu, my_row[u], k, 16);
+          if (live && (r < 0 || r >= routed_cap)) {
+            if (sub == 0) flag_status(status, kStatusBounds);
+            continue;
+          }
         }
-      }
-      if (live) {
-        reinterpret_cast<uint2*>(a_q + r * H + (int64_t)c * kTile)[sub] = out;
-        if (sub == 0) a_s[r * tiles_per_row + c] = s;
+        if (live) {
+          reinterpret_cast<uint2*>(a_q + r * H + (int64_t)c * kTile)[sub] = out;
+          if (sub == 0) a_s[r * tiles_per_row + c] = s;
+        }
       }
     }
   }
