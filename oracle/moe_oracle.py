@@ -478,3 +478,144 @@ def moe_forward(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int,
         y_shared = expert_ffn_r(xs_rows, wg, wu, wd)
     y = combine(y_shared, y_routed, sub_ids, gates[tokens])
     return {"y": y, "ids": ids, "gates": gates, "counts": counts, "s": s}
+
+
+# ---------------------------------------------------------------------------
+# Backward of the expert path in FP8 ([Dissection] section V, Figure 6: the
+# Fprop, Dgrad and Wgrad GEMMs of every linear layer run in FP8 with E4M3
+# everywhere, fine-grained scales and fp32 accumulation; [Explained] step 7;
+# gating stays in high precision, so the router's own backward is not here:
+# the gate gradients are returned for it)
+# ---------------------------------------------------------------------------
+
+def quantize_128x1(a: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Tiles of 128 consecutive rows x 1 column: the 1x128 rule applied to
+    the transposed matrix, for operands whose GEMM reduction runs over rows
+    (the token dimension of a weight gradient). Rows are zero-padded to a
+    multiple of 128 (padding does not change a tile's amax).
+
+    Returns codes [C, R_pad] and scales [C, R_pad/128] of a.T (padded).
+    """
+    a = np.asarray(a, np.float32)
+    r, c = a.shape
+    r_pad = -(-r // TILE) * TILE
+    pad = np.zeros((max(r_pad, TILE), c), np.float32)
+    pad[:r] = a
+    return quantize_1x128(np.ascontiguousarray(pad.T))
+
+
+def dequantize_128x1(codes: np.ndarray, scales: np.ndarray, rows: int) -> np.ndarray:
+    """Inverse of quantize_128x1, back to [rows, C] float64."""
+    return dequantize_1x128(codes, scales).T[:rows]
+
+
+def silu_grad(g: np.ndarray) -> np.ndarray:
+    """d silu(g) / dg = sigmoid(g) (1 + g (1 - sigmoid(g)))."""
+    sg = 1.0 / (1.0 + np.exp(-g))
+    return sg * (1.0 + g * (1.0 - sg))
+
+
+def expert_ffn_backward_q(xq: np.ndarray, xs: np.ndarray, x: np.ndarray, dy: np.ndarray,
+                          wg: np.ndarray, wu: np.ndarray, wd: np.ndarray):
+    """FP8 backward of one expert over its rows (in the permutation's order).
+
+    xq/xs: the forward's 1x128 codes/scales of the rows' input; x: the rows'
+    input values (the bf16 x) for the weight gradient; dy: float32 [rows, H]
+    upstream gradient of the expert's output rows (already times the gate);
+    wg, wu [I, H] and wd [H, I]: dequantised weights.
+      G, U, h recomputed from the dequantised x (float64)
+      Dgrad down:  dh = Q1x128(dy) . Wd               (reduction over H)
+      SwiGLU:      dG = dh U silu'(G),  dU = dh silu(G)
+      Dgrad up:    dx = Q1x128(dG) . Wg + Q1x128(dU) . Wu   (reduction over I)
+      Wgrad down:  dWd = Q128x1(dy)^T . Q128x1(h)     (reduction over rows)
+      Wgrad up:    dWg = Q128x1(dG)^T . Q128x1(x),  dWu likewise with dU
+    Every quantised operand is the float32 rounding of its float64 value; the
+    forward's h quantisation is passed straight through (dh is the gradient
+    of the quantised h). Returns dict of float64 arrays.
+    """
+    rows = dy.shape[0]
+    x_hat = dequantize_1x128(xq, xs)
+    g = x_hat @ wg.T
+    u = x_hat @ wu.T
+    h = silu(g) * u
+    dyq, dys = quantize_1x128(np.asarray(dy, np.float32))
+    dh = dequantize_1x128(dyq, dys) @ wd
+    d_g = dh * u * silu_grad(g)
+    d_u = dh * silu(g)
+    dgq, dgs = quantize_1x128(d_g.astype(np.float32))
+    duq, dus = quantize_1x128(d_u.astype(np.float32))
+    dx = dequantize_1x128(dgq, dgs) @ wg + dequantize_1x128(duq, dus) @ wu
+    q = lambda a: dequantize_128x1(*quantize_128x1(a), rows)
+    x32 = np.asarray(x, np.float32)
+    dwd = q(np.asarray(dy, np.float32)).T @ q(h.astype(np.float32))
+    dwg = q(d_g.astype(np.float32)).T @ q(x32)
+    dwu = q(d_u.astype(np.float32)).T @ q(x32)
+    return {"dx": dx, "dwg": dwg, "dwu": dwu, "dwd": dwd, "dh": dh, "d_g": d_g, "d_u": d_u}
+
+
+def expert_ffn_backward_r(x: np.ndarray, dy: np.ndarray, wg: np.ndarray, wu: np.ndarray,
+                          wd: np.ndarray):
+    """Unquantised float64 backward of expert_ffn_r (chain rule, no FP8)."""
+    x = np.asarray(x, np.float64)
+    dy = np.asarray(dy, np.float64)
+    wg, wu, wd = (np.asarray(w, np.float64) for w in (wg, wu, wd))
+    g = x @ wg.T
+    u = x @ wu.T
+    h = silu(g) * u
+    dh = dy @ wd
+    d_g = dh * u * silu_grad(g)
+    d_u = dh * silu(g)
+    return {"dx": d_g @ wg + d_u @ wu, "dwg": d_g.T @ x, "dwu": d_u.T @ x, "dwd": dy.T @ h}
+
+
+def moe_backward(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int,
+                 weights: ExpertWeights, dy: np.ndarray, mode: str = "Q", ids=None):
+    """Backward of moe_forward's expert path for the upstream gradient dy
+    [T, H] of y, with the routing held fixed (the router's backward stays in
+    high precision and takes the gate gradients returned here):
+      dY rows: g[t,k] * dy[t] for routed slots, dy[t] for the shared expert
+      dx[t]  = sum over the token's K + 1 rows of the experts' input gradients
+      dgates[t,k] = dy[t] . Y_k[t]  (the expert's forward output row)
+      dW*: per expert (index N: the shared expert)
+    Rows of each expert in ascending token order, as the permutation lays
+    them out. Returns dict: dx [T,H], dgates [T,K], dwg/dwu [E,I,H], dwd [E,H,I].
+    """
+    x = np.asarray(x, np.float32)
+    dy = np.asarray(dy, np.float32)
+    t_count, h_dim = x.shape
+    n = gate_w.shape[0]
+    r_ids, r_gates, s, _ = route(x, gate_w, bias, k)
+    if ids is None:
+        ids, gates = r_ids, r_gates
+    else:
+        ids = np.asarray(ids, np.int32)
+        sel = np.take_along_axis(s, ids, axis=1)
+        gates = sel / np.sum(sel, axis=1, keepdims=True)
+    if mode == "Q":
+        xq, xsc = quantize_1x128(x)
+    dx = np.zeros((t_count, h_dim))
+    dgates = np.zeros((t_count, k))
+    out_w = {}
+    for e in list(np.unique(ids)) + [n]:
+        e = int(e)
+        if e == n:
+            rr = np.arange(t_count)
+            kk = None
+            dy_rows = dy.astype(np.float64)
+        else:
+            rr, kk = np.nonzero(ids == e)      # ascending token order
+            dy_rows = gates[rr, kk][:, None] * dy[rr].astype(np.float64)
+        if mode == "Q":
+            wg, wu, wd = weights.dequantised(e)
+            res = expert_ffn_backward_q(xq[rr], xsc[rr], x[rr], dy_rows.astype(np.float32),
+                                        wg, wu, wd)
+            y_e, _, _ = expert_ffn_q(xq[rr], xsc[rr], wg, wu, wd)
+        else:
+            wg, wu, wd = weights.master(e)
+            res = expert_ffn_backward_r(x[rr], dy_rows, wg, wu, wd)
+            y_e = expert_ffn_r(x[rr], wg, wu, wd)
+        np.add.at(dx, rr, res["dx"])
+        if kk is not None:
+            dgates[rr, kk] = np.sum(dy[rr].astype(np.float64) * y_e, axis=1)
+        out_w[e] = (res["dwg"], res["dwu"], res["dwd"])
+    return {"dx": dx, "dgates": dgates, "dw": out_w, "ids": ids, "gates": gates}
