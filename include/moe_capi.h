@@ -198,6 +198,59 @@ int moe_route_noalloc(moe_shape sh, const float* gate_w, const void* x, const fl
                       int32_t* topk_ids, float* topk_gates, int32_t* counts, void* stream);
 
 /*
+ * Backward of the expert path in FP8 ("DeepSeek-V3: Auxiliary-Loss-Free MoE
+ * Load Balancing, Multi-Token Prediction, and FP8 Training at 671B Scale",
+ * section V, Figure 6: Dgrad GEMMs in E4M3 with 1x128 activation tiles,
+ * 128x128 weight blocks and fp32 accumulation). Gating stays in high
+ * precision, so the router's backward is the caller's: it gets the gate
+ * gradients.
+ *
+ * moe_transpose_weights: set-up for the backward. Writes each expert's W13
+ * [2I, H] and W2 [H, I] codes transposed, and their 128x128 block scales
+ * transposed with them (a block keeps its own scale, so these are the
+ * quantised transposed weights):
+ *   w13t E4M3 [N+1, H, 2I], s13t float [N+1, H/128, 2I/128]
+ *   w2t  E4M3 [N+1, I, H],  s2t  float [N+1, I/128, H/128]
+ * Caller-owned device buffers, 16-byte aligned.
+ */
+int moe_transpose_weights(moe_shape sh, const moe_weights* w, uint8_t* w13t, float* s13t,
+                          uint8_t* w2t, float* s2t, void* stream);
+
+/*
+ * Bytes of the backward's own workspace (bws); 0 for a shape the backward
+ * does not support (it needs I to be a multiple of 256 besides the forward's
+ * rules).
+ */
+size_t moe_backward_workspace_size(moe_shape sh);
+
+/*
+ * Backward of the last moe_forward on `ws` (same x, weights and shape) for
+ * the upstream gradient dy of its output, with the routing held fixed:
+ *   dY rows    g[t,k] dy[t] for the routed slots, dy[t] for the shared expert,
+ *              quantised 1x128 along H
+ *   dh         = dY . W2 per expert (FP8 grouped GEMM on w2t), fp32
+ *   [G | U]    recomputed from the forward's quantised x rows (w13), fp32
+ *   dG, dU     = dh U silu'(G), dh silu(G), quantised 1x128
+ *   dX rows    = dG . W_gate + dU . W_up per expert (FP8 grouped GEMM on w13t)
+ *   dx[t]      = the sum of the token's K + 1 row gradients (shared first,
+ *                then slots by ascending expert id), rounded once to bf16
+ *   dgates[t,k] = dy[t] . Y_k[t] with the forward's fp32 expert output row
+ *   w: the forward's weights; wt: moe_transpose_weights' output in a
+ *   moe_weights (w13 = w13t, s13 = s13t, w2 = w2t, s2 = s2t; gate_w unused)
+ *   topk_ids, topk_gates: the forward's [T, K] outputs
+ *   dy, dx: bf16 [T, H], 16-byte aligned; dgates: float [T, K]
+ *   ws: the forward's workspace (its expert output rows are overwritten);
+ *   bws: moe_backward_workspace_size(sh) bytes, 256-byte aligned.
+ * The weight gradients (Wgrad) are not computed by this call.
+ * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE; device
+ * checks in ws's status word (moe_get_status).
+ */
+int moe_backward(moe_shape sh, const moe_weights* w, const moe_weights* wt,
+                 const int32_t* topk_ids, const float* topk_gates, const void* dy, void* ws,
+                 size_t ws_bytes, void* bws, size_t bws_bytes, void* dx, float* dgates,
+                 void* stream);
+
+/*
  * Complementary sequence-wise balance statistics ("DeepSeek-V3:
  * Auxiliary-Loss-Free MoE Load Balancing, Multi-Token Prediction, and FP8
  * Training at 671B Scale", section III; "DeepSeek-V3, explained", step 4),

@@ -61,6 +61,12 @@ SIGNATURES = {
     "moe_route_noalloc": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P]),
     "moe_balance_stats": (ctypes.c_int, [moe_shape, ctypes.c_int32, ctypes.c_float, _P, _SZ, _P,
                                          _P, _P, _P, _P]),
+    "moe_transpose_weights": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P,
+                                             _P, _P]),
+    "moe_backward_workspace_size": (_SZ, [moe_shape]),
+    "moe_backward": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights),
+                                    ctypes.POINTER(moe_weights), _P, _P, _P, _P, _SZ, _P, _SZ,
+                                    _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P, _P, _P,
                                    _P, _SZ, _P]),
     "moe_forward_traced": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P,
@@ -156,6 +162,25 @@ def moe_balance_stats(sh: moe_shape, seq_len: int, alpha: float, ws, topk_ids, f
         sh, seq_len, alpha, _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _ptr(topk_ids, torch.int32, "topk_ids"), _ptr(f, torch.float32, "f"),
         _ptr(P, torch.float32, "P"), _ptr(loss, torch.float32, "loss"), _stream(stream)))
+
+
+def moe_transpose_weights(sh: moe_shape, w: moe_weights, w13t, s13t, w2t, s2t, stream=None):
+    _check("moe_transpose_weights", LIB.moe_transpose_weights(
+        sh, ctypes.byref(w), _ptr(w13t, torch.uint8, "w13t"), _ptr(s13t, torch.float32, "s13t"),
+        _ptr(w2t, torch.uint8, "w2t"), _ptr(s2t, torch.float32, "s2t"), _stream(stream)))
+
+
+def moe_backward_workspace_size(sh: moe_shape) -> int:
+    return int(LIB.moe_backward_workspace_size(sh))
+
+
+def moe_backward(sh: moe_shape, w: moe_weights, wt: moe_weights, topk_ids, topk_gates, dy, ws,
+                 bws, dx, dgates, stream=None):
+    _check("moe_backward", LIB.moe_backward(
+        sh, ctypes.byref(w), ctypes.byref(wt), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(dy, torch.bfloat16, "dy"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _ptr(bws, torch.uint8, "bws"), bws.numel(),
+        _ptr(dx, torch.bfloat16, "dx"), _ptr(dgates, torch.float32, "dgates"), _stream(stream)))
 
 
 ROUTE_NOALLOC_MAX_LOGITS = 1048576

@@ -1,0 +1,248 @@
+// Backward of the expert path in FP8 ("DeepSeek-V3: Auxiliary-Loss-Free MoE
+// Load Balancing, Multi-Token Prediction, and FP8 Training at 671B Scale",
+// section V, Figure 6: the Dgrad GEMMs of every linear layer in E4M3 with
+// fine-grained scales and fp32 accumulation; gating stays in high precision,
+// so the router's own backward is left to the caller, who gets the gate
+// gradients). The GEMMs are the forward's grouped FP8 kernel with the
+// weights' 128x128 blocks transposed; the kernels here are the element-wise
+// steps around them:
+//   transpose_blocks    set-up: W [rows, cols] -> W^T per group, codes and
+//                       block scales (a 128x128 block's scale is its own)
+//   dy_rows_quantize    dY rows = g[t,k] dy[t] (routed) and dy[t] (shared),
+//                       1x128-quantised into the forward's row order
+//   swiglu_backward     dG = dh U silu'(G), dU = dh silu(G) from the
+//                       recomputed [G|U] rows, 1x128-quantised in the
+//                       gate/up-interleaved order of w13
+//   gate_grad           dgates[t,k] = dy[t] . Y[row(t,k)]
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+// One CTA per 128x128 block of one group: bytes through shared memory.
+__global__ void __launch_bounds__(256) transpose_blocks_kernel(const uint8_t* __restrict__ w,
+                                                               const float* __restrict__ s,
+                                                               int64_t rows, int64_t cols,
+                                                               uint8_t* __restrict__ wt,
+                                                               float* __restrict__ st) {
+  __shared__ uint8_t tile[kTile][kTile + 4];
+  const int64_t cb = blockIdx.x, rb = blockIdx.y, g = blockIdx.z;
+  const uint8_t* src = w + g * rows * cols + rb * kTile * cols + cb * kTile;
+  for (int i = threadIdx.x; i < kTile * kTile; i += blockDim.x) {
+    const int r = i / kTile, c = i % kTile;
+    tile[r][c] = src[(int64_t)r * cols + c];
+  }
+  __syncthreads();
+  uint8_t* dst = wt + g * rows * cols + cb * kTile * rows + rb * kTile;
+  for (int i = threadIdx.x; i < kTile * kTile; i += blockDim.x) {
+    const int r = i / kTile, c = i % kTile;  // destination row r (a source column)
+    dst[(int64_t)r * rows + c] = tile[c][r];
+  }
+  if (threadIdx.x == 0) {
+    const int64_t rbn = rows / kTile, cbn = cols / kTile;
+    st[g * rbn * cbn + cb * rbn + rb] = s[g * rbn * cbn + rb * cbn + cb];
+  }
+}
+
+// 16 threads per 128-column tile of dy[t]; for each of the token's K + 1
+// GEMM rows the tile is scaled by that row's gate (1 for the shared row),
+// its amax reduced over the 16 threads and the codes written.
+__global__ void __launch_bounds__(256) dy_rows_quantize_kernel(
+    const uint4* __restrict__ dy, const float* __restrict__ gates, int T, int H, int K,
+    const int32_t* __restrict__ token_row, int64_t routed_cap, uint8_t* __restrict__ q,
+    float* __restrict__ qs, uint32_t* __restrict__ status) {
+  const int sub = threadIdx.x & 15;
+  const int tiles_per_row = H / kTile;
+  const int64_t n_tiles = (int64_t)T * tiles_per_row;
+  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_tiles; base += (int64_t)gridDim.x * 16) {
+    const int64_t tile = base + (threadIdx.x >> 4);
+    const bool live = tile < n_tiles;
+    const int64_t t = live ? tile / tiles_per_row : 0;
+    const int c = live ? (int)(tile - t * tiles_per_row) : 0;
+    const uint4 v = live ? __ldg(dy + tile * 16 + sub) : make_uint4(0, 0, 0, 0);
+    int my_row = -1;
+    float my_gate = 0.0f;
+    if (live && sub < K) {
+      my_row = __ldg(token_row + t * K + sub);
+      my_gate = __ldg(gates + t * K + sub);
+    }
+    const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    for (int k = -1; k < K; ++k) {
+      int64_t r = routed_cap + t;
+      float g = 1.0f;
+      if (k >= 0) {
+        r = __shfl_sync(0xffffffffu, my_row, k, 16);
+        g = __shfl_sync(0xffffffffu, my_gate, k, 16);
+      }
+      float d[8];
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        d[i] = __fmul_rn(g, f[i]);
+        amax = fmaxf(amax, fabsf(d[i]));
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (!live) continue;
+      if (k >= 0 && (r < 0 || r >= routed_cap)) {
+        if (sub == 0) flag_status(status, kStatusBounds);
+        continue;
+      }
+      const float s = tile_scale(amax);
+      uint2 out;
+      out.x = e4m3x4(__fmul_rn(d[0], s), __fmul_rn(d[1], s), __fmul_rn(d[2], s), __fmul_rn(d[3], s));
+      out.y = e4m3x4(__fmul_rn(d[4], s), __fmul_rn(d[5], s), __fmul_rn(d[6], s), __fmul_rn(d[7], s));
+      reinterpret_cast<uint2*>(q + r * H + (int64_t)c * kTile)[sub] = out;
+      if (sub == 0) qs[r * tiles_per_row + c] = s;
+    }
+  }
+}
+
+// 16 threads per (row, 128-channel block c): the block's 128 G and 128 U
+// values sit at columns [256c, 256c + 128) and [256c + 128, 256c + 256) of the
+// recomputed rows (w13's row order); dG and dU are quantised as two 1x128
+// tiles at the same positions of the output rows.
+__global__ void __launch_bounds__(256) swiglu_backward_kernel(
+    const float* __restrict__ gu, const float* __restrict__ dh, int64_t rows, int I,
+    uint8_t* __restrict__ q, float* __restrict__ qs) {
+  const int sub = threadIdx.x & 15;
+  const int blocks = I / kTile;
+  const int64_t n_units = rows * blocks;
+  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_units; base += (int64_t)gridDim.x * 16) {
+    const int64_t unit = base + (threadIdx.x >> 4);
+    const bool live = unit < n_units;
+    const int64_t r = live ? unit / blocks : 0;
+    const int c = live ? (int)(unit - r * blocks) : 0;
+    float dg[8], du[8];
+    float ag = 0.0f, au = 0.0f;
+    if (live) {
+      const float4* gp = reinterpret_cast<const float4*>(gu + r * 2 * I + (int64_t)c * 2 * kTile);
+      const float4* hp = reinterpret_cast<const float4*>(dh + r * I + (int64_t)c * kTile);
+      const float4 g0 = __ldg(gp + 2 * sub), g1 = __ldg(gp + 2 * sub + 1);
+      const float4 u0 = __ldg(gp + 32 + 2 * sub), u1 = __ldg(gp + 32 + 2 * sub + 1);
+      const float4 h0 = __ldg(hp + 2 * sub), h1 = __ldg(hp + 2 * sub + 1);
+      const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // sigmoid with the hardware exp2 and reciprocal, as the forward's SiLU
+        const float sg = __fdividef(1.0f, 1.0f + __expf(-gv[i]));
+        const float dsilu = sg * (1.0f + gv[i] * (1.0f - sg));
+        dg[i] = hv[i] * uv[i] * dsilu;
+        du[i] = hv[i] * (gv[i] * sg);
+        ag = fmaxf(ag, fabsf(dg[i]));
+        au = fmaxf(au, fabsf(du[i]));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dg[i] = du[i] = 0.0f;
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) {
+      ag = fmaxf(ag, __shfl_xor_sync(0xffffffffu, ag, o));
+      au = fmaxf(au, __shfl_xor_sync(0xffffffffu, au, o));
+    }
+    if (!live) continue;
+    const float sg_ = tile_scale(ag), su = tile_scale(au);
+    uint2 og, ou;
+    og.x = e4m3x4(__fmul_rn(dg[0], sg_), __fmul_rn(dg[1], sg_), __fmul_rn(dg[2], sg_), __fmul_rn(dg[3], sg_));
+    og.y = e4m3x4(__fmul_rn(dg[4], sg_), __fmul_rn(dg[5], sg_), __fmul_rn(dg[6], sg_), __fmul_rn(dg[7], sg_));
+    ou.x = e4m3x4(__fmul_rn(du[0], su), __fmul_rn(du[1], su), __fmul_rn(du[2], su), __fmul_rn(du[3], su));
+    ou.y = e4m3x4(__fmul_rn(du[4], su), __fmul_rn(du[5], su), __fmul_rn(du[6], su), __fmul_rn(du[7], su));
+    uint8_t* row = q + r * 2 * I + (int64_t)c * 2 * kTile;
+    reinterpret_cast<uint2*>(row)[sub] = og;
+    reinterpret_cast<uint2*>(row + kTile)[sub] = ou;
+    if (sub == 0) {
+      qs[r * 2 * blocks + 2 * c] = sg_;
+      qs[r * 2 * blocks + 2 * c + 1] = su;
+    }
+  }
+}
+
+// One warp per (token, slot): dgates[t, k] = dy[t] . Y[token_row[t, k]] in fp32
+// (lane-strided partial sums, then a fixed butterfly).
+__global__ void __launch_bounds__(256) gate_grad_kernel(const __nv_bfloat16* __restrict__ dy,
+                                                        const float* __restrict__ y_rows,
+                                                        const int32_t* __restrict__ token_row,
+                                                        int T, int H, int K, int64_t routed_cap,
+                                                        float* __restrict__ dgates,
+                                                        uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t p = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < (int64_t)T * K;
+       p += warps) {
+    const int64_t t = p / K;
+    const int64_t r = token_row[p];
+    if (r < 0 || r >= routed_cap) {
+      if (lane == 0) flag_status(status, kStatusBounds);
+      continue;
+    }
+    const uint2* d2 = reinterpret_cast<const uint2*>(dy + t * H);
+    const float4* y4 = reinterpret_cast<const float4*>(y_rows + r * H);
+    float acc = 0.0f;
+    for (int i = lane; i < H / 4; i += 32) {
+      const uint2 d = __ldg(d2 + i);
+      const float4 yv = __ldg(y4 + i);
+      acc = fmaf(bf16_lo(d.x), yv.x, acc);
+      acc = fmaf(bf16_hi(d.x), yv.y, acc);
+      acc = fmaf(bf16_lo(d.y), yv.z, acc);
+      acc = fmaf(bf16_hi(d.y), yv.w, acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) dgates[p] = acc;
+  }
+}
+
+int grid_for(int64_t units, int per_cta, int sm_count) {
+  int64_t blocks = (units + per_cta - 1) / per_cta;
+  const int64_t cap = (int64_t)sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  return (int)(blocks > 0 ? blocks : 1);
+}
+
+}  // namespace
+
+cudaError_t launch_transpose_blocks(const uint8_t* w, const float* s, int64_t groups, int64_t rows,
+                                    int64_t cols, uint8_t* wt, float* st, cudaStream_t stream) {
+  if (groups == 0) return cudaSuccess;
+  dim3 grid((unsigned)(cols / kTile), (unsigned)(rows / kTile), (unsigned)groups);
+  transpose_blocks_kernel<<<grid, 256, 0, stream>>>(w, s, rows, cols, wt, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dy_rows_quantize(const void* dy, const float* gates, int T, int H, int K,
+                                    const int32_t* token_row, int64_t routed_cap, uint8_t* q,
+                                    float* qs, uint32_t* status, cudaStream_t stream,
+                                    int sm_count) {
+  const int64_t n_tiles = (int64_t)T * (H / kTile);
+  if (n_tiles == 0) return cudaSuccess;
+  dy_rows_quantize_kernel<<<grid_for(n_tiles, 16, sm_count), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(dy), gates, T, H, K, token_row, routed_cap, q, qs, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_backward(const float* gu, const float* dh, int64_t rows, int I,
+                                   uint8_t* q, float* qs, cudaStream_t stream, int sm_count) {
+  const int64_t units = rows * (I / kTile);
+  if (units == 0) return cudaSuccess;
+  swiglu_backward_kernel<<<grid_for(units, 16, sm_count), 256, 0, stream>>>(gu, dh, rows, I, q,
+                                                                           qs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_grad(const void* dy, const float* y_rows, const int32_t* token_row, int T,
+                             int H, int K, int64_t routed_cap, float* dgates, uint32_t* status,
+                             cudaStream_t stream, int sm_count) {
+  const int64_t pairs = (int64_t)T * K;
+  if (pairs == 0) return cudaSuccess;
+  gate_grad_kernel<<<grid_for(pairs, 8, sm_count), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(dy), y_rows, token_row, T, H, K, routed_cap, dgates,
+      status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

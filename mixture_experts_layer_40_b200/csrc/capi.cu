@@ -367,6 +367,123 @@ int moe_expert_down(int32_t H, int32_t I, int32_t n_groups, const int32_t* group
                                         static_cast<cudaStream_t>(stream), sm_count()));
 }
 
+int moe_transpose_weights(moe_shape sh, const moe_weights* w, uint8_t* w13t, float* s13t,
+                          uint8_t* w2t, float* s2t, void* stream) {
+  if (!shape_ok(sh)) return MOE_ERR_SHAPE;
+  if (!w || !w->w13 || !w->s13 || !w->w2 || !w->s2) return MOE_ERR_NULL;
+  if (!w13t || !s13t || !w2t || !s2t) return MOE_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t E = sh.N + 1, H = sh.H, I = sh.I;
+  cudaError_t e = launch_transpose_blocks(w->w13, w->s13, E, 2 * I, H, w13t, s13t, s);
+  if (e == cudaSuccess) e = launch_transpose_blocks(w->w2, w->s2, E, H, I, w2t, s2t, s);
+  return cuda_status(e);
+}
+
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+struct BackwardLayout {
+  size_t dy_q, dy_s, gu, dh, dgu_q, dgu_s, total;
+};
+
+BackwardLayout backward_layout(const moe_shape& sh) {
+  moe_ws_layout L;
+  layout_of(sh, &L);
+  const size_t R = (size_t)L.rows_total, H = sh.H, I = sh.I;
+  BackwardLayout B{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = (off + bytes + 255) / 256 * 256;
+    return at;
+  };
+  B.dy_q = take(R * H);
+  B.dy_s = take(R * (H / kTile) * 4);
+  B.gu = take(R * 2 * I * 4);
+  B.dh = take(R * I * 4);
+  B.dgu_q = take(R * 2 * I);
+  B.dgu_s = take(R * (2 * I / kTile) * 4);
+  B.total = off;
+  return B;
+}
+
+bool backward_shape_ok(const moe_shape& sh) { return shape_ok(sh) && sh.I % 256 == 0; }
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+size_t moe_backward_workspace_size(moe_shape sh) {
+  if (!backward_shape_ok(sh)) return 0;
+  return backward_layout(sh).total;
+}
+
+int moe_backward(moe_shape sh, const moe_weights* w, const moe_weights* wt,
+                 const int32_t* topk_ids, const float* topk_gates, const void* dy, void* ws,
+                 size_t ws_bytes, void* bws, size_t bws_bytes, void* dx, float* dgates,
+                 void* stream) {
+  if (!backward_shape_ok(sh)) return MOE_ERR_SHAPE;
+  if (!w || !wt || !ws || !bws) return MOE_ERR_NULL;
+  moe_ws_layout L;
+  layout_of(sh, &L);
+  const BackwardLayout B = backward_layout(sh);
+  if (ws_bytes < L.total || bws_bytes < B.total) return MOE_ERR_WORKSPACE;
+  if (!aligned(ws, 256) || !aligned(bws, 256)) return MOE_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  if (sh.T == 0) return cuda_status(cudaMemsetAsync(status, 0, 4, s));
+  if (!topk_ids || !topk_gates || !dy || !dx || !dgates) return MOE_ERR_NULL;
+  if (!w->w13 || !w->s13 || !wt->w13 || !wt->s13 || !wt->w2 || !wt->s2) return MOE_ERR_NULL;
+  if (!aligned(dy, 16) || !aligned(dx, 16) || !aligned(w->w13, 16) || !aligned(wt->w13, 16) ||
+      !aligned(wt->w2, 16))
+    return MOE_ERR_ALIGN;
+  const int sms = sm_count();
+  const int32_t* token_row = at<int32_t>(ws, L.token_row);
+  float* y_rows = at<float>(ws, L.y_rows);
+  cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
+  // gate gradients from the forward's fp32 expert output rows (before the
+  // rows buffer is reused for the input gradients)
+  if (e == cudaSuccess)
+    e = launch_gate_grad(dy, y_rows, token_row, sh.T, sh.H, sh.K, L.routed_cap, dgates, status, s,
+                         sms);
+  // dY rows: g dy (routed), dy (shared), 1x128 along H
+  if (e == cudaSuccess)
+    e = launch_dy_rows_quantize(dy, topk_gates, sh.T, sh.H, sh.K, token_row, L.routed_cap,
+                                at<uint8_t>(bws, B.dy_q), at<float>(bws, B.dy_s), status, s, sms);
+  const int32_t* gr = at<int32_t>(ws, L.group_rows);
+  const int32_t* gs = at<int32_t>(ws, L.row_start);
+  // [G | U] recomputed from the forward's x rows: fp32 [rows, 2I]
+  if (e == cudaSuccess) {
+    GroupedGemm gg{2 * sh.I, sh.H, sh.N + 1, gr, gs, L.rows_total, status};
+    e = launch_expert_down(gg, at<uint8_t>(ws, L.a_q), at<float>(ws, L.a_s), w->w13, w->s13,
+                           at<float>(bws, B.gu), s, sms);
+  }
+  // Dgrad of the down projection: dh = dY . W2, fp32 [rows, I]
+  if (e == cudaSuccess) {
+    GroupedGemm gg{sh.I, sh.H, sh.N + 1, gr, gs, L.rows_total, status};
+    e = launch_expert_down(gg, at<uint8_t>(bws, B.dy_q), at<float>(bws, B.dy_s), wt->w2, wt->s2,
+                           at<float>(bws, B.dh), s, sms);
+  }
+  // SwiGLU backward, [dG | dU] 1x128 in w13's row order
+  if (e == cudaSuccess)
+    e = launch_swiglu_backward(at<float>(bws, B.gu), at<float>(bws, B.dh), L.rows_total, sh.I,
+                               at<uint8_t>(bws, B.dgu_q), at<float>(bws, B.dgu_s), s, sms);
+  // Dgrad of the up/gate projection: dX rows = [dG | dU] . W13, fp32 [rows, H]
+  if (e == cudaSuccess) {
+    GroupedGemm gg{sh.H, 2 * sh.I, sh.N + 1, gr, gs, L.rows_total, status};
+    e = launch_expert_down(gg, at<uint8_t>(bws, B.dgu_q), at<float>(bws, B.dgu_s), wt->w13,
+                           wt->s13, y_rows, s, sms);
+  }
+  // dx[t] = the token's K + 1 row gradients, fixed order, one bf16 rounding
+  if (e == cudaSuccess)
+    e = launch_combine(y_rows, topk_ids, nullptr, token_row, sh.T, sh.H, sh.K, L.routed_cap,
+                       L.rows_total, static_cast<__nv_bfloat16*>(dx), status, s);
+  return cuda_status(e);
+}
+
 int moe_get_status(void* ws, void* stream) {
   if (!ws) return MOE_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
     for (int k = 0; k < K; ++k) {
       const int e = ids[(int64_t)t * K + k];
       const int64_t r = token_row[(int64_t)t * K + k];
-      const float g = gates[(int64_t)t * K + k];
+      const float g = gates != nullptr ? gates[(int64_t)t * K + k] : 1.0f;
       if (r < 0 || r >= routed_cap) {
         flag_status(status, kStatusBounds);
         continue;

@@ -52,6 +52,19 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
                              int32_t* ids, float* gates, int32_t* counts, uint32_t* status,
                              cudaStream_t stream, int sm_count);
 
+// Backward of the expert path (backward.cu).
+cudaError_t launch_transpose_blocks(const uint8_t* w, const float* s, int64_t groups, int64_t rows,
+                                    int64_t cols, uint8_t* wt, float* st, cudaStream_t stream);
+cudaError_t launch_dy_rows_quantize(const void* dy, const float* gates, int T, int H, int K,
+                                    const int32_t* token_row, int64_t routed_cap, uint8_t* q,
+                                    float* qs, uint32_t* status, cudaStream_t stream,
+                                    int sm_count);
+cudaError_t launch_swiglu_backward(const float* gu, const float* dh, int64_t rows, int I,
+                                   uint8_t* q, float* qs, cudaStream_t stream, int sm_count);
+cudaError_t launch_gate_grad(const void* dy, const float* y_rows, const int32_t* token_row, int T,
+                             int H, int K, int64_t routed_cap, float* dgates, uint32_t* status,
+                             cudaStream_t stream, int sm_count);
+
 // Sequence-wise balance statistics from the router's logits and top-K ids
 // (f, P [S, N], loss [S]); scratch of balance_scratch_bytes(T, N) bytes.
 size_t balance_scratch_bytes(int64_t T, int64_t N);

@@ -110,6 +110,31 @@ class MoELayer:
         capi.moe_balance_stats(self.shape, seq_len, alpha, self.ws, self.ids, f, p, loss, stream)
         return f, p, loss
 
+    def backward(self, dy: torch.Tensor, stream=None):
+        """Input and gate gradients of the last forward for the upstream
+        gradient dy (bf16 [T, H]); the transposed weights and the backward
+        workspace are made on first use. Returns (dx bf16 [T, H], dgates)."""
+        if getattr(self, "_wt", None) is None:
+            E, H, I = self.N + 1, self.H, self.I
+            dev = self.device
+            self._wt_bufs = (torch.empty((E, H, 2 * I), dtype=torch.uint8, device=dev),
+                             torch.empty((E, H // 128, 2 * I // 128), dtype=torch.float32,
+                                         device=dev),
+                             torch.empty((E, I, H), dtype=torch.uint8, device=dev),
+                             torch.empty((E, I // 128, H // 128), dtype=torch.float32, device=dev))
+            capi.moe_transpose_weights(self.shape, self._cw, *self._wt_bufs, stream)
+            nb = capi.moe_backward_workspace_size(self.shape)
+            if nb == 0:
+                raise ValueError("the backward needs I to be a multiple of 256")
+            self._bws = torch.empty(nb, dtype=torch.uint8, device=dev)
+            w13t, s13t, w2t, s2t = self._wt_bufs
+            self._wt = capi.make_weights(self.weights.gate_w, w13t, s13t, w2t, s2t)
+        dx = torch.empty((self.T, self.H), dtype=torch.bfloat16, device=self.device)
+        dgates = torch.empty((self.T, self.K), dtype=torch.float32, device=self.device)
+        capi.moe_backward(self.shape, self._cw, self._wt, self.ids, self.gates, dy, self.ws,
+                          self._bws, dx, dgates, stream)
+        return dx, dgates
+
     def update_bias(self, bias: torch.Tensor, gamma: float, stream=None) -> None:
         capi.moe_update_bias(bias, self.counts, self.N, self.T, self.K, gamma, stream)
 

@@ -569,7 +569,8 @@ def expert_ffn_backward_r(x: np.ndarray, dy: np.ndarray, wg: np.ndarray, wu: np.
 
 
 def moe_backward(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int,
-                 weights: ExpertWeights, dy: np.ndarray, mode: str = "Q", ids=None):
+                 weights: ExpertWeights, dy: np.ndarray, mode: str = "Q", ids=None,
+                 tokens=None):
     """Backward of moe_forward's expert path for the upstream gradient dy
     [T, H] of y, with the routing held fixed (the router's backward stays in
     high precision and takes the gate gradients returned here):
@@ -578,7 +579,13 @@ def moe_backward(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int,
       dgates[t,k] = dy[t] . Y_k[t]  (the expert's forward output row)
       dW*: per expert (index N: the shared expert)
     Rows of each expert in ascending token order, as the permutation lays
-    them out. Returns dict: dx [T,H], dgates [T,K], dwg/dwu [E,I,H], dwd [E,H,I].
+    them out. With `tokens` (a subset), only those tokens' rows are run: dx
+    and dgates of a token depend on its own rows alone (every Dgrad
+    quantisation tile lies in one row), so they equal the full run's up to
+    float64 rounding order; the weight gradients, which need every row, are
+    then not returned.
+    Returns dict: dx [T,H], dgates [T,K], dw {expert: (dwg [I,H], dwu [I,H],
+    dwd [H,I])}.
     """
     x = np.asarray(x, np.float32)
     dy = np.asarray(dy, np.float32)
@@ -596,14 +603,16 @@ def moe_backward(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int,
     dx = np.zeros((t_count, h_dim))
     dgates = np.zeros((t_count, k))
     out_w = {}
-    for e in list(np.unique(ids)) + [n]:
+    keep = np.zeros(t_count, bool)
+    keep[np.arange(t_count) if tokens is None else np.asarray(tokens)] = True
+    for e in list(np.unique(ids[keep])) + [n]:
         e = int(e)
         if e == n:
-            rr = np.arange(t_count)
+            rr = np.nonzero(keep)[0]
             kk = None
-            dy_rows = dy.astype(np.float64)
+            dy_rows = dy[rr].astype(np.float64)
         else:
-            rr, kk = np.nonzero(ids == e)      # ascending token order
+            rr, kk = np.nonzero((ids == e) & keep[:, None])   # ascending token order
             dy_rows = gates[rr, kk][:, None] * dy[rr].astype(np.float64)
         if mode == "Q":
             wg, wu, wd = weights.dequantised(e)
@@ -617,5 +626,6 @@ def moe_backward(x: np.ndarray, gate_w: np.ndarray, bias: np.ndarray, k: int,
         np.add.at(dx, rr, res["dx"])
         if kk is not None:
             dgates[rr, kk] = np.sum(dy[rr].astype(np.float64) * y_e, axis=1)
-        out_w[e] = (res["dwg"], res["dwu"], res["dwd"])
+        if tokens is None:
+            out_w[e] = (res["dwg"], res["dwu"], res["dwd"])
     return {"dx": dx, "dgates": dgates, "dw": out_w, "ids": ids, "gates": gates}

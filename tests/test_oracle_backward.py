@@ -135,3 +135,15 @@ def test_quantize_128x1_tiles_run_down_the_rows():
     assert not np.any(codes[:, 200:])            # zero padding
     back = O.dequantize_128x1(codes, scales, 200)
     assert np.all(np.abs(back - a) <= np.abs(a) * 2.0 ** -4 + 2.0 ** -10 / np.repeat(scales, 128, 1).T[:200])
+
+
+def test_token_subset_matches_full_run():
+    w, ew, x, gw, b, dy = _small(t=40, n=16, k=4, seed=45)
+    full = O.moe_backward(x, gw, b, w.K, ew, dy, mode="Q")
+    toks = [3, 17, 29]
+    sub = O.moe_backward(x, gw, b, w.K, ew, dy, mode="Q", tokens=toks)
+    np.testing.assert_allclose(sub["dx"][toks], full["dx"][toks], rtol=0,
+                               atol=1e-12 * np.abs(full["dx"]).max())
+    np.testing.assert_allclose(sub["dgates"][toks], full["dgates"][toks], rtol=0,
+                               atol=1e-12 * np.abs(full["dgates"]).max())
+    assert sub["dw"] == {}
