@@ -235,20 +235,27 @@ size_t moe_backward_workspace_size(moe_shape sh);
  *   dx[t]      = the sum of the token's K + 1 row gradients (shared first,
  *                then slots by ascending expert id), rounded once to bf16
  *   dgates[t,k] = dy[t] . Y_k[t] with the forward's fp32 expert output row
+ *   dw2 [N+1, H, I] = per expert, dY^T . h over its rows (Wgrad), fp32
+ *   dw13 [N+1, 2I, H] = per expert, [dG | dU]^T . x over its rows, in w13's
+ *                row order (gate block c, then up block c), fp32
+ * Wgrad operands are quantised in tiles of 128 GEMM rows x 1 channel (the
+ * tiles run along the reduction, which is over tokens here), h and dG/dU
+ * from the recomputed [G | U] and dh, x from the bf16 input.
  *   w: the forward's weights; wt: moe_transpose_weights' output in a
  *   moe_weights (w13 = w13t, s13 = s13t, w2 = w2t, s2 = s2t; gate_w unused)
- *   topk_ids, topk_gates: the forward's [T, K] outputs
+ *   topk_ids, topk_gates: the forward's [T, K] outputs; x: its bf16 input
+ *   (only read for the weight gradients; may be NULL without them)
  *   dy, dx: bf16 [T, H], 16-byte aligned; dgates: float [T, K]
+ *   dw13, dw2: the weight gradients, or both NULL to skip them
  *   ws: the forward's workspace (its expert output rows are overwritten);
  *   bws: moe_backward_workspace_size(sh) bytes, 256-byte aligned.
- * The weight gradients (Wgrad) are not computed by this call.
  * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE; device
  * checks in ws's status word (moe_get_status).
  */
 int moe_backward(moe_shape sh, const moe_weights* w, const moe_weights* wt,
-                 const int32_t* topk_ids, const float* topk_gates, const void* dy, void* ws,
-                 size_t ws_bytes, void* bws, size_t bws_bytes, void* dx, float* dgates,
-                 void* stream);
+                 const int32_t* topk_ids, const float* topk_gates, const void* x, const void* dy,
+                 void* ws, size_t ws_bytes, void* bws, size_t bws_bytes, void* dx, float* dgates,
+                 float* dw13, float* dw2, void* stream);
 
 /*
  * Complementary sequence-wise balance statistics ("DeepSeek-V3:

@@ -65,8 +65,8 @@ SIGNATURES = {
                                              _P, _P]),
     "moe_backward_workspace_size": (_SZ, [moe_shape]),
     "moe_backward": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights),
-                                    ctypes.POINTER(moe_weights), _P, _P, _P, _P, _SZ, _P, _SZ,
-                                    _P, _P, _P]),
+                                    ctypes.POINTER(moe_weights), _P, _P, _P, _P, _P, _SZ, _P, _SZ,
+                                    _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P, _P, _P,
                                    _P, _SZ, _P]),
     "moe_forward_traced": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_weights), _P, _P, _P, _P,
@@ -174,13 +174,15 @@ def moe_backward_workspace_size(sh: moe_shape) -> int:
     return int(LIB.moe_backward_workspace_size(sh))
 
 
-def moe_backward(sh: moe_shape, w: moe_weights, wt: moe_weights, topk_ids, topk_gates, dy, ws,
-                 bws, dx, dgates, stream=None):
+def moe_backward(sh: moe_shape, w: moe_weights, wt: moe_weights, topk_ids, topk_gates, x, dy, ws,
+                 bws, dx, dgates, dw13=None, dw2=None, stream=None):
     _check("moe_backward", LIB.moe_backward(
         sh, ctypes.byref(w), ctypes.byref(wt), _ptr(topk_ids, torch.int32, "topk_ids"),
-        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(dy, torch.bfloat16, "dy"),
-        _ptr(ws, torch.uint8, "ws"), ws.numel(), _ptr(bws, torch.uint8, "bws"), bws.numel(),
-        _ptr(dx, torch.bfloat16, "dx"), _ptr(dgates, torch.float32, "dgates"), _stream(stream)))
+        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(x, torch.bfloat16, "x"),
+        _ptr(dy, torch.bfloat16, "dy"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _ptr(bws, torch.uint8, "bws"), bws.numel(), _ptr(dx, torch.bfloat16, "dx"),
+        _ptr(dgates, torch.float32, "dgates"), _ptr(dw13, torch.float32, "dw13"),
+        _ptr(dw2, torch.float32, "dw2"), _stream(stream)))
 
 
 ROUTE_NOALLOC_MAX_LOGITS = 1048576

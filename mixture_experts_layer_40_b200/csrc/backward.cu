@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) transpose_blocks_kernel(const uint8_t* __
 __global__ void __launch_bounds__(256) dy_rows_quantize_kernel(
     const uint4* __restrict__ dy, const float* __restrict__ gates, int T, int H, int K,
     const int32_t* __restrict__ token_row, int64_t routed_cap, uint8_t* __restrict__ q,
-    float* __restrict__ qs, uint32_t* __restrict__ status) {
+    float* __restrict__ qs, float* __restrict__ row_gate, uint32_t* __restrict__ status) {
   const int sub = threadIdx.x & 15;
   const int tiles_per_row = H / kTile;
   const int64_t n_tiles = (int64_t)T * tiles_per_row;
@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(256) dy_rows_quantize_kernel(
       out.y = e4m3x4(__fmul_rn(d[4], s), __fmul_rn(d[5], s), __fmul_rn(d[6], s), __fmul_rn(d[7], s));
       reinterpret_cast<uint2*>(q + r * H + (int64_t)c * kTile)[sub] = out;
       if (sub == 0) qs[r * tiles_per_row + c] = s;
+      if (sub == 0 && c == 0 && row_gate != nullptr) row_gate[r] = g;
     }
   }
 }
@@ -197,6 +198,87 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const __nv_bfloat16* __r
   }
 }
 
+// Column tiles for the weight gradients: 128 GEMM rows x 1 channel. One CTA
+// per 128-row block and 32 channels: the values (computed on the fly from
+// the source, 0 on padding rows) go through shared memory, 8 threads reduce
+// each channel's amax over the 128 rows, and each writes 16 codes of the
+// channel's transposed row. A operands keep the scale ([C, R/128]); B
+// operands store its inverse, block-major ([R/128, C]), for the per-column
+// promotion of the weight-gradient GEMM.
+enum ColSource { kColDy = 0, kColX = 1, kColH = 2, kColDgu = 3 };
+
+struct ColArgs {
+  const int32_t* row_token;   // [routed_cap] token of each routed GEMM row, -1 on padding
+  int64_t routed_cap;         // rows from here on are the shared expert's: token r - routed_cap
+  int T;
+  const float* row_gate;      // [R] gate of the row's slot (1: shared row)
+  const __nv_bfloat16* src;   // dy or x [T, C] (kColDy, kColX)
+  const float* gu;            // [R, 2I] recomputed G/U rows (kColH, kColDgu)
+  const float* dh;            // [R, I] (kColDgu)
+  int64_t R;                  // GEMM rows (multiple of 128)
+  int C;                      // channels of the output
+  int I;
+  uint8_t* codes;             // [C, R]
+  float* scales;              // A: [C, R/128]; B: inverse, [R/128, C]
+  bool b_operand;
+};
+
+template <int kSrc>
+MOE_DEV float col_value(const ColArgs& a, int64_t r, int c) {
+  const int64_t rs = r - a.routed_cap;
+  const int t = r < a.routed_cap ? a.row_token[r] : (rs < a.T ? (int)rs : -1);
+  if (t < 0) return 0.0f;
+  if (kSrc == kColDy) return __fmul_rn(a.row_gate[r], __bfloat162float(a.src[(int64_t)t * a.C + c]));
+  if (kSrc == kColX) return __bfloat162float(a.src[(int64_t)t * a.C + c]);
+  if (kSrc == kColH) {
+    const float* row = a.gu + r * 2 * a.I + (int64_t)(c / 128) * 256 + c % 128;
+    const float g = row[0], u = row[128];
+    const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+    return g * sg * u;
+  }
+  // kColDgu: channel c of w13's order; block c / 256 holds 128 gate then 128 up
+  const int j = c % 256, ch = (c / 256) * 128 + (j % 128);
+  const float* row = a.gu + r * 2 * a.I + (int64_t)(c / 256) * 256 + (j % 128);
+  const float g = row[0], u = row[128];
+  const float d = a.dh[r * a.I + ch];
+  const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+  return j < 128 ? d * u * (sg * (1.0f + g * (1.0f - sg))) : d * (g * sg);
+}
+
+template <int kSrc>
+__global__ void __launch_bounds__(256) quantize_cols_kernel(const ColArgs a) {
+  __shared__ float vals[kTile][33];
+  const int64_t rb = blockIdx.x;
+  const int c0 = blockIdx.y * 32;
+  for (int i = threadIdx.x; i < kTile * 32; i += blockDim.x) {
+    const int r = i >> 5, c = i & 31;
+    vals[r][c] = (c0 + c < a.C) ? col_value<kSrc>(a, rb * kTile + r, c0 + c) : 0.0f;
+  }
+  __syncthreads();
+  const int c = threadIdx.x >> 3, part = threadIdx.x & 7;  // 8 threads per channel
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(vals[part * 16 + i][c]));
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (c0 + c >= a.C) return;
+  const float s = tile_scale(amax);
+  uint4 out;
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    w[k] = e4m3x4(__fmul_rn(vals[part * 16 + 4 * k][c], s), __fmul_rn(vals[part * 16 + 4 * k + 1][c], s),
+                  __fmul_rn(vals[part * 16 + 4 * k + 2][c], s), __fmul_rn(vals[part * 16 + 4 * k + 3][c], s));
+  out = make_uint4(w[0], w[1], w[2], w[3]);
+  reinterpret_cast<uint4*>(a.codes + (int64_t)(c0 + c) * a.R + rb * kTile)[part] = out;
+  if (part == 0) {
+    if (a.b_operand)
+      a.scales[rb * a.C + c0 + c] = __fdiv_rn(1.0f, s);
+    else
+      a.scales[(int64_t)(c0 + c) * (a.R / kTile) + rb] = s;
+  }
+}
+
 int grid_for(int64_t units, int per_cta, int sm_count) {
   int64_t blocks = (units + per_cta - 1) / per_cta;
   const int64_t cap = (int64_t)sm_count * 8;
@@ -216,12 +298,30 @@ cudaError_t launch_transpose_blocks(const uint8_t* w, const float* s, int64_t gr
 
 cudaError_t launch_dy_rows_quantize(const void* dy, const float* gates, int T, int H, int K,
                                     const int32_t* token_row, int64_t routed_cap, uint8_t* q,
-                                    float* qs, uint32_t* status, cudaStream_t stream,
-                                    int sm_count) {
+                                    float* qs, float* row_gate, uint32_t* status,
+                                    cudaStream_t stream, int sm_count) {
   const int64_t n_tiles = (int64_t)T * (H / kTile);
   if (n_tiles == 0) return cudaSuccess;
   dy_rows_quantize_kernel<<<grid_for(n_tiles, 16, sm_count), 256, 0, stream>>>(
-      reinterpret_cast<const uint4*>(dy), gates, T, H, K, token_row, routed_cap, q, qs, status);
+      reinterpret_cast<const uint4*>(dy), gates, T, H, K, token_row, routed_cap, q, qs, row_gate,
+      status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_cols(int source, const int32_t* row_token, int64_t routed_cap, int T,
+                                 const float* row_gate, const void* src, const float* gu,
+                                 const float* dh, int64_t R, int C, int I, uint8_t* codes,
+                                 float* scales, bool b_operand, cudaStream_t stream) {
+  if (R == 0 || C == 0) return cudaSuccess;
+  ColArgs a{row_token, routed_cap, T, row_gate, static_cast<const __nv_bfloat16*>(src), gu, dh,
+            R, C, I, codes, scales, b_operand};
+  dim3 grid((unsigned)(R / kTile), (unsigned)((C + 31) / 32));
+  switch (source) {
+    case kColDy: quantize_cols_kernel<kColDy><<<grid, 256, 0, stream>>>(a); break;
+    case kColX: quantize_cols_kernel<kColX><<<grid, 256, 0, stream>>>(a); break;
+    case kColH: quantize_cols_kernel<kColH><<<grid, 256, 0, stream>>>(a); break;
+    default: quantize_cols_kernel<kColDgu><<<grid, 256, 0, stream>>>(a); break;
+  }
   return cudaGetLastError();
 }
 

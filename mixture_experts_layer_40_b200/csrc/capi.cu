@@ -385,7 +385,10 @@ namespace moe {
 namespace {
 
 struct BackwardLayout {
-  size_t dy_q, dy_s, gu, dh, dgu_q, dgu_s, total;
+  size_t dy_q, dy_s, gu, dh, dgu_q, dgu_s;
+  // weight gradients: row gates and the column-tile operands
+  size_t row_gate, dyt_q, dyt_s, ht_q, ht_inv, dgut_q, dgut_s, xt_q, xt_inv;
+  size_t total;
 };
 
 BackwardLayout backward_layout(const moe_shape& sh) {
@@ -405,6 +408,15 @@ BackwardLayout backward_layout(const moe_shape& sh) {
   B.dh = take(R * I * 4);
   B.dgu_q = take(R * 2 * I);
   B.dgu_s = take(R * (2 * I / kTile) * 4);
+  B.row_gate = take(R * 4);
+  B.dyt_q = take(H * R);
+  B.dyt_s = take(H * (R / kTile) * 4);
+  B.ht_q = take(I * R);
+  B.ht_inv = take((R / kTile) * I * 4);
+  B.dgut_q = take(2 * I * R);
+  B.dgut_s = take(2 * I * (R / kTile) * 4);
+  B.xt_q = take(H * R);
+  B.xt_inv = take((R / kTile) * H * 4);
   B.total = off;
   return B;
 }
@@ -422,9 +434,9 @@ size_t moe_backward_workspace_size(moe_shape sh) {
 }
 
 int moe_backward(moe_shape sh, const moe_weights* w, const moe_weights* wt,
-                 const int32_t* topk_ids, const float* topk_gates, const void* dy, void* ws,
-                 size_t ws_bytes, void* bws, size_t bws_bytes, void* dx, float* dgates,
-                 void* stream) {
+                 const int32_t* topk_ids, const float* topk_gates, const void* x, const void* dy,
+                 void* ws, size_t ws_bytes, void* bws, size_t bws_bytes, void* dx, float* dgates,
+                 float* dw13, float* dw2, void* stream) {
   if (!backward_shape_ok(sh)) return MOE_ERR_SHAPE;
   if (!w || !wt || !ws || !bws) return MOE_ERR_NULL;
   moe_ws_layout L;
@@ -450,9 +462,14 @@ int moe_backward(moe_shape sh, const moe_weights* w, const moe_weights* wt,
     e = launch_gate_grad(dy, y_rows, token_row, sh.T, sh.H, sh.K, L.routed_cap, dgates, status, s,
                          sms);
   // dY rows: g dy (routed), dy (shared), 1x128 along H
+  const bool wgrad = dw13 != nullptr && dw2 != nullptr;
+  if (wgrad && (!x || !aligned(dw13, 16) || !aligned(dw2, 16))) return MOE_ERR_NULL;
+  if (e == cudaSuccess && wgrad)
+    e = cudaMemsetAsync(at<float>(bws, B.row_gate), 0, (size_t)L.rows_total * 4, s);
   if (e == cudaSuccess)
     e = launch_dy_rows_quantize(dy, topk_gates, sh.T, sh.H, sh.K, token_row, L.routed_cap,
-                                at<uint8_t>(bws, B.dy_q), at<float>(bws, B.dy_s), status, s, sms);
+                                at<uint8_t>(bws, B.dy_q), at<float>(bws, B.dy_s),
+                                wgrad ? at<float>(bws, B.row_gate) : nullptr, status, s, sms);
   const int32_t* gr = at<int32_t>(ws, L.group_rows);
   const int32_t* gs = at<int32_t>(ws, L.row_start);
   // [G | U] recomputed from the forward's x rows: fp32 [rows, 2I]
@@ -481,6 +498,34 @@ int moe_backward(moe_shape sh, const moe_weights* w, const moe_weights* wt,
   if (e == cudaSuccess)
     e = launch_combine(y_rows, topk_ids, nullptr, token_row, sh.T, sh.H, sh.K, L.routed_cap,
                        L.rows_total, static_cast<__nv_bfloat16*>(dx), status, s);
+  if (!wgrad || e != cudaSuccess) return cuda_status(e);
+  // Wgrad: operands in column tiles (128 rows x 1 channel), transposed
+  const int32_t* row_token = at<int32_t>(ws, L.row_token);
+  const int64_t R = L.rows_total;
+  const float* rg = at<float>(bws, B.row_gate);
+  const float* gu = at<float>(bws, B.gu);
+  const int64_t cap = L.routed_cap;
+  uint8_t* b8 = static_cast<uint8_t*>(bws);
+  e = launch_quantize_cols(0, row_token, cap, sh.T, rg, dy, nullptr, nullptr, R, sh.H, sh.I,
+                           b8 + B.dyt_q, at<float>(bws, B.dyt_s), false, s);
+  if (e == cudaSuccess)
+    e = launch_quantize_cols(2, row_token, cap, sh.T, rg, nullptr, gu, nullptr, R, sh.I, sh.I,
+                             b8 + B.ht_q, at<float>(bws, B.ht_inv), true, s);
+  if (e == cudaSuccess)
+    e = launch_quantize_cols(3, row_token, cap, sh.T, rg, nullptr, gu, at<float>(bws, B.dh), R,
+                             2 * sh.I, sh.I, b8 + B.dgut_q, at<float>(bws, B.dgut_s), false, s);
+  if (e == cudaSuccess)
+    e = launch_quantize_cols(1, row_token, cap, sh.T, rg, x, nullptr, nullptr, R, sh.H, sh.I,
+                             b8 + B.xt_q, at<float>(bws, B.xt_inv), true, s);
+  // dW2_e [H, I] = dY_e^T . h_e;  dW13_e [2I, H] = [dG|dU]_e^T . x_e
+  if (e == cudaSuccess)
+    e = launch_wgrad(gr, gs, sh.N + 1, sh.H, sh.I, R, at<uint8_t>(bws, B.dyt_q),
+                     at<float>(bws, B.dyt_s), at<uint8_t>(bws, B.ht_q), at<float>(bws, B.ht_inv),
+                     dw2, status, s, sms);
+  if (e == cudaSuccess)
+    e = launch_wgrad(gr, gs, sh.N + 1, 2 * sh.I, sh.H, R, at<uint8_t>(bws, B.dgut_q),
+                     at<float>(bws, B.dgut_s), at<uint8_t>(bws, B.xt_q), at<float>(bws, B.xt_inv),
+                     dw13, status, s, sms);
   return cuda_status(e);
 }
 

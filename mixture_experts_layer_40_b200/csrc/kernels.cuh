@@ -57,8 +57,21 @@ cudaError_t launch_transpose_blocks(const uint8_t* w, const float* s, int64_t gr
                                     int64_t cols, uint8_t* wt, float* st, cudaStream_t stream);
 cudaError_t launch_dy_rows_quantize(const void* dy, const float* gates, int T, int H, int K,
                                     const int32_t* token_row, int64_t routed_cap, uint8_t* q,
-                                    float* qs, uint32_t* status, cudaStream_t stream,
-                                    int sm_count);
+                                    float* qs, float* row_gate, uint32_t* status,
+                                    cudaStream_t stream, int sm_count);
+// Column-tile (128 GEMM rows x 1 channel) quantisation of a weight-gradient
+// operand, transposed to [C, R]; source 0: gate * dy rows, 1: x rows, 2: h
+// from [G|U], 3: [dG|dU] from [G|U] and dh.
+cudaError_t launch_quantize_cols(int source, const int32_t* row_token, int64_t routed_cap, int T,
+                                 const float* row_gate, const void* src, const float* gu,
+                                 const float* dh, int64_t R, int C, int I, uint8_t* codes,
+                                 float* scales, bool b_operand, cudaStream_t stream);
+// Per-expert weight gradients C_g [M, N] = A_g . B_g^T over each expert's
+// GEMM rows, operands transposed [M|N, R] (wgrad.cu).
+cudaError_t launch_wgrad(const int32_t* group_rows, const int32_t* group_start, int n_groups,
+                         int M, int N, int64_t gemm_rows, const uint8_t* a_t, const float* a_s,
+                         const uint8_t* b_t, const float* b_inv, float* c, uint32_t* status,
+                         cudaStream_t stream, int sm_count);
 cudaError_t launch_swiglu_backward(const float* gu, const float* dh, int64_t rows, int I,
                                    uint8_t* q, float* qs, cudaStream_t stream, int sm_count);
 cudaError_t launch_gate_grad(const void* dy, const float* y_rows, const int32_t* token_row, int T,

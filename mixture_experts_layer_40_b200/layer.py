@@ -110,10 +110,12 @@ class MoELayer:
         capi.moe_balance_stats(self.shape, seq_len, alpha, self.ws, self.ids, f, p, loss, stream)
         return f, p, loss
 
-    def backward(self, dy: torch.Tensor, stream=None):
+    def backward(self, dy: torch.Tensor, x: torch.Tensor | None = None, stream=None):
         """Input and gate gradients of the last forward for the upstream
-        gradient dy (bf16 [T, H]); the transposed weights and the backward
-        workspace are made on first use. Returns (dx bf16 [T, H], dgates)."""
+        gradient dy (bf16 [T, H]), and with the forward's input x also the
+        expert weight gradients; the transposed weights and the backward
+        workspace are made on first use. Returns (dx bf16 [T, H], dgates
+        [T, K]) or, with x, (dx, dgates, dw13 [E, 2I, H], dw2 [E, H, I])."""
         if getattr(self, "_wt", None) is None:
             E, H, I = self.N + 1, self.H, self.I
             dev = self.device
@@ -131,9 +133,14 @@ class MoELayer:
             self._wt = capi.make_weights(self.weights.gate_w, w13t, s13t, w2t, s2t)
         dx = torch.empty((self.T, self.H), dtype=torch.bfloat16, device=self.device)
         dgates = torch.empty((self.T, self.K), dtype=torch.float32, device=self.device)
-        capi.moe_backward(self.shape, self._cw, self._wt, self.ids, self.gates, dy, self.ws,
-                          self._bws, dx, dgates, stream)
-        return dx, dgates
+        dw13 = dw2 = None
+        if x is not None:
+            E = self.N + 1
+            dw13 = torch.empty((E, 2 * self.I, self.H), dtype=torch.float32, device=self.device)
+            dw2 = torch.empty((E, self.H, self.I), dtype=torch.float32, device=self.device)
+        capi.moe_backward(self.shape, self._cw, self._wt, self.ids, self.gates, x, dy, self.ws,
+                          self._bws, dx, dgates, dw13, dw2, stream)
+        return (dx, dgates) if x is None else (dx, dgates, dw13, dw2)
 
     def update_bias(self, bias: torch.Tensor, gamma: float, stream=None) -> None:
         capi.moe_update_bias(bias, self.counts, self.N, self.T, self.K, gamma, stream)

@@ -132,3 +132,83 @@ def test_backward_v3_shape_sampled():
     case, layer, dy, dx, dgates = _run(w, 4)
     tokens = np.sort(np.random.default_rng(5).choice(w.T, 12, replace=False))
     _check(w, case, layer, dy, dx, dgates, tokens=tokens)
+
+
+# Weight gradients: measured on the oracle itself, 1e-7 relative dy
+# perturbations move an expert's dW by up to 1.5% of its RMS (the per-row and
+# per-element spread is larger: rows of a rarely chosen expert sum few
+# tokens). Bound: 4% per expert matrix, 3% over all of them; the Wgrad GEMM
+# itself is checked to 1e-5 on identical quantised operands, and the x
+# operand's column tiles bit-exactly.
+DW_EXPERT, DW_TOTAL = 4e-2, 3e-2
+
+
+def _bws_wgrad_views(layer, w):
+    """The weight-gradient part of the backward workspace (after _bws_views)."""
+    R = layer.layout.rows_total
+    sizes = [R * w.H, R * (w.H // 128) * 4, R * 2 * w.I * 4, R * w.I * 4, R * 2 * w.I,
+             R * (2 * w.I // 128) * 4]
+    off = 0
+    for n in sizes:
+        off = (off + n + 255) // 256 * 256
+    out = []
+    for n, dtype, shape in [(R * 4, torch.float32, (R,)),
+                            (w.H * R, torch.uint8, (w.H, R)),
+                            (w.H * (R // 128) * 4, torch.float32, (w.H, R // 128)),
+                            (w.I * R, torch.uint8, (w.I, R)),
+                            ((R // 128) * w.I * 4, torch.float32, (R // 128, w.I)),
+                            (2 * w.I * R, torch.uint8, (2 * w.I, R)),
+                            (2 * w.I * (R // 128) * 4, torch.float32, (2 * w.I, R // 128)),
+                            (w.H * R, torch.uint8, (w.H, R)),
+                            ((R // 128) * w.H * 4, torch.float32, (R // 128, w.H))]:
+        out.append(layer._bws[off:off + n].view(dtype).view(*shape))
+        off = (off + n + 255) // 256 * 256
+    return out
+
+
+def test_weight_gradients():
+    w = I.Workload("bwg", T=300, H=512, N=32, K=4, I=256, bias_range=0.1, seed=352)
+    case = H.make_case(w)
+    layer = MoELayer(w.T, w.H, w.N, w.K, w.I, device_weights(w, case.pool, case.gate_w, "cuda"))
+    xd = H.x_to_device(case.x_bits)
+    layer.forward(xd, torch.from_numpy(case.bias).cuda())
+    dy_bits = _dy(w, 3)
+    dx, dgates, dw13, dw2 = layer.backward(H.x_to_device(dy_bits), x=xd)
+    assert layer.status() == 0
+    dy = I.bf16_bits_to_f32(dy_bits)
+    gid = layer.ids.cpu().numpy()
+    r_ids, _, _, score = O.route(case.x, case.gate_w, case.bias, w.K)
+    use, _, _ = H.reconcile_ids(gid, r_ids, score, w.K)
+    ref = O.moe_backward(case.x, case.gate_w, case.bias, w.K, case.ew, dy, mode="Q", ids=use)
+    g13 = dw13.cpu().numpy().reshape(w.N + 1, w.I // 128, 2, 128, w.H)
+    g2 = dw2.cpu().numpy()
+    num = den = 0.0
+    for e, (dwg, dwu, dwd) in ref["dw"].items():
+        got_g = g13[e, :, 0].reshape(w.I, w.H)
+        got_u = g13[e, :, 1].reshape(w.I, w.H)
+        for got, want in [(got_g, dwg), (got_u, dwu), (g2[e], dwd)]:
+            err = np.sum((got - want) ** 2)
+            assert np.sqrt(err / np.sum(want ** 2)) < DW_EXPERT, e
+            num += err
+            den += np.sum(want ** 2)
+    assert np.sqrt(num / den) < DW_TOTAL
+    # experts nobody chose get zero gradients
+    unused = sorted(set(range(w.N)) - set(np.unique(gid).tolist()))
+    for e in unused:
+        assert not np.any(g13[e]) and not np.any(g2[e])
+    # the shared expert's x operand in column tiles: exact (x is bf16)
+    L = layer.layout
+    rg, dyt_q, dyt_s, ht_q, ht_inv, dgut_q, dgut_s, xt_q, xt_inv = _bws_wgrad_views(layer, w)
+    sh_rows = slice(L.routed_cap, L.routed_cap + (w.T + 127) // 128 * 128)
+    xq, xs = O.quantize_128x1(case.x)
+    assert np.array_equal(xt_q[:, sh_rows].cpu().numpy(), xq)
+    kb = slice(L.routed_cap // 128, L.routed_cap // 128 + xs.shape[1])
+    assert np.array_equal(xt_inv[kb].cpu().numpy().T, (np.float32(1.0) / xs).astype(np.float32))
+    # the Wgrad GEMM on its own operands (shared expert): fp32 accumulation only
+    a = O.dequantize_1x128(dyt_q[:, sh_rows].cpu().numpy(),
+                           dyt_s[:, kb].cpu().numpy())             # [H, R_e]
+    b = O.e4m3_decode(ht_q[:, sh_rows].cpu().numpy()) * np.repeat(
+        ht_inv[kb].cpu().numpy().T.astype(np.float64), 128, axis=1)  # [I, R_e]
+    c_ref = a @ b.T
+    got = g2[w.N].astype(np.float64)
+    assert np.all(np.abs(got - c_ref) <= 1e-5 * np.sqrt(np.mean(c_ref ** 2)) + 1e-30)
