@@ -51,6 +51,8 @@ def parse():
     p.add_argument("--groups", type=int, default=0,
                    help="node-limited routing: G expert groups (0: top-K over all N)")
     p.add_argument("--topk-groups", type=int, default=0, help="node-limited routing: M groups")
+    p.add_argument("--backward", action="store_true",
+                   help="also time the FP8 expert backward (Dgrad + Wgrad) after the forward")
     p.add_argument("--seq-len", type=int, default=0,
                    help="sequence length for the balance statistics (0: the whole batch)")
     return p.parse_args()
@@ -475,6 +477,37 @@ def run_ours(args, w, rank, world, local_rank):
     clk = clocks.stop() if clocks else None
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev) / args.steps
     bal_ms = bal_ev[0].elapsed_time(bal_ev[1]) / 20
+    # ------------------------------------------------ backward (not part of the step)
+    bwd = None
+    if args.backward and world == 1:
+        gdy = torch.randn((w.T, w.H), device=dev).mul_(0.05).to(torch.bfloat16)
+        step()
+        layer.backward(gdy)             # set-up: transposed weights, workspace
+        layer.backward(gdy, x=x)
+        out = {}
+        for name, kw in [("dgrad", {}), ("dgrad_wgrad", {"x": x})]:
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            ms = 0.0
+            for _ in range(reps):
+                step()                  # the backward needs its own forward's state
+                b0.record(stream)
+                layer.backward(gdy, **kw)
+                b1.record(stream)
+                b1.synchronize()
+                ms += b0.elapsed_time(b1)
+            out[name] = ms / reps
+        if layer.status() != 0:
+            raise RuntimeError("device status error in the backward")
+        rows = w.T * (w.K + 1)
+        flops_d = 2.0 * rows * w.H * w.I * 2 + 2.0 * rows * w.H * w.I + 2.0 * rows * w.H * 2 * w.I
+        flops_w = 2.0 * rows * w.H * w.I + 2.0 * rows * 2 * w.I * w.H
+        bwd = {"dgrad_ms": out["dgrad"], "dgrad_wgrad_ms": out["dgrad_wgrad"],
+               "dgrad_tflops": flops_d / (out["dgrad"] * 1e-3) / 1e12,
+               "wgrad_ms": out["dgrad_wgrad"] - out["dgrad"],
+               "wgrad_out_gb": (w.N + 1) * 3 * w.H * w.I * 4 / 1e9,
+               "note": "moe_backward after a forward; Dgrad = recompute [G|U], dh, dX rows (3 FP8 "
+                       "grouped GEMMs); Wgrad adds dW2 and dW13 in fp32 for all N+1 experts"}
 
     if rank != 0:
         return
@@ -515,6 +548,7 @@ def run_ours(args, w, rank, world, local_rank):
                           "double-buffered, overlapping the neighbouring steps' kernels"},
         "clocks": clk,
         "controller": trace,
+        "backward": bwd,
         "balance_stats": {"ms": bal_ms, "seq_len": seq_len,
                           "note": "moe_balance_stats after the step, not part of it"},
     }
