@@ -206,40 +206,54 @@ def measure_fp8_peak(torch, device):
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_sample_step(w, x, gate_w, bias, ew, step: int, groups: int = 2, shared_rows: int = 64,
-                       node_limit: tuple = (0, 0)):
-    """One bounded sample of the layer on the CPU oracle; returns the time
-    scaled to the whole layer (all T tokens, all N + 1 expert groups)."""
+def oracle_sample_step(w, x, gate_w, bias, ew, step: int, sample_tokens: int = 512,
+                       groups: int = 1, shared_rows: int = 64, node_limit: tuple = (0, 0)):
+    """One bounded sample of the layer on the CPU oracle; returns its time
+    scaled to the whole layer. The sample (a window of `sample_tokens`
+    tokens moving with the step): their quantisation, routing, permutation
+    and combine (scaled by T / sample); `groups` routed experts, each with
+    the sampled tokens that chose it (assembly of the expert's weights timed
+    once per expert, its FFN scaled by T / sample, then both by N / groups);
+    the shared expert on `shared_rows` of the sampled tokens (its FFN scaled
+    to all T tokens)."""
     from oracle import moe_oracle as O
+    n = min(w.T, sample_tokens)
+    t0s = (step * n) % max(1, w.T - n + 1)
+    xs_ = x[t0s:t0s + n]
+    scale = w.T / n
     t0 = time.perf_counter()
-    xq, xs = O.quantize_1x128(x)
-    t_quant = time.perf_counter() - t0
-    t0 = time.perf_counter()
+    xq, xsc = O.quantize_1x128(xs_)
     if node_limit[0] > 1 and node_limit[1] < node_limit[0]:
-        ids, gates, *_ = O.route_grouped(x, gate_w, bias, w.K, node_limit[0], node_limit[1])
+        ids, gates, *_ = O.route_grouped(xs_, gate_w, bias, w.K, node_limit[0], node_limit[1])
     else:
-        ids, gates, _, _ = O.route(x, gate_w, bias, w.K)
+        ids, gates, _, _ = O.route(xs_, gate_w, bias, w.K)
     O.permutation(ids, w.N)
-    t_route = time.perf_counter() - t0
-    y_routed = np.zeros((w.T, w.K, w.H))
-    t0 = time.perf_counter()
+    t_tokens = time.perf_counter() - t0
+    y_routed = np.zeros((n, w.K, w.H))
+    t_assemble = t_ffn = 0.0
     for j in range(groups):
         e = (step * groups + j) % w.N
+        t0 = time.perf_counter()
+        wts = ew.dequantised(e)
+        t_assemble += time.perf_counter() - t0
         rr, kk = np.nonzero(ids == e)
+        t0 = time.perf_counter()
         if len(rr):
-            y_routed[rr, kk] = O.expert_ffn_q(xq[rr], xs[rr], *ew.dequantised(e))[0]
-    t_groups = time.perf_counter() - t0
+            y_routed[rr, kk] = O.expert_ffn_q(xq[rr], xsc[rr], *wts)[0]
+        t_ffn += time.perf_counter() - t0
+    m = min(shared_rows, n)
     t0 = time.perf_counter()
-    r0 = (step * shared_rows) % max(1, w.T - shared_rows + 1)
-    rows = slice(r0, r0 + shared_rows)
-    y_shared = np.zeros((w.T, w.H))
-    y_shared[rows] = O.expert_ffn_q(xq[rows], xs[rows], *ew.dequantised(w.N))[0]
+    wts = ew.dequantised(w.N)
+    t_shared_assemble = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    y_shared = np.zeros((n, w.H))
+    y_shared[:m] = O.expert_ffn_q(xq[:m], xsc[:m], *wts)[0]
     t_shared = time.perf_counter() - t0
     t0 = time.perf_counter()
     O.combine(y_shared, y_routed, ids, gates)
     t_combine = time.perf_counter() - t0
-    return (t_quant + t_route + t_combine + t_groups * w.N / groups
-            + t_shared * w.T / min(shared_rows, w.T))
+    return ((t_tokens + t_combine) * scale + (t_assemble + t_ffn * scale) * w.N / groups
+            + t_shared_assemble + t_shared * w.T / m)
 
 
 def blas_threads():
@@ -314,9 +328,9 @@ def run_reference(args, w, rank):
              for s in range(args.steps)]
     ms = 1e3 * float(np.mean(times))
     value = w.T / (ms * 1e-3)
-    sample = (f"per step: the whole layer's routing, quantisation and combine on all {w.T} tokens, "
-              f"2 of {w.N} routed expert groups with all their tokens and the shared expert on 64 "
-              f"tokens; group and shared time scaled to all groups and tokens")
+    sample = (f"per step: quantisation, routing, permutation and combine of 512 of the {w.T} "
+              f"tokens, 1 of {w.N} routed experts on its sampled tokens and the shared expert on 64; "
+              f"scaled to all tokens and experts")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -559,9 +573,9 @@ def run_ours(args, w, rank, world, local_rank):
         v = w.T / float(np.mean(t))
         line["cpu_baseline"] = {
             "value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"2 steps; each: quantisation, routing and combine of all {w.T} tokens, 2 of "
-                      f"{w.N} routed expert groups with all their tokens and the shared expert on "
-                      f"64 tokens, group and shared time scaled to the whole layer"}
+            "sample": f"2 steps; each: quantisation, routing, permutation and combine of 512 of "
+                      f"the {w.T} tokens, 1 of {w.N} routed experts on its sampled tokens and the "
+                      f"shared expert on 64, scaled to all tokens and experts"}
     print(json.dumps(line), flush=True)
 
 
