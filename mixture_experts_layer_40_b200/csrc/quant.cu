@@ -83,50 +83,60 @@ __global__ void __launch_bounds__(256) quantize_scatter_kernel(
     const uint4* __restrict__ x, int T, int H, int K, const int32_t* __restrict__ token_row,
     int64_t routed_cap, uint8_t* __restrict__ a_q, float* __restrict__ a_s,
     uint32_t* __restrict__ status) {
-  constexpr int kPerThread = 2;  // tiles in flight per thread (both loads issued first)
-  const int sub = threadIdx.x & 15;
+  // 8 threads per tile, 16 consecutive elements each (two 128-bit loads, one
+  // 128-bit store of codes per destination row); two tiles in flight
+  constexpr int kPerThread = 2;
+  const int sub = threadIdx.x & 7;
   const int tiles_per_row = H / kTile;
   const int64_t n_tiles = (int64_t)T * tiles_per_row;
-  const int64_t step = (int64_t)gridDim.x * 16;
-  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_tiles; base += step * kPerThread) {
-    uint4 v[kPerThread];
-    int my_row[kPerThread];
+  const int64_t step = (int64_t)gridDim.x * 32;
+  for (int64_t base = (int64_t)blockIdx.x * 32; base < n_tiles; base += step * kPerThread) {
+    uint4 v0[kPerThread], v1[kPerThread];
+    int row_a[kPerThread], row_b[kPerThread];   // destinations k = sub and k = sub + 8
     int64_t tile[kPerThread];
 #pragma unroll
     for (int u = 0; u < kPerThread; ++u) {
-      tile[u] = base + u * step + (threadIdx.x >> 4);
+      tile[u] = base + u * step + (threadIdx.x >> 3);
       const bool live = tile[u] < n_tiles;
       const int64_t t = live ? tile[u] / tiles_per_row : 0;
-      v[u] = live ? __ldcs(x + tile[u] * 16 + sub) : make_uint4(0, 0, 0, 0);
-      my_row[u] = (live && sub < K) ? __ldg(token_row + t * K + sub) : -1;
+      v0[u] = live ? __ldcs(x + tile[u] * 16 + 2 * sub) : make_uint4(0, 0, 0, 0);
+      v1[u] = live ? __ldcs(x + tile[u] * 16 + 2 * sub + 1) : make_uint4(0, 0, 0, 0);
+      row_a[u] = (live && sub < K) ? __ldg(token_row + t * K + sub) : -1;
+      row_b[u] = (live && sub + 8 < K) ? __ldg(token_row + t * K + sub + 8) : -1;
     }
 #pragma unroll
     for (int u = 0; u < kPerThread; ++u) {
       const bool live = tile[u] < n_tiles;
       const int64_t t = live ? tile[u] / tiles_per_row : 0;
       const int c = live ? (int)(tile[u] - t * tiles_per_row) : 0;
-      float f[8] = {bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y),
-                    bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w)};
+      float f[16] = {bf16_lo(v0[u].x), bf16_hi(v0[u].x), bf16_lo(v0[u].y), bf16_hi(v0[u].y),
+                     bf16_lo(v0[u].z), bf16_hi(v0[u].z), bf16_lo(v0[u].w), bf16_hi(v0[u].w),
+                     bf16_lo(v1[u].x), bf16_hi(v1[u].x), bf16_lo(v1[u].y), bf16_hi(v1[u].y),
+                     bf16_lo(v1[u].z), bf16_hi(v1[u].z), bf16_lo(v1[u].w), bf16_hi(v1[u].w)};
       float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       const float s = tile_scale(amax);
-      uint2 out;
+      uint4 out;
       out.x = e4m3x4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
       out.y = e4m3x4(__fmul_rn(f[4], s), __fmul_rn(f[5], s), __fmul_rn(f[6], s), __fmul_rn(f[7], s));
+      out.z = e4m3x4(__fmul_rn(f[8], s), __fmul_rn(f[9], s), __fmul_rn(f[10], s), __fmul_rn(f[11], s));
+      out.w = e4m3x4(__fmul_rn(f[12], s), __fmul_rn(f[13], s), __fmul_rn(f[14], s), __fmul_rn(f[15], s));
       for (int k = -1; k < K; ++k) {
         int64_t r = routed_cap + t;
         if (k >= 0) {
-          r = __shfl_sync(0xffffffffu, my_row[u], k, 16);
+          const int ra = __shfl_sync(0xffffffffu, row_a[u], k & 7, 8);
+          const int rb = __shfl_sync(0xffffffffu, row_b[u], k & 7, 8);
+          r = k < 8 ? ra : rb;
           if (live && (r < 0 || r >= routed_cap)) {
             if (sub == 0) flag_status(status, kStatusBounds);
             continue;
           }
         }
         if (live) {
-          reinterpret_cast<uint2*>(a_q + r * H + (int64_t)c * kTile)[sub] = out;
+          reinterpret_cast<uint4*>(a_q + r * H + (int64_t)c * kTile)[sub] = out;
           if (sub == 0) a_s[r * tiles_per_row + c] = s;
         }
       }
@@ -139,7 +149,7 @@ cudaError_t launch_quantize_scatter(const void* x, int T, int H, int K, const in
                                     uint32_t* status, cudaStream_t stream, int sm_count) {
   const int64_t n_tiles = (int64_t)T * (H / kTile);
   if (n_tiles == 0) return cudaSuccess;
-  int64_t blocks = (n_tiles + 15) / 16;
+  int64_t blocks = (n_tiles + 31) / 32;
   const int64_t cap = (int64_t)sm_count * 8;
   if (blocks > cap) blocks = cap;
   quantize_scatter_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
