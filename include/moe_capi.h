@@ -1,5 +1,7 @@
 /*
- * moe_capi.h — C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ * moe_capi.h — C ABI of the B200 (sm_100a) DeepSeekMoE layer: the forward,
+ * the bias controller, node-limited routing, the sequence-wise balance
+ * statistics and the FP8 backward of the expert path.
  *
  * The layer (sources: "DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing,
  * Multi-Token Prediction, and FP8 Training at 671B Scale", trishampatil.com,
@@ -15,6 +17,11 @@
  *   FFN(u)  = W_down (silu(W_gate u) * (W_up u))          SwiGLU, FP8 E4M3:
  *             u and h in 1x128 tiles, weights in 128x128 blocks, fp32 sums
  *   b_i    <- b_i + gamma * sign(T*K/N - c_i)             per step, c_i = load
+ *
+ * and, for training, the gradients of y with respect to x (through the
+ * experts), the gates and the expert weights, with the Dgrad and Wgrad GEMMs
+ * in FP8 as well ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing, ...",
+ * section V, Figure 6).
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers, row-major, owned by the caller;
