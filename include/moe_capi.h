@@ -359,6 +359,88 @@ int moe_expert_down(int32_t H, int32_t I, int32_t n_groups, const int32_t* group
                     uint32_t* status_ws, void* stream);
 
 /*
+ * Expert parallelism ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing,
+ * Multi-Token Prediction, and FP8 Training at 671B Scale", section V,
+ * "Training at Scale" and "Custom all-to-all kernels"; "DeepSeek-V3,
+ * explained", recipe step 8). The layer runs on W ranks (1 <= W <= 16, one GPU
+ * each, N % W == 0, N/W a multiple of 16 and >= 16). Rank d holds routed
+ * experts [d N/W, (d+1) N/W) plus the shared expert, as a moe_weights with
+ * El + 1 = N/W + 1 weight sets (its El experts in order, then the shared
+ * expert), and the whole gate gate_w [N, H]. Every rank routes its own T
+ * tokens. A token travels once to each rank that holds one of its experts,
+ * as one packed FP8 row:
+ *   [codes: H bytes][scales: H/128 float][local ids: K int32][gates: K float]
+ * padded to moe_ep_row_bytes(sh) (a multiple of 16). Local id k is the
+ * expert's index on the destination (-1: slot k's expert is elsewhere; its
+ * gate is then 0). A step, on every rank:
+ *   1. moe_ep_dispatch: route, then fill `send` with this rank's rows,
+ *      destination-major (rank 0's rows first), tokens ascending within each
+ *      destination; send_counts[2d] = rows for rank d, send_counts[2d+1] =
+ *      (token, slot) pairs for rank d.
+ *   2. the caller exchanges send_counts (an all-to-all of 2 int32 per pair of
+ *      ranks) and then the rows (an all-to-all with those row counts); the
+ *      received rows are source-major. moe_ep_shared may run meanwhile.
+ *   3. moe_ep_experts on the received rows: out[j] = sum over row j's local
+ *      slots, by ascending expert id, of gate * expert(x_j), fp32 [R, H].
+ *   4. the caller sends each `out` row back to its source (the reverse
+ *      all-to-all), which then holds them in its send order.
+ *   5. moe_ep_combine: y_t = shared_t + sum over the token's destination
+ *      ranks, ascending, of the returned rows (fp32), rounded once to bf16.
+ * The quantisation, GEMMs and gates are the single-GPU layer's, so each
+ * expert output matches moe_forward's; only the order of the fp32 additions
+ * in the combine differs. Device checks go to the status word at the start
+ * of the workspace used (moe_get_status).
+ */
+
+/* Bytes of one packed dispatch row (0 for an invalid shape). */
+int64_t moe_ep_row_bytes(moe_shape sh);
+
+/* Workspace of moe_ep_dispatch / moe_ep_shared / moe_ep_combine (0 if the
+ * shape or W is not supported). */
+size_t moe_ep_dispatch_workspace_size(moe_shape sh, int32_t W);
+
+/*
+ * Step 1. gate_w: float [N, H]; x: bf16 [T, H]; bias: float [N]. Optional
+ * outputs as in moe_forward (topk_ids and topk_gates [T, K] with global expert
+ * ids; counts [N] of this rank's tokens, for moe_update_bias after a sum over
+ * ranks). send: uint8 [send_cap, moe_ep_row_bytes], 16-byte aligned
+ * (T * min(W, K) rows always suffice; a row beyond send_cap is dropped and
+ * flagged). send_counts: int32 [W, 2] device. ws: the source workspace,
+ * 256-byte aligned; it keeps the send slots and the shared-expert rows for
+ * steps 1b and 5. T = 0 clears send_counts and counts only.
+ */
+int moe_ep_dispatch(moe_shape sh, int32_t W, const float* gate_w, const void* x, const float* bias,
+                    int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
+                    uint8_t* send, int64_t send_cap, int32_t* send_counts, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* Step 1b: the shared expert on this rank's tokens (after moe_ep_dispatch on
+ * the same ws), fp32 rows kept in ws for moe_ep_combine. w_local: this rank's
+ * weights (El + 1 sets); gate_w is not read. */
+int moe_ep_shared(moe_shape sh, int32_t W, const moe_weights* w_local, void* ws, size_t ws_bytes,
+                  void* stream);
+
+/* Workspace of moe_ep_experts for R received rows holding `pairs` slots with
+ * a local expert (0 if unsupported, or pairs > R K). */
+size_t moe_ep_expert_workspace_size(moe_shape sh, int32_t W, int64_t R, int64_t pairs);
+
+/*
+ * Step 3. recv: R packed rows, 16-byte aligned; pairs: the sum of the
+ * received send_counts[2d+1] (checked on the device against the rows). out:
+ * float [R, H], 16-byte aligned. w_local: this rank's weights; gate_w is not
+ * read. ws: moe_ep_expert_workspace_size(sh, W, R, pairs) bytes, 256-byte
+ * aligned. R = 0 does nothing.
+ */
+int moe_ep_experts(moe_shape sh, int32_t W, const moe_weights* w_local, const uint8_t* recv,
+                   int64_t R, int64_t pairs, float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Step 5. ret: float [ret_rows, H], the returned rows in this rank's send
+ * order (ret_rows = its total send rows); ws: the workspace of its
+ * moe_ep_dispatch and moe_ep_shared; y: bf16 [T, H], 16-byte aligned. */
+int moe_ep_combine(moe_shape sh, int32_t W, const float* ret, int64_t ret_rows, void* ws,
+                   size_t ws_bytes, void* y, void* stream);
+
+/*
  * Synchronises `stream`, reads and clears the device status word at the
  * start of `ws` (a forward workspace or a bare uint32 status word). Returns
  * MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_BOUNDS (timeout reported first), or

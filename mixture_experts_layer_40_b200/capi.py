@@ -74,6 +74,15 @@ SIGNATURES = {
     "moe_update_bias": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _F32, _P]),
     "moe_expert_up": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_down": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_ep_row_bytes": (_I64, [moe_shape]),
+    "moe_ep_dispatch_workspace_size": (_SZ, [moe_shape, _I32]),
+    "moe_ep_dispatch": (ctypes.c_int, [moe_shape, _I32, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P,
+                                       _SZ, _P]),
+    "moe_ep_shared": (ctypes.c_int, [moe_shape, _I32, ctypes.POINTER(moe_weights), _P, _SZ, _P]),
+    "moe_ep_expert_workspace_size": (_SZ, [moe_shape, _I32, _I64, _I64]),
+    "moe_ep_experts": (ctypes.c_int, [moe_shape, _I32, ctypes.POINTER(moe_weights), _P, _I64,
+                                      _I64, _P, _P, _SZ, _P]),
+    "moe_ep_combine": (ctypes.c_int, [moe_shape, _I32, _P, _I64, _P, _SZ, _P, _P]),
     "moe_get_status": (ctypes.c_int, [_P, _P]),
     "moe_device_sm_count": (ctypes.c_int, []),
 }
@@ -251,6 +260,50 @@ def moe_expert_down(H, I, n_groups, group_rows, group_start, rows, h_q, h_s, w2,
         H, I, n_groups, _ptr(group_rows, torch.int32), _ptr(group_start, torch.int32), rows,
         _ptr(h_q, torch.uint8), _ptr(h_s, torch.float32), _ptr(w2, torch.uint8),
         _ptr(s2, torch.float32), _ptr(y_rows, torch.float32), _ptr(status), _stream(stream)))
+
+
+def moe_ep_row_bytes(sh: moe_shape) -> int:
+    return int(LIB.moe_ep_row_bytes(sh))
+
+
+def moe_ep_dispatch_workspace_size(sh: moe_shape, W: int) -> int:
+    return int(LIB.moe_ep_dispatch_workspace_size(sh, W))
+
+
+def moe_ep_expert_workspace_size(sh: moe_shape, W: int, R: int, pairs: int) -> int:
+    return int(LIB.moe_ep_expert_workspace_size(sh, W, R, pairs))
+
+
+def moe_ep_dispatch(sh: moe_shape, W: int, gate_w, x, bias, send, send_counts, ws,
+                    topk_ids=None, topk_gates=None, counts=None, stream=None):
+    """send: uint8 [send_cap, moe_ep_row_bytes(sh)]; send_counts: int32 [W, 2]."""
+    _check("moe_ep_dispatch", LIB.moe_ep_dispatch(
+        sh, W, _ptr(gate_w, torch.float32, "gate_w"), _ptr(x, torch.bfloat16, "x"),
+        _ptr(bias, torch.float32, "bias"), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
+        _ptr(send, torch.uint8, "send"), send.shape[0] if send is not None else 0,
+        _ptr(send_counts, torch.int32, "send_counts"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)))
+
+
+def moe_ep_shared(sh: moe_shape, W: int, w_local: moe_weights, ws, stream=None):
+    _check("moe_ep_shared", LIB.moe_ep_shared(
+        sh, W, ctypes.byref(w_local), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_ep_experts(sh: moe_shape, W: int, w_local: moe_weights, recv, R: int, pairs: int, out, ws,
+                   stream=None):
+    """recv: uint8 [>= R, row_bytes]; out: float32 [>= R, H]."""
+    _check("moe_ep_experts", LIB.moe_ep_experts(
+        sh, W, ctypes.byref(w_local), _ptr(recv, torch.uint8, "recv"), R, pairs,
+        _ptr(out, torch.float32, "out"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)))
+
+
+def moe_ep_combine(sh: moe_shape, W: int, ret, ret_rows: int, ws, y, stream=None):
+    _check("moe_ep_combine", LIB.moe_ep_combine(
+        sh, W, _ptr(ret, torch.float32, "ret"), ret_rows, _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _ptr(y, torch.bfloat16, "y"), _stream(stream)))
 
 
 def moe_get_status(ws, stream=None) -> int:

@@ -276,7 +276,8 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   e = mark(1, e);
   // a6-a7: offsets, stable expert-major scatter of the (token, slot) pairs
   if (e == cudaSuccess)
-    e = launch_permute(ids, counts, sh.T, sh.N, sh.K, L.routed_cap, at<int32_t>(ws, L.offsets),
+    e = launch_permute(ids, counts, sh.T, sh.N, sh.K, (int64_t)sh.T * sh.K, L.routed_cap,
+                       at<int32_t>(ws, L.offsets),
                        at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
                        at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.token_row), status, s);
   e = mark(2, e);

@@ -1,0 +1,591 @@
+// Expert parallelism: the layer split over W ranks (one GPU each), routed
+// experts sharded contiguously (rank d holds experts [d N/W, (d+1) N/W)), the
+// shared expert and the gate replicated. "DeepSeek-V3: Auxiliary-Loss-Free MoE
+// Load Balancing, ..." section V ("Training at Scale", "Custom all-to-all
+// kernels"): a token is sent once to each rank that holds one of its experts
+// and reaches all of its experts there; dispatch, expert MLP and combine are
+// separate steps so the exchange can overlap other work. "DeepSeek-V3,
+// explained", recipe step 8: 64-way expert parallelism.
+//
+// Per step, on every rank (the exchanges between the steps belong to the
+// caller: two all-to-alls with row counts known from send_counts):
+//   dispatch (source) : route its own tokens, plan the send rows (rank-major,
+//                       token ascending, one row per (token, rank) that holds
+//                       one of its experts), quantise x 1x128 once into the
+//                       send rows and into its shared-expert GEMM rows
+//   shared   (source) : the shared expert on its own tokens, fp32 rows
+//   experts  (dest)   : received rows -> expert-major GEMM rows of its local
+//                       experts -> grouped FP8 up/down GEMMs -> per received
+//                       row, the gate-weighted sum over its local experts
+//                       (fp32, ascending expert id)
+//   combine  (source) : y_t = shared_t + sum over ranks (ascending) of the
+//                       returned partial sums, rounded once to bf16
+// Every slot and row is fixed by the data, so results do not depend on timing.
+#include "block_scan.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kMaxRanks = 16;
+constexpr int kMaxK = 16;
+
+inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+bool ep_ok(const moe_shape& sh, int W) {
+  if (!shape_ok(sh) || W < 1 || W > kMaxRanks || sh.N % W != 0) return false;
+  const int El = sh.N / W;
+  return El >= 16 && El % 16 == 0;
+}
+
+// Bytes of one packed dispatch row: codes [H] u8, scales [H/128] f32, local
+// expert ids [K] i32 (-1: not on this rank), gates [K] f32; 16-byte multiple.
+int64_t row_bytes_of(const moe_shape& sh) {
+  return round_up((int64_t)sh.H + 4 * (sh.H / kTile) + 8 * (int64_t)sh.K, 16);
+}
+__host__ __device__ inline int64_t meta_offset(int H) { return (int64_t)H + 4 * (int64_t)(H / kTile); }
+
+struct SourceLayout {
+  int64_t rows;  // shared-expert GEMM rows (T rounded up to 128)
+  size_t status, counts, topk_ids, topk_gates, logits, gate_split, send_slot, grp;
+  size_t a_q, a_s, h_q, h_s, y_shared, total;
+};
+
+SourceLayout source_layout(const moe_shape& sh, int W) {
+  const int64_t T = sh.T, H = sh.H, N = sh.N, K = sh.K, I = sh.I;
+  SourceLayout L{};
+  L.rows = round_up(T, kTile);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t a = off;
+    off = (size_t)round_up((int64_t)(off + bytes), 256);
+    return a;
+  };
+  L.status = take(16);
+  L.counts = take(N * 4);
+  L.topk_ids = take((size_t)(T * K) * 4);
+  L.topk_gates = take((size_t)(T * K) * 4);
+  L.logits = take((size_t)(T * N) * 4);
+  L.gate_split = take(router_split_bytes((int)N, (int)H));
+  L.send_slot = take((size_t)(T * W) * 4);
+  L.grp = take(2 * 4);
+  L.a_q = take((size_t)(L.rows * H));
+  L.a_s = take((size_t)(L.rows * (H / kTile)) * 4);
+  L.h_q = take((size_t)(L.rows * I));
+  L.h_s = take((size_t)(L.rows * (I / kTile)) * 4);
+  L.y_shared = take((size_t)(L.rows * H) * 4);
+  L.total = off;
+  return L;
+}
+
+struct ExpertLayout {
+  int64_t routed_cap;
+  size_t status, counts, offsets, group_rows, row_start, ids, gates, token_row, row_token;
+  size_t a_q, a_s, h_q, h_s, y_rows, total;
+};
+
+ExpertLayout expert_layout(const moe_shape& sh, int W, int64_t R, int64_t pairs) {
+  const int64_t El = sh.N / W, H = sh.H, K = sh.K, I = sh.I;
+  ExpertLayout L{};
+  L.routed_cap = round_up(pairs + El * (kTile - 1), kTile);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t a = off;
+    off = (size_t)round_up((int64_t)(off + bytes), 256);
+    return a;
+  };
+  L.status = take(16);
+  L.counts = take(El * 4);
+  L.offsets = take((El + 1) * 4);
+  L.group_rows = take((El + 1) * 4);
+  L.row_start = take((El + 1) * 4);
+  L.ids = take((size_t)(R * K) * 4);
+  L.gates = take((size_t)(R * K) * 4);
+  L.token_row = take((size_t)(R * K) * 4);
+  L.row_token = take((size_t)L.routed_cap * 4);
+  L.a_q = take((size_t)L.routed_cap * H);
+  L.a_s = take((size_t)L.routed_cap * (H / kTile) * 4);
+  L.h_q = take((size_t)L.routed_cap * I);
+  L.h_s = take((size_t)L.routed_cap * (I / kTile) * 4);
+  L.y_rows = take((size_t)L.routed_cap * H * 4);
+  L.total = off;
+  return L;
+}
+
+// Sum of one int per thread over the block; red: shared int[32].
+MOE_DEV int block_sum(int v, int* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int r = 0;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) r += red[i];
+  __syncthreads();
+  return r;
+}
+
+// Dispatch plan: one CTA (1024 threads) per destination rank d. Pass 1 counts
+// the tokens bound for d, those bound for lower ranks (which precede d's rows
+// in the send buffer) and the (token, slot) pairs for d; pass 2 numbers d's
+// tokens in token order and writes each row's local ids and gates.
+__global__ void __launch_bounds__(1024) ep_plan_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ gates, int T, int K, int N, int W,
+    int H, uint8_t* __restrict__ send, int64_t row_bytes, int64_t send_cap,
+    int32_t* __restrict__ send_slot, int32_t* __restrict__ send_counts, int32_t* __restrict__ grp,
+    uint32_t* __restrict__ status) {
+  __shared__ int sums[33];
+  __shared__ int red[32];
+  const int d = blockIdx.x;
+  const int El = N / W;
+  int rows_d = 0, before = 0, pairs_d = 0;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    uint32_t mask = 0;
+    for (int k = 0; k < K; ++k) {
+      const int e = __ldg(ids + (int64_t)t * K + k);
+      if (e < 0 || e >= N) continue;  // flagged below
+      const int r = e / El;
+      mask |= 1u << r;
+      pairs_d += (r == d);
+    }
+    rows_d += (int)((mask >> d) & 1u);
+    before += __popc(mask & ((1u << d) - 1u));
+  }
+  rows_d = block_sum(rows_d, red);
+  before = block_sum(before, red);
+  pairs_d = block_sum(pairs_d, red);
+  const int64_t meta_off = meta_offset(H);
+  int running = 0;
+  for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+    const int t = t0 + threadIdx.x;
+    bool sel = false;
+    if (t < T) {
+      for (int k = 0; k < K; ++k) {
+        const int e = __ldg(ids + (int64_t)t * K + k);
+        if (e < 0 || e >= N) {
+          flag_status(status, kStatusBounds);
+          continue;
+        }
+        sel |= (e / El == d);
+      }
+    }
+    int total;
+    const int pos = block_scan_flag(sel, sums, &total);
+    if (t < T) {
+      int32_t slot = -1;
+      if (sel) {
+        const int64_t s = (int64_t)before + running + pos;
+        if (s < send_cap) {
+          slot = (int32_t)s;
+          uint8_t* meta = send + s * row_bytes + meta_off;
+          int32_t* lid = reinterpret_cast<int32_t*>(meta);
+          float* g = reinterpret_cast<float*>(meta) + K;
+          for (int k = 0; k < K; ++k) {
+            const int e = __ldg(ids + (int64_t)t * K + k);
+            const bool here = e >= 0 && e < N && e / El == d;
+            lid[k] = here ? e - d * El : -1;
+            g[k] = here ? __ldg(gates + (int64_t)t * K + k) : 0.0f;
+          }
+        } else {
+          flag_status(status, kStatusBounds);
+        }
+      }
+      send_slot[(int64_t)t * W + d] = slot;
+    }
+    running += total;
+  }
+  if (threadIdx.x == 0) {
+    send_counts[2 * d] = rows_d;
+    send_counts[2 * d + 1] = pairs_d;
+    if (running != rows_d) flag_status(status, kStatusBounds);
+    if (d == 0) {  // the shared expert's single GEMM group: rows [0, T)
+      grp[0] = T;
+      grp[1] = 0;
+    }
+  }
+}
+
+// x -> 1x128 E4M3 codes and scales, written to the token's shared-expert row
+// t and to its send rows send_slot[t, d] (at most W <= 16). 8 threads per
+// tile, 16 elements each; lane k of a tile's 8 threads holds the slots of
+// ranks k and k + 8.
+__global__ void __launch_bounds__(256) ep_pack_kernel(const uint4* __restrict__ x, int T, int H,
+                                                      int W, const int32_t* __restrict__ send_slot,
+                                                      uint8_t* __restrict__ send, int64_t row_bytes,
+                                                      uint8_t* __restrict__ a_q,
+                                                      float* __restrict__ a_s) {
+  const int sub = threadIdx.x & 7;
+  const int tiles_per_row = H / kTile;
+  const int64_t n_tiles = (int64_t)T * tiles_per_row;
+  // the whole CTA iterates together so that every shuffle is warp-convergent
+  for (int64_t base = (int64_t)blockIdx.x * 32; base < n_tiles; base += (int64_t)gridDim.x * 32) {
+    const int64_t tile = base + (threadIdx.x >> 3);
+    const bool live = tile < n_tiles;
+    const int64_t t = live ? tile / tiles_per_row : 0;
+    const int c = live ? (int)(tile - t * tiles_per_row) : 0;
+    const uint4 v0 = live ? __ldcs(x + tile * 16 + 2 * sub) : make_uint4(0, 0, 0, 0);
+    const uint4 v1 = live ? __ldcs(x + tile * 16 + 2 * sub + 1) : make_uint4(0, 0, 0, 0);
+    const int slot_a = (live && sub < W) ? __ldg(send_slot + t * W + sub) : -1;
+    const int slot_b = (live && sub + 8 < W) ? __ldg(send_slot + t * W + sub + 8) : -1;
+    float f[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
+                   bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
+                   bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
+                   bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = tile_scale(amax);
+    uint4 out;
+    out.x = e4m3x4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
+    out.y = e4m3x4(__fmul_rn(f[4], s), __fmul_rn(f[5], s), __fmul_rn(f[6], s), __fmul_rn(f[7], s));
+    out.z = e4m3x4(__fmul_rn(f[8], s), __fmul_rn(f[9], s), __fmul_rn(f[10], s), __fmul_rn(f[11], s));
+    out.w = e4m3x4(__fmul_rn(f[12], s), __fmul_rn(f[13], s), __fmul_rn(f[14], s), __fmul_rn(f[15], s));
+    if (live) {
+      reinterpret_cast<uint4*>(a_q + t * H + (int64_t)c * kTile)[sub] = out;
+      if (sub == 0) a_s[t * tiles_per_row + c] = s;
+    }
+    for (int d = 0; d < W; ++d) {
+      const int sa = __shfl_sync(0xffffffffu, slot_a, d & 7, 8);
+      const int sb = __shfl_sync(0xffffffffu, slot_b, d & 7, 8);
+      const int slot = d < 8 ? sa : sb;
+      if (live && slot >= 0) {
+        uint8_t* row = send + (int64_t)slot * row_bytes;
+        reinterpret_cast<uint4*>(row + (int64_t)c * kTile)[sub] = out;
+        if (sub == 0) reinterpret_cast<float*>(row + H)[c] = s;
+      }
+    }
+  }
+}
+
+// Received rows: local ids and gates into dense [R, K] arrays, counts per
+// local expert (counts zero on entry).
+__global__ void __launch_bounds__(256) ep_recv_index_kernel(
+    const uint8_t* __restrict__ recv, int64_t R, int K, int H, int64_t row_bytes, int El,
+    int32_t* __restrict__ ids, float* __restrict__ gates, int32_t* __restrict__ counts,
+    uint32_t* __restrict__ status) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R * K) return;
+  const int64_t j = i / K;
+  const int k = (int)(i - j * K);
+  const uint8_t* meta = recv + j * row_bytes + meta_offset(H);
+  int lid = reinterpret_cast<const int32_t*>(meta)[k];
+  const float g = reinterpret_cast<const float*>(meta)[K + k];
+  if (lid < -1 || lid >= El) {
+    flag_status(status, kStatusBounds);
+    lid = -1;
+  }
+  ids[i] = lid;
+  gates[i] = g;
+  if (lid >= 0) atomicAdd(counts + lid, 1);
+}
+
+// Codes and scales of received row j copied to its GEMM rows token_row[j, k]
+// (slots without a row are skipped). 8 threads per 128-byte tile.
+__global__ void __launch_bounds__(256) ep_gather_rows_kernel(
+    const uint8_t* __restrict__ recv, int64_t R, int H, int K, int64_t row_bytes,
+    const int32_t* __restrict__ token_row, int64_t routed_cap, uint8_t* __restrict__ a_q,
+    float* __restrict__ a_s, uint32_t* __restrict__ status) {
+  const int sub = threadIdx.x & 7;
+  const int tiles_per_row = H / kTile;
+  const int64_t n_tiles = R * tiles_per_row;
+  for (int64_t base = (int64_t)blockIdx.x * 32; base < n_tiles; base += (int64_t)gridDim.x * 32) {
+    const int64_t tile = base + (threadIdx.x >> 3);
+    if (tile >= n_tiles) continue;  // no shuffles below
+    const int64_t j = tile / tiles_per_row;
+    const int c = (int)(tile - j * tiles_per_row);
+    const uint8_t* row = recv + j * row_bytes;
+    const uint4 v = reinterpret_cast<const uint4*>(row + (int64_t)c * kTile)[sub];
+    const float s = reinterpret_cast<const float*>(row + H)[c];
+    for (int k = 0; k < K; ++k) {
+      const int64_t r = __ldg(token_row + j * K + k);
+      if (r < 0) continue;
+      if (r >= routed_cap) {
+        if (sub == 0) flag_status(status, kStatusBounds);
+        continue;
+      }
+      reinterpret_cast<uint4*>(a_q + r * H + (int64_t)c * kTile)[sub] = v;
+      if (sub == 0) a_s[r * tiles_per_row + c] = s;
+    }
+  }
+}
+
+// Per received row: out[j] = sum over its local slots, by ascending expert
+// id, of g * Y[row], fp32 (the rank's share of the token's combine).
+__global__ void __launch_bounds__(128) ep_reduce_kernel(
+    const float* __restrict__ y_rows, const int32_t* __restrict__ ids,
+    const float* __restrict__ gates, const int32_t* __restrict__ token_row, int H, int K,
+    int64_t routed_cap, float* __restrict__ out, uint32_t* __restrict__ status) {
+  __shared__ int64_t s_row[kMaxK];
+  __shared__ float s_gate[kMaxK];
+  __shared__ int s_n;
+  const int64_t j = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int id[kMaxK];
+    int n = 0;
+    for (int k = 0; k < K; ++k) {
+      const int e = ids[j * K + k];
+      if (e < 0) continue;
+      const int64_t r = token_row[j * K + k];
+      if (r < 0 || r >= routed_cap) {
+        flag_status(status, kStatusBounds);
+        continue;
+      }
+      int m = n;  // insertion by ascending expert id
+      while (m > 0 && id[m - 1] > e) {
+        id[m] = id[m - 1];
+        s_row[m] = s_row[m - 1];
+        s_gate[m] = s_gate[m - 1];
+        --m;
+      }
+      id[m] = e;
+      s_row[m] = r;
+      s_gate[m] = gates[j * K + k];
+      ++n;
+    }
+    s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n;
+  float4* o = reinterpret_cast<float4*>(out + j * H);
+  for (int c = threadIdx.x; c < H / 4; c += blockDim.x) {
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int k = 0; k < n; ++k) {
+      const float4 u = __ldcs(reinterpret_cast<const float4*>(y_rows + s_row[k] * H) + c);
+      const float g = s_gate[k];
+      acc.x = fmaf(g, u.x, acc.x);
+      acc.y = fmaf(g, u.y, acc.y);
+      acc.z = fmaf(g, u.z, acc.z);
+      acc.w = fmaf(g, u.w, acc.w);
+    }
+    o[c] = acc;
+  }
+}
+
+// y_t = shared_t + the returned partial sums of t's send rows, ranks
+// ascending, fp32, one rounding to bf16.
+__global__ void __launch_bounds__(128) ep_combine_kernel(
+    const float* __restrict__ y_shared, const float* __restrict__ ret,
+    const int32_t* __restrict__ send_slot, int H, int W, int64_t ret_rows,
+    __nv_bfloat16* __restrict__ y, uint32_t* __restrict__ status) {
+  __shared__ int64_t s_slot[kMaxRanks];
+  __shared__ int s_n;
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int d = 0; d < W; ++d) {
+      const int64_t slot = send_slot[t * W + d];
+      if (slot < 0) continue;
+      if (slot >= ret_rows) {
+        flag_status(status, kStatusBounds);
+        continue;
+      }
+      s_slot[n++] = slot;
+    }
+    s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n;
+  const float4* ys = reinterpret_cast<const float4*>(y_shared + t * H);
+  uint4* out = reinterpret_cast<uint4*>(y + t * H);
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    const float4 v0 = __ldcs(ys + 2 * c), v1 = __ldcs(ys + 2 * c + 1);
+    float acc[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    for (int i = 0; i < n; ++i) {
+      const float4* p = reinterpret_cast<const float4*>(ret + s_slot[i] * H);
+      const float4 u0 = __ldcs(p + 2 * c), u1 = __ldcs(p + 2 * c + 1);
+      acc[0] += u0.x;
+      acc[1] += u0.y;
+      acc[2] += u0.z;
+      acc[3] += u0.w;
+      acc[4] += u1.x;
+      acc[5] += u1.y;
+      acc[6] += u1.z;
+      acc[7] += u1.w;
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    out[c] = o;
+  }
+}
+
+unsigned tile_grid(int64_t n_tiles) {
+  int64_t blocks = (n_tiles + 31) / 32;
+  const int64_t cap = (int64_t)moe_device_sm_count() * 8;
+  if (cap > 0 && blocks > cap) blocks = cap;
+  return (unsigned)(blocks > 0 ? blocks : 1);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int64_t moe_ep_row_bytes(moe_shape sh) { return shape_ok(sh) ? row_bytes_of(sh) : 0; }
+
+size_t moe_ep_dispatch_workspace_size(moe_shape sh, int32_t W) {
+  return ep_ok(sh, W) ? source_layout(sh, W).total : 0;
+}
+
+size_t moe_ep_expert_workspace_size(moe_shape sh, int32_t W, int64_t R, int64_t pairs) {
+  if (!ep_ok(sh, W) || R < 0 || pairs < 0 || pairs > R * sh.K || R * sh.K >= (1ll << 31))
+    return 0;
+  return expert_layout(sh, W, R, pairs).total;
+}
+
+int moe_ep_dispatch(moe_shape sh, int32_t W, const float* gate_w, const void* x, const float* bias,
+                    int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
+                    uint8_t* send, int64_t send_cap, int32_t* send_counts, void* ws,
+                    size_t ws_bytes, void* stream) {
+  if (!ep_ok(sh, W) || send_cap < 0 || send_cap >= (1ll << 31)) return MOE_ERR_SHAPE;
+  if (!send_counts || !ws) return MOE_ERR_NULL;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
+  const SourceLayout L = source_layout(sh, W);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  int32_t* counts = counts_opt ? counts_opt : at<int32_t>(ws, L.counts);
+  cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(send_counts, 0, (size_t)W * 2 * 4, s);
+  if (sh.T == 0 || e != cudaSuccess) return cuda_status(e);
+  if (!gate_w || !x || !bias || !send) return MOE_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(gate_w, 16) || !aligned(send, 16)) return MOE_ERR_ALIGN;
+  const int sms = moe_device_sm_count();
+  int32_t* ids = topk_ids_opt ? topk_ids_opt : at<int32_t>(ws, L.topk_ids);
+  float* gates = topk_gates_opt ? topk_gates_opt : at<float>(ws, L.topk_gates);
+  e = launch_router_tc(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
+                       at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
+                       counts, status, s, sms);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const int64_t rb = row_bytes_of(sh);
+  int32_t* send_slot = at<int32_t>(ws, L.send_slot);
+  ep_plan_kernel<<<W, 1024, 0, s>>>(ids, gates, sh.T, sh.K, sh.N, W, sh.H, send, rb, send_cap,
+                                    send_slot, send_counts, at<int32_t>(ws, L.grp), status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const int64_t n_tiles = (int64_t)sh.T * (sh.H / kTile);
+  ep_pack_kernel<<<tile_grid(n_tiles), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), sh.T, sh.H,
+                                                    W, send_slot, send, rb,
+                                                    at<uint8_t>(ws, L.a_q), at<float>(ws, L.a_s));
+  return cuda_status(cudaGetLastError());
+}
+
+int moe_ep_shared(moe_shape sh, int32_t W, const moe_weights* w_local, void* ws, size_t ws_bytes,
+                  void* stream) {
+  if (!ep_ok(sh, W)) return MOE_ERR_SHAPE;
+  if (!ws) return MOE_ERR_NULL;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
+  const SourceLayout L = source_layout(sh, W);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (sh.T == 0) return MOE_OK;
+  if (!w_local || !w_local->w13 || !w_local->s13 || !w_local->w2 || !w_local->s2)
+    return MOE_ERR_NULL;
+  if (!aligned(w_local->w13, 16) || !aligned(w_local->w2, 16)) return MOE_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = moe_device_sm_count();
+  const int64_t El = sh.N / W, H = sh.H, I = sh.I;
+  // the shared expert is the last of the rank's El + 1 weight sets
+  const uint8_t* w13 = w_local->w13 + El * 2 * I * H;
+  const float* s13 = w_local->s13 + El * (2 * I / kTile) * (H / kTile);
+  const uint8_t* w2 = w_local->w2 + El * H * I;
+  const float* s2 = w_local->s2 + El * (H / kTile) * (I / kTile);
+  const int32_t* grp = at<int32_t>(ws, L.grp);
+  GroupedGemm gg{sh.H, sh.I, 1, grp, grp + 1, L.rows, at<uint32_t>(ws, L.status)};
+  cudaError_t e = launch_expert_up(gg, at<uint8_t>(ws, L.a_q), at<float>(ws, L.a_s), w13, s13,
+                                   at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), s, sms);
+  if (e == cudaSuccess)
+    e = launch_expert_down(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w2, s2,
+                           at<float>(ws, L.y_shared), s, sms);
+  return cuda_status(e);
+}
+
+int moe_ep_experts(moe_shape sh, int32_t W, const moe_weights* w_local, const uint8_t* recv,
+                   int64_t R, int64_t pairs, float* out, void* ws, size_t ws_bytes,
+                   void* stream) {
+  if (!ep_ok(sh, W) || R < 0 || pairs < 0 || pairs > R * sh.K || R * sh.K >= (1ll << 31))
+    return MOE_ERR_SHAPE;
+  if (!ws) return MOE_ERR_NULL;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
+  const ExpertLayout L = expert_layout(sh, W, R, pairs);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
+  if (R == 0 || e != cudaSuccess) return cuda_status(e);
+  if (!w_local || !w_local->w13 || !w_local->s13 || !w_local->w2 || !w_local->s2 || !recv || !out)
+    return MOE_ERR_NULL;
+  if (!aligned(w_local->w13, 16) || !aligned(w_local->w2, 16) || !aligned(recv, 16) ||
+      !aligned(out, 16))
+    return MOE_ERR_ALIGN;
+  const int sms = moe_device_sm_count();
+  const int El = sh.N / W;
+  const int64_t rb = row_bytes_of(sh);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* ids = at<int32_t>(ws, L.ids);
+  float* gates = at<float>(ws, L.gates);
+  int32_t* token_row = at<int32_t>(ws, L.token_row);
+  e = cudaMemsetAsync(counts, 0, (size_t)El * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(token_row, 0xFF, (size_t)(R * sh.K) * 4, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const int64_t n_idx = R * sh.K;
+  ep_recv_index_kernel<<<(unsigned)((n_idx + 255) / 256), 256, 0, s>>>(recv, R, sh.K, sh.H, rb, El,
+                                                                       ids, gates, counts, status);
+  e = cudaGetLastError();
+  if (e == cudaSuccess)
+    e = launch_permute(ids, counts, (int)R, El, sh.K, pairs, L.routed_cap,
+                       at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.group_rows),
+                       at<int32_t>(ws, L.row_start), at<int32_t>(ws, L.row_token), token_row,
+                       status, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const int64_t n_tiles = R * (sh.H / kTile);
+  ep_gather_rows_kernel<<<tile_grid(n_tiles), 256, 0, s>>>(recv, R, sh.H, sh.K, rb, token_row,
+                                                           L.routed_cap, at<uint8_t>(ws, L.a_q),
+                                                           at<float>(ws, L.a_s), status);
+  e = cudaGetLastError();
+  GroupedGemm gg{sh.H, sh.I, El, at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
+                 L.routed_cap, status};
+  if (e == cudaSuccess)
+    e = launch_expert_up(gg, at<uint8_t>(ws, L.a_q), at<float>(ws, L.a_s), w_local->w13,
+                         w_local->s13, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), s, sms);
+  if (e == cudaSuccess)
+    e = launch_expert_down(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w_local->w2,
+                           w_local->s2, at<float>(ws, L.y_rows), s, sms);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  ep_reduce_kernel<<<(unsigned)R, 128, 0, s>>>(at<float>(ws, L.y_rows), ids, gates, token_row,
+                                               sh.H, sh.K, L.routed_cap, out, status);
+  return cuda_status(cudaGetLastError());
+}
+
+int moe_ep_combine(moe_shape sh, int32_t W, const float* ret, int64_t ret_rows, void* ws,
+                   size_t ws_bytes, void* y, void* stream) {
+  if (!ep_ok(sh, W) || ret_rows < 0) return MOE_ERR_SHAPE;
+  if (!ws) return MOE_ERR_NULL;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
+  const SourceLayout L = source_layout(sh, W);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (sh.T == 0) return MOE_OK;
+  if (!y || (ret_rows > 0 && !ret)) return MOE_ERR_NULL;
+  if (!aligned(y, 16) || !aligned(ret, 16)) return MOE_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ep_combine_kernel<<<(unsigned)sh.T, 128, 0, s>>>(
+      at<float>(ws, L.y_shared), ret, at<int32_t>(ws, L.send_slot), sh.H, W, ret_rows,
+      static_cast<__nv_bfloat16*>(y), at<uint32_t>(ws, L.status));
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -86,9 +86,11 @@ cudaError_t launch_balance_stats(const float* logits, const int32_t* ids, int T,
                                  float* loss, cudaStream_t stream);
 
 // Permutation: scan of counts into group tables, stable scatter of the
-// (token, slot) pairs into expert-major GEMM rows.
+// (token, slot) pairs into expert-major GEMM rows. Slots whose id is
+// negative are skipped (their token_row entries are left as they are);
+// `pairs` is the number of slots with an id, checked against the counts.
 cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K,
-                           int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
+                           int64_t pairs, int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
                            int32_t* row_start, int32_t* row_token, int32_t* token_row,
                            uint32_t* status, cudaStream_t stream);
 // 1x128 quantisation of x written to each token's shared-expert row

@@ -7,72 +7,17 @@
 //             order, with a block-wide prefix sum over ballots, and records
 //             each (token, slot)'s GEMM row; the activation quantiser then
 //             writes every token's codes straight into its rows
+#include "block_scan.cuh"
 #include "kernels.cuh"
 
 namespace moe {
 
 namespace {
 
-// Block-wide exclusive prefix sum of a 0/1 flag over up to 1024 threads.
-// Returns this thread's prefix; *total receives the block sum.
-MOE_DEV int block_scan_flag(bool flag, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nwarps = blockDim.x >> 5;
-  const uint32_t ballot = __ballot_sync(0xffffffffu, flag);
-  const int in_warp = __popc(ballot & ((1u << lane) - 1u));
-  if (lane == 0) warp_sums[warp] = __popc(ballot);
-  __syncthreads();
-  if (warp == 0) {
-    int v = lane < nwarps ? warp_sums[lane] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += u;
-    }
-    if (lane < nwarps) warp_sums[lane] = incl - v;
-    if (lane == 31) warp_sums[32] = incl;
-  }
-  __syncthreads();
-  const int res = warp_sums[warp] + in_warp;
-  *total = warp_sums[32];
-  __syncthreads();
-  return res;
-}
-
-// Exclusive scan of v over the block (up to 1024 threads, one value each).
-MOE_DEV int block_scan_int(int v, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nwarps = blockDim.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < nwarps ? warp_sums[lane] : 0;
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += u;
-    }
-    if (lane < nwarps) warp_sums[lane] = wi - w;
-    if (lane == 31) warp_sums[32] = wi;
-  }
-  __syncthreads();
-  const int res = warp_sums[warp] + incl - v;
-  *total = warp_sums[32];
-  __syncthreads();
-  return res;
-}
-
-// One CTA of 1024 threads; N <= 1024.
+// One CTA of 1024 threads; N <= 1024. `pairs` is the number of (token, slot)
+// pairs the counts must add up to.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ counts, int N,
-                                                    int T, int K, int64_t routed_cap,
+                                                    int T, int64_t pairs, int64_t routed_cap,
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ group_rows,
                                                     int32_t* __restrict__ row_start,
@@ -93,7 +38,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
     offsets[N] = total_c;
     group_rows[N] = T;
     row_start[N] = (int32_t)routed_cap;
-    if ((int64_t)total_c != (int64_t)T * K || (int64_t)total_p > routed_cap) {
+    if ((int64_t)total_c != pairs || (int64_t)total_p > routed_cap) {
       flag_status(status, kStatusBounds);
     }
   }
@@ -139,11 +84,11 @@ __global__ void __launch_bounds__(1024) scatter_kernel(const int32_t* __restrict
 }  // namespace
 
 cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K,
-                           int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
+                           int64_t pairs, int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
                            int32_t* row_start, int32_t* row_token, int32_t* token_row,
                            uint32_t* status, cudaStream_t stream) {
-  scan_kernel<<<1, 1024, 0, stream>>>(counts, N, T, K, routed_cap, offsets, group_rows, row_start,
-                                      status);
+  scan_kernel<<<1, 1024, 0, stream>>>(counts, N, T, pairs, routed_cap, offsets, group_rows,
+                                      row_start, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(row_token, 0xFF, (size_t)routed_cap * sizeof(int32_t), stream);

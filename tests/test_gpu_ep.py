@@ -1,0 +1,250 @@
+"""GPU parity of the expert-parallel layer (the moe_ep_* calls through the C
+ABI). W ranks are emulated one after another on one GPU: every rank's
+dispatch, then the exchange done by slicing (what an all-to-all delivers:
+rows source-major, each source's rows in its send order), every rank's
+experts, the exchange back, every rank's combine. No kernel waits on another
+rank's work.
+
+Checks, per rank:
+  * routing, gates and counts identical to moe_forward's on the same tokens;
+  * the send plan (row counts, pair counts, slots: destination-major, tokens
+    ascending) and every packed row's local ids and gates, bit-exact against
+    their definition; the packed codes and scales bit-exact against the
+    oracle's 1x128 quantisation;
+  * the output against moe_forward with all experts on one GPU: each expert
+    output is the same GEMM result, only the order of the fp32 additions in
+    the combine differs, so values agree to one bf16 ulp (plus a 4e-6 RMS
+    allowance for cancellation) and almost all are identical;
+  * the output against the oracle (small shapes), as for the forward.
+The product's ExpertParallelMoE is also run over a real one-rank NCCL group."""
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from mixture_experts_layer_40_b200 import capi, ep
+from mixture_experts_layer_40_b200 import inputs as I
+from mixture_experts_layer_40_b200.layer import MoELayer, device_weights
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from __graft_entry__ import build
+    build()
+    assert torch.cuda.is_available()
+
+
+def rank_x(w: I.Workload, rank: int, T: int) -> np.ndarray:
+    return I.make_x(I.Workload(w.name, T=T, H=w.H, N=w.N, K=w.K, I=w.I, seed=w.seed + 101 * (rank + 1)))
+
+
+def emulate(w: I.Workload, W: int, xs_bits, dw, bias: np.ndarray, G: int = 0, M: int = 0):
+    """One expert-parallel step over W emulated ranks; returns per-rank dicts."""
+    N, K, Hd = w.N, w.K, w.H
+    el = N // W
+    bd = torch.from_numpy(bias).cuda()
+    wl_t = [ep.local_weights(dw.w13, dw.s13, dw.w2, dw.s2, N, W, r) for r in range(W)]
+    wl = [capi.make_weights(dw.gate_w, *t) for t in wl_t]
+    rb = capi.moe_ep_row_bytes(capi.shape_of(1, Hd, N, K, w.I, G, M))
+    ranks = []
+    for r, xb in enumerate(xs_bits):
+        T = xb.shape[0]
+        sh = capi.shape_of(T, Hd, N, K, w.I, G, M)
+        st = {"T": T, "sh": sh, "x_bits": xb}
+        st["xd"] = H.x_to_device(xb) if T else torch.empty(0, Hd, dtype=torch.bfloat16,
+                                                             device="cuda")
+        st["send"] = torch.zeros(max(T * min(W, K), 1), rb, dtype=torch.uint8, device="cuda")
+        st["sc"] = torch.full((W, 2), -7, dtype=torch.int32, device="cuda")
+        st["ws"] = torch.empty(capi.moe_ep_dispatch_workspace_size(sh, W), dtype=torch.uint8,
+                               device="cuda")
+        st["ids"] = torch.empty(T, K, dtype=torch.int32, device="cuda")
+        st["gates"] = torch.empty(T, K, dtype=torch.float32, device="cuda")
+        st["counts"] = torch.full((N,), -1, dtype=torch.int32, device="cuda")
+        capi.moe_ep_dispatch(sh, W, dw.gate_w, st["xd"], bd, st["send"], st["sc"], st["ws"],
+                             topk_ids=st["ids"] if T else None,
+                             topk_gates=st["gates"] if T else None, counts=st["counts"])
+        capi.moe_ep_shared(sh, W, wl[r], st["ws"])
+        ranks.append(st)
+    torch.cuda.synchronize()
+    rows = np.stack([st["sc"].cpu().numpy()[:, 0] for st in ranks])   # [src, dst]
+    pairs = np.stack([st["sc"].cpu().numpy()[:, 1] for st in ranks])
+    off = np.concatenate([np.zeros((W, 1), np.int64), np.cumsum(rows, axis=1)], axis=1)
+    outs = []
+    for d in range(W):
+        recv = torch.cat([ranks[s]["send"][off[s, d]:off[s, d + 1]] for s in range(W)])
+        R, P = int(rows[:, d].sum()), int(pairs[:, d].sum())
+        sh = ranks[0]["sh"]
+        ews = torch.empty(capi.moe_ep_expert_workspace_size(sh, W, R, P), dtype=torch.uint8,
+                          device="cuda")
+        out = torch.empty(R, Hd, dtype=torch.float32, device="cuda")
+        capi.moe_ep_experts(sh, W, wl[d], recv, R, P, out, ews)
+        assert capi.moe_get_status(ews) == 0
+        outs.append(out)
+    for s, st in enumerate(ranks):
+        # rank d's output rows from source s sit after those of sources < s
+        parts = []
+        for d in range(W):
+            start = int(rows[:s, d].sum())
+            parts.append(outs[d][start:start + rows[s, d]])
+        ret = torch.cat(parts)
+        y = torch.empty(st["T"], Hd, dtype=torch.bfloat16, device="cuda")
+        capi.moe_ep_combine(st["sh"], W, ret, int(rows[s].sum()), st["ws"], y)
+        assert capi.moe_get_status(st["ws"]) == 0
+        st["y"] = y
+        st["rows"], st["pairs"] = rows[s], pairs[s]
+    torch.cuda.synchronize()
+    return ranks
+
+
+def check_plan(w: I.Workload, W: int, st):
+    T, K, el = st["T"], w.K, w.N // W
+    rows, pairs = st["rows"], st["pairs"]
+    if T == 0:
+        assert not rows.any() and not pairs.any()
+        return
+    ids = st["ids"].cpu().numpy()
+    gates = st["gates"].cpu().numpy()
+    dest = ids // el
+    expect_rows = [int(np.any(dest == d, axis=1).sum()) for d in range(W)]
+    expect_pairs = [int((dest == d).sum()) for d in range(W)]
+    assert list(rows) == expect_rows and list(pairs) == expect_pairs
+    send = st["send"].cpu().numpy()
+    hd = w.H
+    q, s = O.quantize_1x128(I.bf16_bits_to_f32(st["x_bits"]))
+    slot = 0
+    for d in range(W):
+        for t in np.nonzero(np.any(dest == d, axis=1))[0]:
+            row = send[slot]
+            assert np.array_equal(row[:hd], q[t])
+            assert np.array_equal(row[hd:hd + 4 * (hd // 128)].view(np.uint32), s[t].view(np.uint32))
+            meta = row[hd + 4 * (hd // 128):hd + 4 * (hd // 128) + 8 * K]
+            lid = meta[:4 * K].view(np.int32)
+            g = meta[4 * K:].view(np.float32)
+            here = dest[t] == d
+            assert np.array_equal(lid, np.where(here, ids[t] - d * el, -1))
+            assert np.array_equal(g.view(np.uint32), np.where(here, gates[t], 0.0).astype(np.float32).view(np.uint32))
+            slot += 1
+    assert slot == sum(expect_rows)
+
+
+def check_against_forward(w: I.Workload, st, dw, bias, G=0, M=0):
+    T = st["T"]
+    if T == 0:
+        return None
+    layer = MoELayer(T, w.H, w.N, w.K, w.I, dw, groups=G, topk_groups=M)
+    y_f = layer.forward(st["xd"], torch.from_numpy(bias).cuda())
+    assert layer.status() == 0
+    assert torch.equal(layer.ids, st["ids"]) and torch.equal(layer.gates, st["gates"])
+    assert torch.equal(layer.counts, st["counts"])
+    a = st["y"].float().cpu().numpy()
+    b = y_f.float().cpu().numpy()
+    rms = float(np.sqrt(np.mean(b.astype(np.float64) ** 2)))
+    _, e = np.frexp(np.maximum(np.abs(a), np.abs(b)))
+    ulp = np.ldexp(1.0, e - 8)  # bf16: 8 significant bits
+    diff = np.abs(a - b)
+    assert np.all(diff <= ulp + 4e-6 * rms), float(np.max(diff / (ulp + 4e-6 * rms)))
+    assert np.mean(a == b) >= 0.95
+    return layer
+
+
+def check_against_oracle(w: I.Workload, st, case_gate_w, ew, bias):
+    if st["T"] == 0:
+        return
+    x = I.bf16_bits_to_f32(st["x_bits"])
+    ids = st["ids"].cpu().numpy()
+    ref = O.moe_forward(x, case_gate_w, bias, w.K, ew, mode="Q", ids=ids)
+    H.check_rows(st["y"].float().cpu().numpy(), ref["y"])
+
+
+def _setup(w: I.Workload):
+    case = H.make_case(w)
+    dw = device_weights(w, case.pool, case.gate_w, "cuda")
+    return case, dw
+
+
+@pytest.mark.parametrize("W,Ts", [(2, [300, 171]), (2, [77, 0])])
+def test_ep_two_ranks(W, Ts):
+    w = I.Workload("ep2", T=max(Ts), H=512, N=32, K=4, I=256, bias_range=0.1, seed=21)
+    case, dw = _setup(w)
+    xs = [rank_x(w, r, t) for r, t in enumerate(Ts)]
+    ranks = emulate(w, W, xs, dw, case.bias)
+    for st in ranks:
+        check_plan(w, W, st)
+        check_against_forward(w, st, dw, case.bias)
+        check_against_oracle(w, st, case.gate_w, case.ew, case.bias)
+
+
+def test_ep_four_ranks_node_limited():
+    # groups = ranks: every token reaches at most 2 of the 4 ranks
+    w = I.Workload("ep4", T=200, H=256, N=64, K=4, I=128, bias_range=0.1, seed=22)
+    case, dw = _setup(w)
+    Ts = [200, 1, 0, 129]
+    xs = [rank_x(w, r, t) for r, t in enumerate(Ts)]
+    ranks = emulate(w, 4, xs, dw, case.bias, G=4, M=2)
+    for st in ranks:
+        check_plan(w, 4, st)
+        if st["T"]:
+            dest = st["ids"].cpu().numpy() // 16
+            assert max(len(set(r)) for r in dest) <= 2
+        check_against_forward(w, st, dw, case.bias, G=4, M=2)
+
+
+def test_ep_all_tokens_on_one_rank():
+    # the bias sends every token to experts 0..3, all on rank 0: rank 1 gets no rows
+    w = I.Workload("ep1", T=150, H=256, N=32, K=4, I=128, bias_range=0.1, seed=23)
+    case, dw = _setup(w)
+    bias = case.bias.copy()
+    bias[:4] = 5.0
+    xs = [rank_x(w, r, 150) for r in range(2)]
+    ranks = emulate(w, 2, xs, dw, bias)
+    for st in ranks:
+        assert list(st["rows"]) == [150, 0] and list(st["pairs"]) == [600, 0]
+        check_plan(w, 2, st)
+        check_against_forward(w, st, dw, bias)
+
+
+def test_ep_v3_shape_eight_ranks():
+    w = I.WORKLOADS["v3_prefill"]
+    case, dw = _setup(w)
+    Ts = [96, 130, 64, 1, 128, 100, 37, 96]
+    xs = [rank_x(w, r, t) for r, t in enumerate(Ts)]
+    ranks = emulate(w, 8, xs, dw, case.bias)
+    for st in ranks:
+        check_plan(w, 8, st)
+        check_against_forward(w, st, dw, case.bias)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_expert_parallel_layer_one_rank_nccl():
+    import torch.distributed as dist
+    w = I.Workload("ep_nccl", T=256, H=512, N=32, K=4, I=256, bias_range=0.1, seed=24)
+    case, dw = _setup(w)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1)
+    try:
+        w13, s13, w2, s2 = ep.local_weights(dw.w13, dw.s13, dw.w2, dw.s2, w.N, 1, 0)
+        layer = ep.ExpertParallelMoE(w.T, w.H, w.N, w.K, w.I, 1, 0, dw.gate_w, w13, s13, w2, s2)
+        xb = rank_x(w, 0, 200)
+        xd = H.x_to_device(xb)
+        bd = torch.from_numpy(case.bias).cuda()
+        y = layer.forward(xd, bd)
+        torch.cuda.synchronize()
+        assert layer.status() == 0
+        assert layer.last["send_rows"] == [200] and layer.last["pairs"] == 800
+        st = {"T": 200, "xd": xd, "y": y, "ids": layer.ids[:200], "gates": layer.gates[:200],
+              "counts": layer.counts}
+        check_against_forward(w, st, dw, case.bias)
+        total = layer.batch_counts()
+        assert int(total.sum()) == 800
+    finally:
+        dist.destroy_process_group()
