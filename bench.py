@@ -51,6 +51,9 @@ def parse():
     p.add_argument("--groups", type=int, default=0,
                    help="node-limited routing: G expert groups (0: top-K over all N)")
     p.add_argument("--topk-groups", type=int, default=0, help="node-limited routing: M groups")
+    p.add_argument("--ep", action="store_true",
+                   help="expert parallelism: the routed experts sharded over the ranks "
+                        "(ep.ExpertParallelMoE), every rank routing its own batch")
     p.add_argument("--backward", action="store_true",
                    help="also time the FP8 expert backward (Dgrad + Wgrad) after the forward")
     p.add_argument("--seq-len", type=int, default=0,
@@ -579,6 +582,122 @@ def run_ours(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_ep(args, w, rank, world, local_rank):
+    """One expert-parallel step per iteration: every rank routes its own T
+    tokens, holds N/world routed experts and the shared expert, and exchanges
+    rows with the others over NCCL (ep.ExpertParallelMoE); then the
+    batch-level bias update. Weak scaling over ranks."""
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    from __graft_entry__ import build
+    build()
+    from mixture_experts_layer_40_b200 import capi, ep
+    from mixture_experts_layer_40_b200 import inputs as I
+    from mixture_experts_layer_40_b200.layer import device_weights
+
+    own_group = False
+    if not dist.is_initialized():   # one rank without torchrun: a one-rank NCCL group
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1)
+        own_group = True
+    try:
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        pool = I.make_weight_pool(w)
+        gate_w = I.make_gate_w(w)
+        full = device_weights(w, pool, gate_w, dev)
+        del pool
+        local = ep.local_weights(full.w13, full.s13, full.w2, full.s2, w.N, world, rank)
+        gw = full.gate_w
+        del full
+        torch.cuda.empty_cache()
+        layer = ep.ExpertParallelMoE(w.T, w.H, w.N, w.K, w.I, world, rank, gw, *local,
+                                     groups=args.groups, topk_groups=args.topk_groups)
+        x_bits = I.make_x(rank_batch(w, rank))
+        x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        x = x_host.to(dev)
+        y_host = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
+        bias = torch.from_numpy(I.make_bias(w)).to(dev)
+        stream = torch.cuda.current_stream()
+
+        def step(x_in):
+            y = layer.forward(x_in, bias)
+            total = layer.batch_counts()
+            capi.moe_update_bias(bias, total, w.N, w.T * world, w.K, w.gamma)
+            return y
+
+        def barrier():
+            dist.barrier()
+            torch.cuda.synchronize()
+
+        for _ in range(args.warmup):
+            step(x)
+        barrier()
+        if layer.status() != 0:
+            raise RuntimeError("device status error during warm-up")
+        clocks = ClockSampler(local_rank) if rank == 0 else None
+        if clocks:
+            clocks.start()
+        barrier()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(x)
+        t1.record(stream)
+        barrier()
+        ms_step = max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps
+        if layer.status() != 0:
+            raise RuntimeError("device status error in the timed region")
+        # end to end: each step uploads x from pinned memory and downloads y
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            xd = x_host.to(dev, non_blocking=True)
+            y_host.copy_(step(xd), non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+        clk = clocks.stop() if clocks else None
+        last = layer.last
+        rb = layer.row_bytes
+        send = int(sum(last["send_rows"]))
+        if rank == 0:
+            line = {
+                "metric": METRIC, "value": w.T * world / (ms_step * 1e-3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+                "config": dict(run_config(args, w, world),
+                               parallelism=f"ep{world} (routed experts sharded over ranks; own "
+                                           f"batch per GPU)"),
+                "gpu_launches": 16 * args.steps,
+                "e2e": {"value": w.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2,
+                        "copies": "pinned host buffers, on the compute stream"},
+                "clocks": clk,
+                "ep": {"ranks": world, "experts_per_rank": w.N // world,
+                       "send_rows_rank0": last["send_rows"], "recv_rows_rank0": last["recv_rows"],
+                       "dispatch_bytes_rank0": send * rb, "return_bytes_rank0": send * w.H * 4,
+                       "host_syncs_per_step": 1,
+                       "note": "library kernels: dispatch (router, plan, pack), shared expert, "
+                               "local experts, combine, bias update; exchanges: NCCL "
+                               "all-to-all of counts, rows and partial sums, all-reduce of "
+                               "counts"},
+            }
+            print(json.dumps(line), flush=True)
+    finally:
+        if own_group:
+            dist.destroy_process_group()
+
+
 def main():
     args = parse()
     from mixture_experts_layer_40_b200 import inputs as I
@@ -598,7 +717,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, w, rank, world, local_rank)
+        if args.ep:
+            run_ep(args, w, rank, world, local_rank)
+        else:
+            run_ours(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
