@@ -605,7 +605,7 @@ def run_ep(args, w, rank, world, local_rank):
             port = sk.getsockname()[1]
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
-                                world_size=1)
+                                world_size=1, device_id=torch.device("cuda", local_rank))
         own_group = True
     try:
         dev = torch.device("cuda", local_rank)
