@@ -55,7 +55,7 @@ __host__ __device__ inline int64_t meta_offset(int H) { return (int64_t)H + 4 * 
 
 struct SourceLayout {
   int64_t rows;  // shared-expert GEMM rows (T rounded up to 128)
-  size_t status, counts, topk_ids, topk_gates, logits, gate_split, send_slot, grp;
+  size_t status, counts, topk_ids, topk_gates, logits, gate_split, send_slot, grp, plan;
   size_t a_q, a_s, h_q, h_s, y_shared, total;
 };
 
@@ -77,6 +77,7 @@ SourceLayout source_layout(const moe_shape& sh, int W) {
   L.gate_split = take(router_split_bytes((int)N, (int)H));
   L.send_slot = take((size_t)(T * W) * 4);
   L.grp = take(2 * 4);
+  L.plan = take((size_t)2 * ((T + 1023) / 1024) * W * 4);  // per-chunk rows and pairs
   L.a_q = take((size_t)(L.rows * H));
   L.a_s = take((size_t)(L.rows * (H / kTile)) * 4);
   L.h_q = take((size_t)(L.rows * I));
@@ -133,84 +134,113 @@ MOE_DEV int block_sum(int v, int* red) {
   return r;
 }
 
-// Dispatch plan: one CTA (1024 threads) per destination rank d. Pass 1 counts
-// the tokens bound for d, those bound for lower ranks (which precede d's rows
-// in the send buffer) and the (token, slot) pairs for d; pass 2 numbers d's
-// tokens in token order and writes each row's local ids and gates.
-__global__ void __launch_bounds__(1024) ep_plan_kernel(
-    const int32_t* __restrict__ ids, const float* __restrict__ gates, int T, int K, int N, int W,
-    int H, uint8_t* __restrict__ send, int64_t row_bytes, int64_t send_cap,
-    int32_t* __restrict__ send_slot, int32_t* __restrict__ send_counts, int32_t* __restrict__ grp,
-    uint32_t* __restrict__ status) {
-  __shared__ int sums[33];
+// Dispatch plan, in chunks of kPlanChunk tokens (one thread per token).
+// ep_count_kernel, one CTA per chunk: per destination rank d, the chunk's
+// tokens bound for d (rows) and its (token, slot) pairs for d.
+// ep_slot_kernel, one CTA per (chunk, d): the chunk's first row for d is the
+// rows of every lower rank plus d's rows in earlier chunks; a block scan
+// numbers the chunk's tokens for d in token order, and each row gets its
+// local ids and gates. Positions come from scans only, never from atomics.
+constexpr int kPlanChunk = 1024;
+
+__global__ void __launch_bounds__(kPlanChunk) ep_count_kernel(
+    const int32_t* __restrict__ ids, int T, int K, int N, int W, int32_t* __restrict__ chunk_rows,
+    int32_t* __restrict__ chunk_pairs, uint32_t* __restrict__ status) {
   __shared__ int red[32];
-  const int d = blockIdx.x;
+  const int c = blockIdx.x;
+  const int t = c * kPlanChunk + threadIdx.x;
   const int El = N / W;
-  int rows_d = 0, before = 0, pairs_d = 0;
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    uint32_t mask = 0;
+  uint32_t mask = 0;
+  int np[kMaxRanks];
+#pragma unroll
+  for (int d = 0; d < kMaxRanks; ++d) np[d] = 0;
+  if (t < T) {
     for (int k = 0; k < K; ++k) {
       const int e = __ldg(ids + (int64_t)t * K + k);
-      if (e < 0 || e >= N) continue;  // flagged below
+      if (e < 0 || e >= N) {
+        flag_status(status, kStatusBounds);
+        continue;
+      }
       const int r = e / El;
       mask |= 1u << r;
-      pairs_d += (r == d);
+#pragma unroll
+      for (int d = 0; d < kMaxRanks; ++d) np[d] += (r == d);
     }
-    rows_d += (int)((mask >> d) & 1u);
-    before += __popc(mask & ((1u << d) - 1u));
   }
-  rows_d = block_sum(rows_d, red);
-  before = block_sum(before, red);
-  pairs_d = block_sum(pairs_d, red);
-  const int64_t meta_off = meta_offset(H);
-  int running = 0;
-  for (int t0 = 0; t0 < T; t0 += blockDim.x) {
-    const int t = t0 + threadIdx.x;
-    bool sel = false;
-    if (t < T) {
+#pragma unroll
+  for (int d = 0; d < kMaxRanks; ++d) {
+    if (d < W) {  // the same for the whole block, so the barriers inside are safe
+      const int rows = __syncthreads_count((mask >> d) & 1u);
+      const int pairs = block_sum(np[d], red);
+      if (threadIdx.x == 0) {
+        chunk_rows[c * W + d] = rows;
+        chunk_pairs[c * W + d] = pairs;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPlanChunk) ep_slot_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ gates, int T, int K, int N, int W,
+    int H, int n_chunks, const int32_t* __restrict__ chunk_rows,
+    const int32_t* __restrict__ chunk_pairs, uint8_t* __restrict__ send, int64_t row_bytes,
+    int64_t send_cap, int32_t* __restrict__ send_slot, int32_t* __restrict__ send_counts,
+    int32_t* __restrict__ grp, uint32_t* __restrict__ status) {
+  __shared__ int sums[33];
+  __shared__ int64_t s_base;
+  const int c = blockIdx.x, d = blockIdx.y;
+  const int El = N / W;
+  if (threadIdx.x == 0) {
+    int64_t base = 0;
+    for (int cc = 0; cc < n_chunks; ++cc)
+      for (int dd = 0; dd < d; ++dd) base += chunk_rows[cc * W + dd];
+    for (int cc = 0; cc < c; ++cc) base += chunk_rows[cc * W + d];
+    s_base = base;
+    if (c == 0) {
+      int rows = 0, pairs = 0;
+      for (int cc = 0; cc < n_chunks; ++cc) {
+        rows += chunk_rows[cc * W + d];
+        pairs += chunk_pairs[cc * W + d];
+      }
+      send_counts[2 * d] = rows;
+      send_counts[2 * d + 1] = pairs;
+      if (d == 0) {  // the shared expert's single GEMM group: rows [0, T)
+        grp[0] = T;
+        grp[1] = 0;
+      }
+    }
+  }
+  const int t = c * kPlanChunk + threadIdx.x;
+  bool sel = false;
+  if (t < T) {
+    for (int k = 0; k < K; ++k) {
+      const int e = __ldg(ids + (int64_t)t * K + k);
+      sel |= (e >= 0 && e < N && e / El == d);
+    }
+  }
+  int total;
+  const int pos = block_scan_flag(sel, sums, &total);  // synchronises: s_base is visible
+  if (threadIdx.x == 0 && total != chunk_rows[c * W + d]) flag_status(status, kStatusBounds);
+  if (t >= T) return;
+  int32_t slot = -1;
+  if (sel) {
+    const int64_t s = s_base + pos;
+    if (s < send_cap) {
+      slot = (int32_t)s;
+      uint8_t* meta = send + s * row_bytes + meta_offset(H);
+      int32_t* lid = reinterpret_cast<int32_t*>(meta);
+      float* g = reinterpret_cast<float*>(meta) + K;
       for (int k = 0; k < K; ++k) {
         const int e = __ldg(ids + (int64_t)t * K + k);
-        if (e < 0 || e >= N) {
-          flag_status(status, kStatusBounds);
-          continue;
-        }
-        sel |= (e / El == d);
+        const bool here = e >= 0 && e < N && e / El == d;
+        lid[k] = here ? e - d * El : -1;
+        g[k] = here ? __ldg(gates + (int64_t)t * K + k) : 0.0f;
       }
-    }
-    int total;
-    const int pos = block_scan_flag(sel, sums, &total);
-    if (t < T) {
-      int32_t slot = -1;
-      if (sel) {
-        const int64_t s = (int64_t)before + running + pos;
-        if (s < send_cap) {
-          slot = (int32_t)s;
-          uint8_t* meta = send + s * row_bytes + meta_off;
-          int32_t* lid = reinterpret_cast<int32_t*>(meta);
-          float* g = reinterpret_cast<float*>(meta) + K;
-          for (int k = 0; k < K; ++k) {
-            const int e = __ldg(ids + (int64_t)t * K + k);
-            const bool here = e >= 0 && e < N && e / El == d;
-            lid[k] = here ? e - d * El : -1;
-            g[k] = here ? __ldg(gates + (int64_t)t * K + k) : 0.0f;
-          }
-        } else {
-          flag_status(status, kStatusBounds);
-        }
-      }
-      send_slot[(int64_t)t * W + d] = slot;
-    }
-    running += total;
-  }
-  if (threadIdx.x == 0) {
-    send_counts[2 * d] = rows_d;
-    send_counts[2 * d + 1] = pairs_d;
-    if (running != rows_d) flag_status(status, kStatusBounds);
-    if (d == 0) {  // the shared expert's single GEMM group: rows [0, T)
-      grp[0] = T;
-      grp[1] = 0;
+    } else {
+      flag_status(status, kStatusBounds);
     }
   }
+  send_slot[(int64_t)t * W + d] = slot;
 }
 
 // x -> 1x128 E4M3 codes and scales, written to the token's shared-expert row
@@ -474,8 +504,16 @@ int moe_ep_dispatch(moe_shape sh, int32_t W, const float* gate_w, const void* x,
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const int64_t rb = row_bytes_of(sh);
   int32_t* send_slot = at<int32_t>(ws, L.send_slot);
-  ep_plan_kernel<<<W, 1024, 0, s>>>(ids, gates, sh.T, sh.K, sh.N, W, sh.H, send, rb, send_cap,
-                                    send_slot, send_counts, at<int32_t>(ws, L.grp), status);
+  const int n_chunks = (sh.T + kPlanChunk - 1) / kPlanChunk;
+  int32_t* chunk_rows = at<int32_t>(ws, L.plan);
+  int32_t* chunk_pairs = chunk_rows + (size_t)n_chunks * W;
+  ep_count_kernel<<<n_chunks, kPlanChunk, 0, s>>>(ids, sh.T, sh.K, sh.N, W, chunk_rows,
+                                                  chunk_pairs, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  ep_slot_kernel<<<dim3(n_chunks, W), kPlanChunk, 0, s>>>(
+      ids, gates, sh.T, sh.K, sh.N, W, sh.H, n_chunks, chunk_rows, chunk_pairs, send, rb,
+      send_cap, send_slot, send_counts, at<int32_t>(ws, L.grp), status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const int64_t n_tiles = (int64_t)sh.T * (sh.H / kTile);

@@ -167,7 +167,7 @@ def _setup(w: I.Workload):
     return case, dw
 
 
-@pytest.mark.parametrize("W,Ts", [(2, [300, 171]), (2, [77, 0])])
+@pytest.mark.parametrize("W,Ts", [(2, [300, 171]), (2, [77, 0]), (2, [2500, 1025])])
 def test_ep_two_ranks(W, Ts):
     w = I.Workload("ep2", T=max(Ts), H=512, N=32, K=4, I=256, bias_range=0.1, seed=21)
     case, dw = _setup(w)
