@@ -678,7 +678,7 @@ def run_ep(args, w, rank, world, local_rank):
                 "config": dict(run_config(args, w, world),
                                parallelism=f"ep{world} (routed experts sharded over ranks; own "
                                            f"batch per GPU)"),
-                "gpu_launches": 16 * args.steps,
+                "gpu_launches": 17 * args.steps,
                 "e2e": {"value": w.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                         "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2,
                         "copies": "pinned host buffers, on the compute stream"},
