@@ -248,3 +248,50 @@ def test_expert_parallel_layer_one_rank_nccl():
         assert int(total.sum()) == 800
     finally:
         dist.destroy_process_group()
+
+
+def _dispatch_one(w, W, xb, dw, bias, send_cap=None, guard=0):
+    T = xb.shape[0]
+    sh = capi.shape_of(T, w.H, w.N, w.K, w.I)
+    rb = capi.moe_ep_row_bytes(sh)
+    cap = T * min(W, w.K) if send_cap is None else send_cap
+    send = torch.zeros(cap + guard, rb, dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(W, 2, dtype=torch.int32, device="cuda")
+    ws = torch.empty(capi.moe_ep_dispatch_workspace_size(sh, W), dtype=torch.uint8, device="cuda")
+    capi.moe_ep_dispatch(sh, W, dw.gate_w, H.x_to_device(xb), torch.from_numpy(bias).cuda(),
+                         send[:cap], sc, ws)
+    return sh, send, sc, ws
+
+
+def test_ep_wrong_pair_count_is_reported():
+    # a receiver told the wrong number of (row, slot) pairs reports MOE_ERR_BOUNDS
+    # through its status word; every index is checked before use, so no access
+    # leaves its buffer, and a call with the right count afterwards is clean
+    w = I.Workload("ep_err", T=200, H=256, N=32, K=4, I=128, bias_range=0.1, seed=25)
+    case, dw = _setup(w)
+    sh, send, sc, ws = _dispatch_one(w, 2, rank_x(w, 0, 200), dw, case.bias)
+    torch.cuda.synchronize()
+    assert capi.moe_get_status(ws) == 0
+    rows, pairs = sc.cpu().numpy()[0]
+    wl_t = ep.local_weights(dw.w13, dw.s13, dw.w2, dw.s2, w.N, 2, 0)
+    wl = capi.make_weights(dw.gate_w, *wl_t)
+    recv = send[:rows]
+    out = torch.empty(rows, w.H, dtype=torch.float32, device="cuda")
+    for p in (pairs - 1, pairs + 1, pairs):
+        ews = torch.empty(capi.moe_ep_expert_workspace_size(sh, 2, int(rows), int(p)),
+                          dtype=torch.uint8, device="cuda")
+        capi.moe_ep_experts(sh, 2, wl, recv, int(rows), int(p), out, ews)
+        assert capi.moe_get_status(ews) == (0 if p == pairs else -5)
+
+
+def test_ep_send_buffer_too_small_is_reported():
+    # rows beyond send_cap are dropped and flagged; the guard rows after the
+    # buffer stay untouched
+    w = I.Workload("ep_cap", T=200, H=256, N=32, K=4, I=128, bias_range=0.1, seed=26)
+    case, dw = _setup(w)
+    sh, send, sc, ws = _dispatch_one(w, 2, rank_x(w, 0, 200), dw, case.bias, send_cap=150,
+                                     guard=64)
+    torch.cuda.synchronize()
+    assert capi.moe_get_status(ws) == -5
+    assert int(sc.cpu()[:, 0].sum()) > 150     # the plan still counts every row
+    assert not send[150:].any().item()
