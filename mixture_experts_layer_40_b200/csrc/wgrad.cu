@@ -22,6 +22,16 @@ namespace moe {
 
 namespace {
 
+// 128-bit read-only load issued where it stands (the volatile asm keeps the
+// compiler from sinking it towards its first use).
+MOE_DEV float4 ldg_early4(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
 constexpr int kBM = 128, kBN = 256, kBK = 128;
 constexpr int kStages = 3;  // two stages' worth of smem goes to output staging
 constexpr int kABytes = kBM * kBK, kBBytes = kBN * kBK;
@@ -183,6 +193,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < kbn; ++kb, ++kbi) {
         const float inv_a = __fdividef(1.0f, ldg_early(sa_row + kb));
         const float4* binv = reinterpret_cast<const float4*>(p.b_inv + (int64_t)(kb0 + kb) * p.N + x0);
+        // the column scales of each 32-column group (the same addresses in every
+        // lane) are requested before that group's accumulator load, the first
+        // group's before the wait for the accumulator, so their latency overlaps
+        float4 b[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) b[q] = ldg_early4(binv + q);
         const int buf = kbi & 1;
         ok = __all_sync(0xffffffffu,
                         mbar_wait(smem_u32(&sh.tfull[buf]), (uint32_t)(kbi >> 1) & 1u, abort, p.status));
@@ -191,6 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t0 = lane_addr + (uint32_t)(buf * kBN + 128 * eg);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+          if (j > 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) b[q] = ldg_early4(binv + 8 * j + q);
+          }
           float v[32];
           tmem_ld32(t0 + 32 * j, v);
           tmem_wait_ld();
@@ -201,11 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 b = __ldg(binv + 8 * j + q);   // same address in every lane
-            acc[32 * j + 4 * q + 0] = fmaf(v[4 * q + 0], inv_a * b.x, acc[32 * j + 4 * q + 0]);
-            acc[32 * j + 4 * q + 1] = fmaf(v[4 * q + 1], inv_a * b.y, acc[32 * j + 4 * q + 1]);
-            acc[32 * j + 4 * q + 2] = fmaf(v[4 * q + 2], inv_a * b.z, acc[32 * j + 4 * q + 2]);
-            acc[32 * j + 4 * q + 3] = fmaf(v[4 * q + 3], inv_a * b.w, acc[32 * j + 4 * q + 3]);
+            acc[32 * j + 4 * q + 0] = fmaf(v[4 * q + 0], inv_a * b[q].x, acc[32 * j + 4 * q + 0]);
+            acc[32 * j + 4 * q + 1] = fmaf(v[4 * q + 1], inv_a * b[q].y, acc[32 * j + 4 * q + 1]);
+            acc[32 * j + 4 * q + 2] = fmaf(v[4 * q + 2], inv_a * b[q].z, acc[32 * j + 4 * q + 2]);
+            acc[32 * j + 4 * q + 3] = fmaf(v[4 * q + 3], inv_a * b[q].w, acc[32 * j + 4 * q + 3]);
           }
         }
       }
