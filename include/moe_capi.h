@@ -441,6 +441,49 @@ int moe_ep_combine(moe_shape sh, int32_t W, const float* ret, int64_t ret_rows, 
                    size_t ws_bytes, void* y, void* stream);
 
 /*
+ * Peer mode: the same steps without the two row all-to-alls and without any
+ * host synchronisation. The kernels move the rows themselves, with plain
+ * stores to the other ranks' buffers over NVLink/NVSwitch, so
+ * moving the data overlaps computing it. Every rank owns, in its own memory:
+ *   recv   uint8 [W * T_cap, row_bytes]  receive buffer: segment s (rows
+ *          s*T_cap ..) holds the rows source s sends to this rank;
+ *   counts int32 [W]  counts[s] = rows source s wrote into its segment;
+ *   ret    float [W * T_cap, H]  return buffer: segment d holds the partial
+ *          sums rank d sends back for this rank's rows.
+ * The calls take DEVICE arrays of W pointers to those buffers on every rank
+ * (peer_recv[d], peer_counts[d], peer_ret[s]), mapped into this process
+ * (CUDA IPC or symmetric memory); index `rank` is the caller's own. T_cap
+ * (>= every rank's T) is the same on all ranks. Order of a step, every rank:
+ *   moe_ep_dispatch_peer  (writes rows, ids, gates and its count into peers)
+ *   barrier               (e.g. a stream-ordered all-reduce of one int)
+ *   moe_ep_shared, moe_ep_experts_peer (writes partials into the sources)
+ *   barrier
+ *   moe_ep_combine_peer
+ * The kernels end their remote writes with a system-scope fence; the
+ * barriers order every rank's writes before any rank reads them, and the
+ * next step's writes after this step's reads. No kernel waits on another
+ * rank.
+ */
+size_t moe_ep_peer_expert_workspace_size(moe_shape sh, int32_t W, int32_t T_cap);
+
+int moe_ep_dispatch_peer(moe_shape sh, int32_t W, int32_t rank, int32_t T_cap,
+                         const float* gate_w, const void* x, const float* bias,
+                         int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
+                         uint8_t* const* peer_recv, int32_t* const* peer_counts,
+                         int32_t* send_counts_opt, void* ws, size_t ws_bytes, void* stream);
+
+/* recv, recv_counts: this rank's own buffers; peer_ret: device array [W] of
+ * the ranks' return buffers; ws: moe_ep_peer_expert_workspace_size bytes. */
+int moe_ep_experts_peer(moe_shape sh, int32_t W, int32_t rank, int32_t T_cap,
+                        const moe_weights* w_local, const uint8_t* recv,
+                        const int32_t* recv_counts, float* const* peer_ret, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* ret: this rank's own return buffer; ws: its dispatch workspace. */
+int moe_ep_combine_peer(moe_shape sh, int32_t W, int32_t T_cap, const float* ret, void* ws,
+                        size_t ws_bytes, void* y, void* stream);
+
+/*
  * Synchronises `stream`, reads and clears the device status word at the
  * start of `ws` (a forward workspace or a bare uint32 status word). Returns
  * MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_BOUNDS (timeout reported first), or

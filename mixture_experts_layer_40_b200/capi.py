@@ -83,6 +83,12 @@ SIGNATURES = {
     "moe_ep_experts": (ctypes.c_int, [moe_shape, _I32, ctypes.POINTER(moe_weights), _P, _I64,
                                       _I64, _P, _P, _SZ, _P]),
     "moe_ep_combine": (ctypes.c_int, [moe_shape, _I32, _P, _I64, _P, _SZ, _P, _P]),
+    "moe_ep_peer_expert_workspace_size": (_SZ, [moe_shape, _I32, _I32]),
+    "moe_ep_dispatch_peer": (ctypes.c_int, [moe_shape, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P,
+                                            _P, _P, _P, _P, _SZ, _P]),
+    "moe_ep_experts_peer": (ctypes.c_int, [moe_shape, _I32, _I32, _I32,
+                                           ctypes.POINTER(moe_weights), _P, _P, _P, _P, _SZ, _P]),
+    "moe_ep_combine_peer": (ctypes.c_int, [moe_shape, _I32, _I32, _P, _P, _SZ, _P, _P]),
     "moe_get_status": (ctypes.c_int, [_P, _P]),
     "moe_device_sm_count": (ctypes.c_int, []),
 }
@@ -303,6 +309,38 @@ def moe_ep_experts(sh: moe_shape, W: int, w_local: moe_weights, recv, R: int, pa
 def moe_ep_combine(sh: moe_shape, W: int, ret, ret_rows: int, ws, y, stream=None):
     _check("moe_ep_combine", LIB.moe_ep_combine(
         sh, W, _ptr(ret, torch.float32, "ret"), ret_rows, _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _ptr(y, torch.bfloat16, "y"), _stream(stream)))
+
+
+def moe_ep_peer_expert_workspace_size(sh: moe_shape, W: int, T_cap: int) -> int:
+    return int(LIB.moe_ep_peer_expert_workspace_size(sh, W, T_cap))
+
+
+def moe_ep_dispatch_peer(sh: moe_shape, W: int, rank: int, T_cap: int, gate_w, x, bias,
+                         peer_recv, peer_counts, ws, topk_ids=None, topk_gates=None, counts=None,
+                         send_counts=None, stream=None):
+    """peer_recv, peer_counts: int64 device tensors [W] of device pointers."""
+    _check("moe_ep_dispatch_peer", LIB.moe_ep_dispatch_peer(
+        sh, W, rank, T_cap, _ptr(gate_w, torch.float32, "gate_w"), _ptr(x, torch.bfloat16, "x"),
+        _ptr(bias, torch.float32, "bias"), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
+        _ptr(peer_recv, torch.int64, "peer_recv"), _ptr(peer_counts, torch.int64, "peer_counts"),
+        _ptr(send_counts, torch.int32, "send_counts"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)))
+
+
+def moe_ep_experts_peer(sh: moe_shape, W: int, rank: int, T_cap: int, w_local: moe_weights, recv,
+                        recv_counts, peer_ret, ws, stream=None):
+    """peer_ret: int64 device tensor [W] of device pointers."""
+    _check("moe_ep_experts_peer", LIB.moe_ep_experts_peer(
+        sh, W, rank, T_cap, ctypes.byref(w_local), _ptr(recv, torch.uint8, "recv"),
+        _ptr(recv_counts, torch.int32, "recv_counts"), _ptr(peer_ret, torch.int64, "peer_ret"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_ep_combine_peer(sh: moe_shape, W: int, T_cap: int, ret, ws, y, stream=None):
+    _check("moe_ep_combine_peer", LIB.moe_ep_combine_peer(
+        sh, W, T_cap, _ptr(ret, torch.float32, "ret"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _ptr(y, torch.bfloat16, "y"), _stream(stream)))
 
 

@@ -15,7 +15,7 @@ namespace moe {
 namespace {
 
 // One CTA of 1024 threads; N <= 1024. `pairs` is the number of (token, slot)
-// pairs the counts must add up to.
+// pairs the counts must add up to (negative: not checked).
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ counts, int N,
                                                     int T, int64_t pairs, int64_t routed_cap,
                                                     int32_t* __restrict__ offsets,
@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
     offsets[N] = total_c;
     group_rows[N] = T;
     row_start[N] = (int32_t)routed_cap;
-    if ((int64_t)total_c != pairs || (int64_t)total_p > routed_cap) {
+    if ((pairs >= 0 && (int64_t)total_c != pairs) || (int64_t)total_p > routed_cap) {
       flag_status(status, kStatusBounds);
     }
   }

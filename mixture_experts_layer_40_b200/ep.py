@@ -19,6 +19,12 @@ All arithmetic runs in the library's CUDA kernels; this module only sizes
 buffers and moves rows between ranks with torch.distributed (NCCL on GPUs).
 The row counts are read on the host once per step, because they size the
 exchanges.
+
+With peer=True the rows are not exchanged by all-to-alls: the dispatch and
+expert kernels store them straight into the other ranks' receive and return
+buffers (mapped into every process with CUDA IPC), and two stream-ordered
+all-reduces of one int act as the barriers. There is no host
+synchronisation in a step.
 """
 from __future__ import annotations
 
@@ -72,7 +78,8 @@ class ExpertParallelMoE:
 
     def __init__(self, T: int, H: int, N: int, K: int, I: int, W: int, rank: int,
                  gate_w: torch.Tensor, w13: torch.Tensor, s13: torch.Tensor, w2: torch.Tensor,
-                 s2: torch.Tensor, groups: int = 0, topk_groups: int = 0, group=None):
+                 s2: torch.Tensor, groups: int = 0, topk_groups: int = 0, group=None,
+                 peer: bool = False):
         self.T, self.H, self.N, self.K, self.I, self.W, self.rank = T, H, N, K, I, W, rank
         self.G, self.M = groups, topk_groups
         self.group = group
@@ -95,6 +102,36 @@ class ExpertParallelMoE:
         self.counts = torch.zeros(N, dtype=torch.int32, device=dev)
         self._ews = torch.empty(0, dtype=torch.uint8, device=dev)
         self.last = {}
+        self.peer = peer
+        if peer:
+            # every rank's receive buffer, its counts and its return buffer,
+            # T rows per source; other ranks' copies mapped into this process
+            self.recv = torch.zeros(W * T, self.row_bytes, dtype=torch.uint8, device=dev)
+            self.recv_counts = torch.zeros(W, dtype=torch.int32, device=dev)
+            self.ret = torch.zeros(W * T, H, dtype=torch.float32, device=dev)
+            ptrs = lambda views: torch.tensor([v.data_ptr() for v in views], dtype=torch.int64,
+                                              device=dev)
+            self._views = [self._peer_views(t) for t in (self.recv, self.recv_counts, self.ret)]
+            self.p_recv, self.p_counts, self.p_ret = (ptrs(v) for v in self._views)
+            self._ews = torch.empty(capi.moe_ep_peer_expert_workspace_size(sh, W, T),
+                                    dtype=torch.uint8, device=dev)
+            self._flag = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def _peer_views(self, t: torch.Tensor):
+        """t on every rank, as tensors of this process (CUDA IPC handles
+        gathered over the group; this rank's own entry is t itself)."""
+        if self.W == 1:
+            return [t]
+        from torch.multiprocessing.reductions import reduce_tensor
+        rebuild, args = reduce_tensor(t)
+        gathered = [None] * self.W
+        dist.all_gather_object(gathered, args, group=self.group)
+        return [t if r == self.rank else rebuild(*gathered[r]) for r in range(self.W)]
+
+    def _barrier(self):
+        """Every rank's kernels enqueued so far finish before any rank's
+        next kernel starts (a stream-ordered all-reduce of one int)."""
+        dist.all_reduce(self._flag, group=self.group)
 
     def _shape(self, T: int):
         return capi.shape_of(T, self.H, self.N, self.K, self.I, self.G, self.M)
@@ -114,6 +151,8 @@ class ExpertParallelMoE:
             raise ValueError(f"batch of {T} tokens exceeds the {self.T} this layer was sized for")
         sh = self._shape(T)
         c = capi
+        if self.peer:
+            return self._forward_peer(sh, x, bias)
         c.moe_ep_dispatch(sh, self.W, self.gate_w, x, bias, self.send, self.send_counts, self.ws,
                           topk_ids=self.ids[:T], topk_gates=self.gates[:T], counts=self.counts)
         recv_counts = exchange_counts(self.send_counts, self.group)
@@ -134,6 +173,22 @@ class ExpertParallelMoE:
         y = torch.empty(T, self.H, dtype=torch.bfloat16, device=self.device)
         c.moe_ep_combine(sh, self.W, ret, S, self.ws, y)
         self.last = {"send_rows": send_rows, "recv_rows": recv_rows, "pairs": pairs}
+        return y
+
+    def _forward_peer(self, sh, x, bias):
+        c = capi
+        T = x.shape[0]
+        c.moe_ep_dispatch_peer(sh, self.W, self.rank, self.T, self.gate_w, x, bias, self.p_recv,
+                               self.p_counts, self.ws, topk_ids=self.ids[:T],
+                               topk_gates=self.gates[:T], counts=self.counts,
+                               send_counts=self.send_counts)
+        self._barrier()          # every rank's rows are in place
+        c.moe_ep_shared(sh, self.W, self.w_local, self.ws)
+        c.moe_ep_experts_peer(sh, self.W, self.rank, self.T, self.w_local, self.recv,
+                              self.recv_counts, self.p_ret, self._ews)
+        self._barrier()          # every rank's partial sums are back
+        y = torch.empty(T, self.H, dtype=torch.bfloat16, device=self.device)
+        c.moe_ep_combine_peer(sh, self.W, self.T, self.ret, self.ws, y)
         return y
 
     def batch_counts(self) -> torch.Tensor:

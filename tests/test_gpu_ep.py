@@ -295,3 +295,94 @@ def test_ep_send_buffer_too_small_is_reported():
     assert capi.moe_get_status(ws) == -5
     assert int(sc.cpu()[:, 0].sum()) > 150     # the plan still counts every row
     assert not send[150:].any().item()
+
+
+def emulate_peer(w: I.Workload, W: int, T_cap: int, steps, dw, bias: np.ndarray, G=0, M=0):
+    """Steps of the peer mode over W emulated ranks on one GPU. Every rank's
+    receive, count and return buffers are ordinary allocations here and the
+    pointer arrays hold their addresses; the barriers of a real run are the
+    order of the calls (all dispatches, then all experts, then all combines).
+    Returns, per step, the list of per-rank outputs."""
+    N, K, Hd = w.N, w.K, w.H
+    bd = torch.from_numpy(bias).cuda()
+    wl_t = [ep.local_weights(dw.w13, dw.s13, dw.w2, dw.s2, N, W, r) for r in range(W)]
+    wl = [capi.make_weights(dw.gate_w, *t) for t in wl_t]
+    sh_cap = capi.shape_of(T_cap, Hd, N, K, w.I, G, M)
+    rb = capi.moe_ep_row_bytes(sh_cap)
+    recv = [torch.zeros(W * T_cap, rb, dtype=torch.uint8, device="cuda") for _ in range(W)]
+    cnt = [torch.full((W,), -3, dtype=torch.int32, device="cuda") for _ in range(W)]
+    ret = [torch.zeros(W * T_cap, Hd, dtype=torch.float32, device="cuda") for _ in range(W)]
+    ptrs = lambda ts: torch.tensor([t.data_ptr() for t in ts], dtype=torch.int64, device="cuda")
+    p_recv, p_cnt, p_ret = ptrs(recv), ptrs(cnt), ptrs(ret)
+    ws = [torch.empty(capi.moe_ep_dispatch_workspace_size(sh_cap, W), dtype=torch.uint8,
+                      device="cuda") for _ in range(W)]
+    ews = [torch.empty(capi.moe_ep_peer_expert_workspace_size(sh_cap, W, T_cap),
+                       dtype=torch.uint8, device="cuda") for _ in range(W)]
+    outs = []
+    for xs_bits in steps:
+        shs = [capi.shape_of(xb.shape[0], Hd, N, K, w.I, G, M) for xb in xs_bits]
+        for r, xb in enumerate(xs_bits):
+            T = xb.shape[0]
+            xd = H.x_to_device(xb) if T else torch.empty(0, Hd, dtype=torch.bfloat16, device="cuda")
+            capi.moe_ep_dispatch_peer(shs[r], W, r, T_cap, dw.gate_w, xd, bd, p_recv, p_cnt, ws[r])
+            capi.moe_ep_shared(shs[r], W, wl[r], ws[r])
+        for d in range(W):
+            capi.moe_ep_experts_peer(shs[d], W, d, T_cap, wl[d], recv[d], cnt[d], p_ret, ews[d])
+        ys = []
+        for s in range(W):
+            y = torch.empty(xs_bits[s].shape[0], Hd, dtype=torch.bfloat16, device="cuda")
+            capi.moe_ep_combine_peer(shs[s], W, T_cap, ret[s], ws[s], y)
+            ys.append(y)
+        torch.cuda.synchronize()
+        for r in range(W):
+            assert capi.moe_get_status(ws[r]) == 0 and capi.moe_get_status(ews[r]) == 0
+        outs.append(ys)
+    return outs
+
+
+@pytest.mark.parametrize("W,Ts,GM", [(2, [300, 171], (0, 0)), (4, [200, 1, 0, 129], (4, 2))])
+def test_ep_peer_mode_equals_all_to_all_mode(W, Ts, GM):
+    # the same rows, the same per-row sums and the same combine order: identical bits
+    w = I.Workload("ep_peer", T=max(Ts), H=256, N=16 * W, K=4, I=128, bias_range=0.1, seed=27)
+    case, dw = _setup(w)
+    xs = [rank_x(w, r, t) for r, t in enumerate(Ts)]
+    a2a = emulate(w, W, xs, dw, case.bias, G=GM[0], M=GM[1])
+    (peer,) = emulate_peer(w, W, max(Ts), [xs], dw, case.bias, G=GM[0], M=GM[1])
+    for st, y in zip(a2a, peer):
+        assert torch.equal(st["y"], y)
+
+
+def test_ep_peer_mode_second_step_reuses_the_buffers():
+    # step 2 sends different batches through the same buffers, rank 1 sending
+    # nothing (its count must read 0 everywhere, not step 1's)
+    w = I.Workload("ep_peer2", T=240, H=256, N=32, K=4, I=128, bias_range=0.1, seed=28)
+    case, dw = _setup(w)
+    step1 = [rank_x(w, 0, 240), rank_x(w, 1, 200)]
+    step2 = [rank_x(w, 5, 120), np.zeros((0, w.H), np.uint16)]
+    outs = emulate_peer(w, 2, 240, [step1, step2], dw, case.bias)
+    for step, ys in zip([step1, step2], outs):
+        ref = emulate(w, 2, step, dw, case.bias)
+        for st, y in zip(ref, ys):
+            assert torch.equal(st["y"], y)
+
+
+def test_expert_parallel_layer_peer_mode_one_rank_nccl():
+    import torch.distributed as dist
+    w = I.Workload("ep_nccl_peer", T=256, H=512, N=32, K=4, I=256, bias_range=0.1, seed=29)
+    case, dw = _setup(w)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1)
+    try:
+        loc = ep.local_weights(dw.w13, dw.s13, dw.w2, dw.s2, w.N, 1, 0)
+        a2a = ep.ExpertParallelMoE(w.T, w.H, w.N, w.K, w.I, 1, 0, dw.gate_w, *loc)
+        peer = ep.ExpertParallelMoE(w.T, w.H, w.N, w.K, w.I, 1, 0, dw.gate_w, *loc, peer=True)
+        bd = torch.from_numpy(case.bias).cuda()
+        for t in (200, 256, 17):
+            xd = H.x_to_device(rank_x(w, 0, t))
+            y_a = a2a.forward(xd, bd)
+            y_p = peer.forward(xd, bd)
+            torch.cuda.synchronize()
+            assert a2a.status() == 0 and peer.status() == 0
+            assert torch.equal(y_a, y_p)
+    finally:
+        dist.destroy_process_group()
