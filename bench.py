@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--ep", action="store_true",
                    help="expert parallelism: the routed experts sharded over the ranks "
                         "(ep.ExpertParallelMoE), every rank routing its own batch")
+    p.add_argument("--peer", action="store_true",
+                   help="with --ep: the kernels store rows straight into the other ranks' "
+                        "buffers (CUDA IPC), no all-to-alls and no host synchronisation")
     p.add_argument("--backward", action="store_true",
                    help="also time the FP8 expert backward (Dgrad + Wgrad) after the forward")
     p.add_argument("--seq-len", type=int, default=0,
@@ -619,7 +622,8 @@ def run_ep(args, w, rank, world, local_rank):
         del full
         torch.cuda.empty_cache()
         layer = ep.ExpertParallelMoE(w.T, w.H, w.N, w.K, w.I, world, rank, gw, *local,
-                                     groups=args.groups, topk_groups=args.topk_groups)
+                                     groups=args.groups, topk_groups=args.topk_groups,
+                                     peer=args.peer)
         x_bits = I.make_x(rank_batch(w, rank))
         x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
         x = x_host.to(dev)
@@ -666,9 +670,9 @@ def run_ep(args, w, rank, world, local_rank):
         barrier()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
         clk = clocks.stop() if clocks else None
-        last = layer.last
         rb = layer.row_bytes
-        send = int(sum(last["send_rows"]))
+        sc = layer.send_counts.cpu()
+        send = int(sc[:, 0].sum())
         if rank == 0:
             line = {
                 "metric": METRIC, "value": w.T * world / (ms_step * 1e-3), "unit": "tokens/s",
@@ -684,13 +688,19 @@ def run_ep(args, w, rank, world, local_rank):
                         "copies": "pinned host buffers, on the compute stream"},
                 "clocks": clk,
                 "ep": {"ranks": world, "experts_per_rank": w.N // world,
-                       "send_rows_rank0": last["send_rows"], "recv_rows_rank0": last["recv_rows"],
+                       "mode": "peer" if args.peer else "all-to-all",
+                       "send_rows_rank0": sc[:, 0].tolist(),
                        "dispatch_bytes_rank0": send * rb, "return_bytes_rank0": send * w.H * 4,
-                       "host_syncs_per_step": 1,
-                       "note": "library kernels: dispatch (router, plan, pack), shared expert, "
-                               "local experts, combine, bias update; exchanges: NCCL "
-                               "all-to-all of counts, rows and partial sums, all-reduce of "
-                               "counts"},
+                       "host_syncs_per_step": 0 if args.peer else 1,
+                       "note": ("library kernels: dispatch (router, plan, pack) storing rows "
+                                "into the ranks' receive buffers, shared expert, local experts "
+                                "storing partial sums into the sources' return buffers, "
+                                "combine, bias update; two all-reduce barriers and the count "
+                                "all-reduce" if args.peer else
+                                "library kernels: dispatch (router, plan, pack), shared expert, "
+                                "local experts, combine, bias update; exchanges: NCCL "
+                                "all-to-all of counts, rows and partial sums, all-reduce of "
+                                "counts")},
             }
             print(json.dumps(line), flush=True)
     finally:
