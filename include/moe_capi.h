@@ -1,7 +1,8 @@
 /*
  * moe_capi.h — C ABI of the B200 (sm_100a) DeepSeekMoE layer: the forward,
  * the bias controller, node-limited routing, the sequence-wise balance
- * statistics and the FP8 backward of the expert path.
+ * statistics, the FP8 backward of the expert path, and the layer with its
+ * routed experts sharded over several GPUs (expert parallelism).
  *
  * The layer (sources: "DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing,
  * Multi-Token Prediction, and FP8 Training at 671B Scale", trishampatil.com,
