@@ -66,8 +66,9 @@ typedef enum {
  * token, I intermediate size of every expert (routed and shared: the shared
  * expert has the routed experts' shape, "DeepSeek-V3, explained", step 3).
  * Supported: T >= 0 (T = 0 is an empty batch: the calls do no work, clear
- * the counts they output and accept NULL token-sized buffers); H a multiple of 256; I a multiple of 128; N a multiple
- * of 16 with 16 <= N <= 1024; 1 <= K <= min(N, 16).
+ * the counts they output and accept NULL token-sized buffers); H a multiple
+ * of 256; I a multiple of 128; N a multiple of 16 with 16 <= N <= 1024;
+ * 1 <= K <= min(N, 16).
  *
  * G, M: node-limited routing ("DeepSeek-V3, explained", recipe step 5;
  * "DeepSeek-V3 Technical Report" (deepforge.srivtx.xyz), "Balancing without
