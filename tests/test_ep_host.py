@@ -199,3 +199,31 @@ def test_ep_calls_reject_bad_arguments_on_the_host(capi):
     assert lib.moe_ep_shared(sh, 2, None, ctypes.c_void_p(addr), 256, null) == -6
     assert lib.moe_ep_combine(sh, 2, null, 0, ctypes.c_void_p(addr + 8), 1 << 40, null,
                               null) == -7
+
+
+def test_peer_mode_calls_reject_bad_arguments_on_the_host(capi):
+    import ctypes
+    lib = capi.LIB
+    sh = capi.shape_of(64, 256, 32, 4, 128)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(256)  # never dereferenced: every call below fails its checks first
+    # rank outside [0, W), T above T_cap, T_cap < 1, W not dividing N into >= 16 experts
+    for W, rank, T_cap in [(2, 2, 64), (2, -1, 64), (2, 0, 63), (2, 0, 0), (4, 0, 64)]:
+        assert lib.moe_ep_dispatch_peer(sh, W, rank, T_cap, null, null, null, null, null, null,
+                                        fake, fake, null, null, 0, null) == -1
+        assert lib.moe_ep_experts_peer(sh, W, rank, T_cap, None, null, fake, fake, null, 0,
+                                       null) == -1
+    assert lib.moe_ep_combine_peer(sh, 2, 63, null, null, 0, null, null) == -1
+    # missing pointer arrays
+    assert lib.moe_ep_dispatch_peer(sh, 2, 0, 64, null, null, null, null, null, null, null, fake,
+                                    null, null, 0, null) == -2
+    assert lib.moe_ep_experts_peer(sh, 2, 1, 64, None, null, null, fake, null, 0, null) == -2
+    assert lib.moe_ep_experts_peer(sh, 2, 1, 64, None, null, fake, null, null, 0, null) == -2
+    # workspace sizes: W T_cap rows of min(K, N/W) slots each, growing with T_cap
+    a = capi.moe_ep_peer_expert_workspace_size(sh, 2, 64)
+    b = capi.moe_ep_peer_expert_workspace_size(sh, 2, 128)
+    assert 0 < a < b
+    assert capi.moe_ep_peer_expert_workspace_size(sh, 2, 0) == 0
+    assert capi.moe_ep_peer_expert_workspace_size(sh, 3, 64) == 0
+    # the receiver's buffer for W T_cap rows holds at least its codes and the fp32 rows
+    assert a > 2 * 64 * 4 * (256 + 256 * 4)
