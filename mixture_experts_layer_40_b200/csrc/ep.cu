@@ -21,6 +21,16 @@
 //   combine  (source) : y_t = shared_t + sum over ranks (ascending) of the
 //                       returned partial sums, rounded once to bf16
 // Every slot and row is fixed by the data, so results do not depend on timing.
+//
+// Two ways to move the rows. All-to-all mode: dispatch fills a local send
+// buffer (destination-major) and the caller exchanges it, and later the
+// partial sums, with all-to-alls. Peer mode: dispatch stores each row straight
+// into its destination's receive buffer (one segment of T_cap rows per
+// source) and the reduction stores each partial sum straight into its
+// source's return buffer, through device pointers to the other ranks' memory;
+// the caller only places a barrier after each of the two phases. Both modes
+// use the same plan, the same packed rows and the same sums, so they give the
+// same bits.
 #include "block_scan.cuh"
 #include "kernels.cuh"
 
