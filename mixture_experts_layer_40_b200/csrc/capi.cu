@@ -2,6 +2,7 @@
 // workspace layout, tensor maps, and the launch sequence of the forward.
 #include <mutex>
 
+#include "host_util.h"
 #include "kernels.cuh"
 
 namespace moe {
@@ -40,20 +41,14 @@ int sm_count() {
   return cached[dev];
 }
 
-inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
-inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 
 void layout_of(const moe_shape& s, moe_ws_layout* L) {
   const int64_t T = s.T, H = s.H, N = s.N, K = s.K, I = s.I;
   L->routed_cap = round_up(T * K + N * (kTile - 1), kTile);
   L->rows_total = L->routed_cap + round_up(T, kTile);
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t at = off;
-    off = (size_t)round_up((int64_t)(off + bytes), 256);
-    return at;
-  };
+  Carver carve;
+  auto take = [&](size_t bytes) { return carve.take(bytes); };
   L->status = take(16);
   L->counts = take(N * 4);
   L->offsets = take((N + 1) * 4);
@@ -71,15 +66,9 @@ void layout_of(const moe_shape& s, moe_ws_layout* L) {
   L->y_rows = take((size_t)L->rows_total * H * 4);
   L->gate_split = take(router_split_bytes((int)N, (int)H));
   L->bal_scratch = take(balance_scratch_bytes(T, N));
-  L->total = off;
+  L->total = carve.off;
 }
 
-template <typename T>
-T* at(void* ws, size_t off) {
-  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
-}
-
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 }  // namespace
 
@@ -397,12 +386,8 @@ BackwardLayout backward_layout(const moe_shape& sh) {
   layout_of(sh, &L);
   const size_t R = (size_t)L.rows_total, H = sh.H, I = sh.I;
   BackwardLayout B{};
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t at = off;
-    off = (off + bytes + 255) / 256 * 256;
-    return at;
-  };
+  Carver carve;
+  auto take = [&](size_t bytes) { return carve.take(bytes); };
   B.dy_q = take(R * H);
   B.dy_s = take(R * (H / kTile) * 4);
   B.gu = take(R * 2 * I * 4);
@@ -418,7 +403,7 @@ BackwardLayout backward_layout(const moe_shape& sh) {
   B.dgut_s = take(2 * I * (R / kTile) * 4);
   B.xt_q = take(H * R);
   B.xt_inv = take((R / kTile) * H * 4);
-  B.total = off;
+  B.total = carve.off;
   return B;
 }
 

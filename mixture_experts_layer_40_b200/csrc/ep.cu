@@ -32,6 +32,7 @@
 // use the same plan, the same packed rows and the same sums, so they give the
 // same bits.
 #include "block_scan.cuh"
+#include "host_util.h"
 #include "kernels.cuh"
 
 namespace moe {
@@ -41,14 +42,6 @@ namespace {
 constexpr int kMaxRanks = 16;
 constexpr int kMaxK = 16;
 
-inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
-inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
-
-template <typename T>
-T* at(void* ws, size_t off) {
-  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
-}
 
 bool ep_ok(const moe_shape& sh, int W) {
   if (!shape_ok(sh) || W < 1 || W > kMaxRanks || sh.N % W != 0) return false;
@@ -74,12 +67,8 @@ SourceLayout source_layout(const moe_shape& sh, int W) {
   const int64_t T = sh.T, H = sh.H, N = sh.N, K = sh.K, I = sh.I;
   SourceLayout L{};
   L.rows = round_up(T, kTile);
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t a = off;
-    off = (size_t)round_up((int64_t)(off + bytes), 256);
-    return a;
-  };
+  Carver carve;
+  auto take = [&](size_t bytes) { return carve.take(bytes); };
   L.status = take(16);
   L.counts = take(N * 4);
   L.topk_ids = take((size_t)(T * K) * 4);
@@ -96,7 +85,7 @@ SourceLayout source_layout(const moe_shape& sh, int W) {
   L.h_q = take((size_t)(L.rows * I));
   L.h_s = take((size_t)(L.rows * (I / kTile)) * 4);
   L.y_shared = take((size_t)(L.rows * H) * 4);
-  L.total = off;
+  L.total = carve.off;
   return L;
 }
 
@@ -110,12 +99,8 @@ ExpertLayout expert_layout(const moe_shape& sh, int W, int64_t R, int64_t pairs)
   const int64_t El = sh.N / W, H = sh.H, K = sh.K, I = sh.I;
   ExpertLayout L{};
   L.routed_cap = round_up(pairs + El * (kTile - 1), kTile);
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t a = off;
-    off = (size_t)round_up((int64_t)(off + bytes), 256);
-    return a;
-  };
+  Carver carve;
+  auto take = [&](size_t bytes) { return carve.take(bytes); };
   L.status = take(16);
   L.counts = take(El * 4);
   L.offsets = take((El + 1) * 4);
@@ -130,7 +115,7 @@ ExpertLayout expert_layout(const moe_shape& sh, int W, int64_t R, int64_t pairs)
   L.h_q = take((size_t)L.routed_cap * I);
   L.h_s = take((size_t)L.routed_cap * (I / kTile) * 4);
   L.y_rows = take((size_t)L.routed_cap * H * 4);
-  L.total = off;
+  L.total = carve.off;
   return L;
 }
 

@@ -44,13 +44,6 @@ float* scratch_on_current_device() {
   return addr[dev];
 }
 
-int current_sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
-}
-
 }  // namespace
 }  // namespace moe
 
@@ -76,6 +69,6 @@ extern "C" int moe_route_noalloc(moe_shape sh, const float* gate_w, const void* 
   cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)sh.N * sizeof(int32_t), s);
   if (e == cudaSuccess)
     e = launch_router(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M, scratch, topk_ids,
-                      topk_gates, counts, nullptr, s, current_sm_count());
+                      topk_gates, counts, nullptr, s, moe_device_sm_count());
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
