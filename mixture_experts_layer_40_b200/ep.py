@@ -104,6 +104,13 @@ class ExpertParallelMoE:
         self.last = {}
         self.peer = peer
         if peer:
+            # the segments are T rows on every rank: a rank with another T would
+            # address the others' buffers with the wrong stride
+            if W > 1:
+                ts = [None] * W
+                dist.all_gather_object(ts, (T, H, N, K, I), group=group)
+                if any(t != ts[0] for t in ts):
+                    raise ValueError(f"peer mode needs the same (T, H, N, K, I) on every rank: {ts}")
             # every rank's receive buffer, its counts and its return buffer,
             # T rows per source; other ranks' copies mapped into this process
             self.recv = torch.zeros(W * T, self.row_bytes, dtype=torch.uint8, device=dev)
