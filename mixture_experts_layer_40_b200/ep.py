@@ -103,14 +103,15 @@ class ExpertParallelMoE:
         self._ews = torch.empty(0, dtype=torch.uint8, device=dev)
         self.last = {}
         self.peer = peer
+        if W > 1:
+            # the packed row layout needs the same H, N, K, I and routing groups
+            # on every rank; peer mode also needs the same T (its segment stride)
+            sizes = [None] * W
+            dist.all_gather_object(sizes, (T, H, N, K, I, groups, topk_groups), group=group)
+            first = 0 if peer else 1
+            if any(t[first:] != sizes[0][first:] for t in sizes):
+                raise ValueError(f"ranks were built with different sizes: {sizes}")
         if peer:
-            # the segments are T rows on every rank: a rank with another T would
-            # address the others' buffers with the wrong stride
-            if W > 1:
-                ts = [None] * W
-                dist.all_gather_object(ts, (T, H, N, K, I), group=group)
-                if any(t != ts[0] for t in ts):
-                    raise ValueError(f"peer mode needs the same (T, H, N, K, I) on every rank: {ts}")
             # every rank's receive buffer, its counts and its return buffer,
             # T rows per source; other ranks' copies mapped into this process
             self.recv = torch.zeros(W * T, self.row_bytes, dtype=torch.uint8, device=dev)
