@@ -58,6 +58,18 @@ def exchange_rows(send: torch.Tensor, send_rows: list[int], recv_rows: list[int]
     return recv, work
 
 
+def check_same_layout(sizes: tuple, W: int, peer: bool, group=None) -> None:
+    """sizes = (T, H, N, K, I, G, M) of this rank. The packed row layout needs
+    the same H, N, K, I and routing groups on every rank; peer mode also needs
+    the same T, the stride of every rank's buffer segments. Raises ValueError
+    on every rank otherwise (a collective: all ranks call it)."""
+    gathered = [None] * W
+    dist.all_gather_object(gathered, tuple(sizes), group=group)
+    first = 0 if peer else 1
+    if any(t[first:] != gathered[0][first:] for t in gathered):
+        raise ValueError(f"ranks were built with different sizes (T, H, N, K, I, G, M): {gathered}")
+
+
 def local_weights(w13: torch.Tensor, s13: torch.Tensor, w2: torch.Tensor, s2: torch.Tensor,
                   N: int, W: int, rank: int):
     """Rank `rank`'s weight sets out of the full [N+1, ...] tensors: its N/W
@@ -104,13 +116,7 @@ class ExpertParallelMoE:
         self.last = {}
         self.peer = peer
         if W > 1:
-            # the packed row layout needs the same H, N, K, I and routing groups
-            # on every rank; peer mode also needs the same T (its segment stride)
-            sizes = [None] * W
-            dist.all_gather_object(sizes, (T, H, N, K, I, groups, topk_groups), group=group)
-            first = 0 if peer else 1
-            if any(t[first:] != sizes[0][first:] for t in sizes):
-                raise ValueError(f"ranks were built with different sizes: {sizes}")
+            check_same_layout((T, H, N, K, I, groups, topk_groups), W, peer, group)
         if peer:
             # every rank's receive buffer, its counts and its return buffer,
             # T rows per source; other ranks' copies mapped into this process

@@ -227,3 +227,33 @@ def test_peer_mode_calls_reject_bad_arguments_on_the_host(capi):
     assert capi.moe_ep_peer_expert_workspace_size(sh, 3, 64) == 0
     # the receiver's buffer for W T_cap rows holds at least its codes and the fp32 rows
     assert a > 2 * 64 * 4 * (256 + 256 * 4)
+
+
+def _layout_main(rank, world, port, out_dir):
+    _init(rank, world, port)
+    try:
+        from mixture_experts_layer_40_b200 import ep
+        res = {}
+        T = 100 + rank  # different batch sizes: fine for all-to-all, not for peer mode
+        for name, sizes, peer in [("a2a_T", (T, 256, 32, 4, 128, 0, 0), False),
+                                  ("peer_T", (T, 256, 32, 4, 128, 0, 0), True),
+                                  ("a2a_K", (100, 256, 32, 4 + rank, 128, 0, 0), False),
+                                  ("peer_same", (100, 256, 32, 4, 128, 0, 0), True)]:
+            try:
+                ep.check_same_layout(sizes, world, peer)
+                res[name] = "ok"
+            except ValueError:
+                res[name] = "refused"
+        with open(os.path.join(out_dir, f"l{rank}.json"), "w") as fh:
+            json.dump(res, fh)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ranks_with_different_layouts_are_refused(tmp_path):
+    world = 2
+    mp.start_processes(_layout_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       start_method="spawn")
+    for r in range(world):
+        res = json.load(open(tmp_path / f"l{r}.json"))
+        assert res == {"a2a_T": "ok", "peer_T": "refused", "a2a_K": "refused", "peer_same": "ok"}
