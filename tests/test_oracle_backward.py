@@ -11,7 +11,6 @@ bit for bit, since the tile scale halves exactly), zero in -> zero out, and
 the FP8-versus-float64 error band.
 """
 import numpy as np
-import pytest
 
 from oracle import moe_oracle as O
 from mixture_experts_layer_40_b200 import inputs as I

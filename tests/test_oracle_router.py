@@ -12,7 +12,6 @@ import math
 from fractions import Fraction
 
 import numpy as np
-import pytest
 
 from oracle import moe_oracle as O
 from mixture_experts_layer_40_b200 import inputs as I

@@ -9,7 +9,6 @@ the second call is not disturbed by what the first left in the shared array,
 and that sizes beyond the array are refused before any work is queued. The
 file is named to run last, so a run that stops at its first failure has
 already run every other test."""
-import ctypes
 
 import numpy as np
 import pytest
