@@ -28,9 +28,10 @@ notes with its reason):
   * Top-K ties go to the lower expert id; output order is biased score
     descending.
   * Load target is the mean T*K/N, compared in integers as T*K - N*c_i.
-  * Expert FFN outputs stay at full precision; the layer output y is the
-    BF16 result. The combine sums in float64, shared expert first, then
-    routed experts by ascending id.
+  * Expert FFN outputs Y are BF16 (the FP8 GEMMs give BF16 outputs), each
+    rounded once from its float64 sum; the combine sums them in float64,
+    shared expert first, then routed experts by ascending id, and the layer
+    output y is that float64 sum (the kernels round it once more, to bf16).
   * No residual add; no routed scaling factor.
   * Node-limited routing ranks groups by the sum of their K/M highest
     *biased* scores (the selection side, as [Deepforge] ranks experts by
@@ -327,25 +328,50 @@ def silu(a: np.ndarray) -> np.ndarray:
     return a / (1.0 + np.exp(-a))
 
 
-def expert_ffn_q(xq: np.ndarray, xs: np.ndarray, wg_deq: np.ndarray,
-                 wu_deq: np.ndarray, wd_deq: np.ndarray):
-    """Quantisation-faithful expert FFN for a set of rows.
+def round_bf16(a: np.ndarray) -> np.ndarray:
+    """Round float64 values to bfloat16 (8 significant bits), half to even,
+    in one step from the exact value. Values are assumed inside the bf16
+    normal range (no overflow, no subnormals), as every expert output is."""
+    a = np.asarray(a, np.float64)
+    m, e = np.frexp(a)                      # a = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.round(m * 256.0) / 256.0, e)
 
-    xq/xs: 1x128 codes and scales of the rows' input. w*_deq: float64
-    dequantised weights, gate [I,H], up [I,H], down [H,I].
-    h = silu(x_hat W_gate^T) * (x_hat W_up^T) in float64, re-quantised 1x128
-    from its float32 rounding, then Y = h_hat W_down^T in float64. Y is not
-    rounded: the layer's BF16 output ([Dissection] section V, Figure 6) is y,
-    rounded once after the combine.
-    Returns (Y float64 [rows,H], hq uint8 [rows,I], hs float32 [rows,I/128]).
+
+def expert_up_q(xq: np.ndarray, xs: np.ndarray, wg_deq: np.ndarray, wu_deq: np.ndarray):
+    """Up/gate stage of the quantised expert FFN for a set of rows.
+
+    xq/xs: 1x128 codes and scales of the rows' input; wg_deq/wu_deq: float64
+    dequantised gate and up weights [I, H]. G = x_hat W_gate^T and
+    U = x_hat W_up^T in float64, h = silu(G) * U, then h is re-quantised 1x128
+    from its float32 rounding (the down GEMM takes E4M3 inputs,
+    [Dissection] section V, Figure 6).
+    Returns (h float64 [rows, I], hq uint8 [rows, I], hs float32 [rows, I/128]).
     """
     x_hat = dequantize_1x128(xq, xs)
     g = x_hat @ wg_deq.T
     u = x_hat @ wu_deq.T
     h = silu(g) * u
     hq, hs = quantize_1x128(h.astype(np.float32))
-    y = dequantize_1x128(hq, hs) @ wd_deq.T
-    return y, hq, hs
+    return h, hq, hs
+
+
+def expert_down_q(hq: np.ndarray, hs: np.ndarray, wd_deq: np.ndarray) -> np.ndarray:
+    """Down stage: Y = h_hat W_down^T summed in float64, not yet rounded.
+    hq/hs: 1x128 codes and scales of h; wd_deq: float64 [H, I]."""
+    return dequantize_1x128(hq, hs) @ wd_deq.T
+
+
+def expert_ffn_q(xq: np.ndarray, xs: np.ndarray, wg_deq: np.ndarray,
+                 wu_deq: np.ndarray, wd_deq: np.ndarray):
+    """Quantisation-faithful expert FFN for a set of rows: expert_up_q, then
+    expert_down_q, then the float64 sum rounded to bf16 (the FP8 GEMMs take
+    E4M3 inputs, accumulate in FP32 and give BF16 outputs, [Dissection]
+    section V, Figure 6).
+    Returns (Y float64 [rows, H] holding bf16 values, hq uint8 [rows, I],
+    hs float32 [rows, I/128]).
+    """
+    _, hq, hs = expert_up_q(xq, xs, wg_deq, wu_deq)
+    return round_bf16(expert_down_q(hq, hs, wd_deq)), hq, hs
 
 
 def expert_ffn_r(x: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray):

@@ -146,3 +146,173 @@ def test_token_subset_matches_full_run():
     np.testing.assert_allclose(sub["dgates"][toks], full["dgates"][toks], rtol=0,
                                atol=1e-12 * np.abs(full["dgates"]).max())
     assert sub["dw"] == {}
+
+
+# --------------------------------------------------------------------------
+# Lossless cases: every quantised operand sits on the E4M3 grid of its own
+# tile (tile amax 448 * 2^m, so the tile scale is a power of two, or every
+# element equal), so each FP8 GEMM must reproduce the float64 chain rule of
+# expert_ffn_backward_r (itself pinned by finite differences above) up to
+# float64 summation order; the same operands tiled along the other axis are
+# lossy, so an oracle that tiled an operand the wrong way fails.
+#
+# Structure (H = I = 128, one block per weight): W_gate = 1/4 in channel c0
+# of every row, so G = 64 everywhere for x = 256 (silu(64) = 64 and
+# silu'(64) = 1 exactly in float64); W_up = 2^-3 P_sigma and
+# W_down = 2^-2 P_pi (scaled permutations); so U = 32, h = 2048,
+# dh = 2^-2 dy permuted, dG = 32 dh and dU = 64 dh.
+# --------------------------------------------------------------------------
+
+def _lossless_weights(seed):
+    rng = np.random.default_rng(seed)
+    wg = np.zeros((128, 128), np.float32)
+    wg[:, 5] = 0.25
+    wu = np.zeros((128, 128), np.float32)
+    wu[np.arange(128), rng.permutation(128)] = 2.0 ** -3
+    wd = np.zeros((128, 128), np.float32)
+    wd[rng.permutation(128), np.arange(128)] = 2.0 ** -2
+    deq = []
+    for m in (wg, wu, wd):
+        d = O.dequantize_128x128(*O.quantize_128x128(m))
+        assert np.array_equal(d, m.astype(np.float64))      # lossless blocks
+        deq.append(d)
+    return deq
+
+
+def _grid_values(rng, shape):
+    """Random finite E4M3 values (both signs, subnormals included)."""
+    codes = rng.integers(0, 0x7F, shape).astype(np.uint8)
+    codes |= (rng.integers(0, 2, shape) << 7).astype(np.uint8)
+    return O.e4m3_decode(codes)
+
+
+def _on_grid(rows, cols, exps, axis, rng):
+    """Values whose tiles along `axis` (1: along a row, 0: down a column)
+    are lossless: grid values times 2^(m - 8), the tile's largest = 448 * 2^(m - 8)."""
+    v = _grid_values(rng, (rows, cols))
+    if axis == 1:
+        v[np.arange(rows), rng.integers(0, cols, rows)] = 448.0
+        v *= 2.0 ** (np.asarray(exps, np.float64)[:, None] - 8)
+    else:
+        v[rng.integers(0, rows, cols), np.arange(cols)] = 448.0
+        v *= 2.0 ** (np.asarray(exps, np.float64)[None, :] - 8)
+    return v.astype(np.float32)
+
+
+def _fp8_vs_chain_rule(x, dy, wg, wu, wd):
+    xq, xs = O.quantize_1x128(x)
+    q = O.expert_ffn_backward_q(xq, xs, x, dy, wg, wu, wd)
+    r = O.expert_ffn_backward_r(x, dy.astype(np.float64), wg, wu, wd)
+    return q, r
+
+
+def _close(a, b):
+    return np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(b))
+
+
+def test_dgrad_lossless_rows_equal_the_chain_rule():
+    """Dgrad quantises dy and dG/dU in 1x128 tiles along each row. Rows with
+    magnitudes 2^40 apart make 128x1 tiles lossy, 1x128 tiles exact."""
+    rng = np.random.default_rng(51)
+    wg, wu, wd = _lossless_weights(51)
+    x = np.full((8, 128), 256.0, np.float32)
+    dy = _on_grid(8, 128, [-20, -14, -8, -2, 4, 10, 16, 20], axis=1, rng=rng)
+    q, r = _fp8_vs_chain_rule(x, dy, wg, wu, wd)
+    assert np.array_equal(q["dh"], dy.astype(np.float64) @ wd)
+    assert _close(q["dx"], r["dx"])
+    # the same dy in 128x1 tiles loses the small rows
+    wrong = O.dequantize_128x1(*O.quantize_128x1(dy), 8)
+    assert not _close(wrong, dy.astype(np.float64))
+
+
+def test_wgrad_lossless_columns_equal_the_chain_rule():
+    """Wgrad quantises dy and h in 128x1 tiles down each column for
+    dW_down = Q(dy)^T . Q(h). Columns of dy with magnitudes up to 2^40 apart
+    are exact in 128x1 tiles and lossy in 1x128 tiles. (dW_gate and dW_up
+    take dG/dU from the Dgrad's row-quantised dy, which these columns make
+    lossy; they are pinned by the next tests.)"""
+    rng = np.random.default_rng(52)
+    wg, wu, wd = _lossless_weights(52)
+    x = np.full((128, 128), 256.0, np.float32)
+    dy = _on_grid(128, 128, rng.integers(-20, 21, 128), axis=0, rng=rng)
+    q, r = _fp8_vs_chain_rule(x, dy, wg, wu, wd)
+    assert _close(q["dwd"], r["dwd"])
+    wrong = O.dequantize_1x128(*O.quantize_1x128(dy))
+    assert not _close(wrong, dy.astype(np.float64))
+
+
+def test_wgrad_down_uses_h_quantised_down_its_columns():
+    """dW_down = Q(dy)^T . Q(h) with h in 128x1 tiles. A dy that selects one
+    row per output channel (a power of two, lossless) makes dW_down expose
+    the quantised h row by row; it must equal the page's per-tile rule
+    ("DeepSeek-V3 Technical Report" (deepforge), "Per-tile FP8 scaling")
+    applied to each column of h, computed here from float64 products.
+    Skipping h's quantisation, or tiling it along the rows, fails."""
+    from tests.test_oracle_codec import _page_rounding_rule
+    rng = np.random.default_rng(53)
+    rows, h_dim, i_dim = 128, 256, 128
+    x = I.bf16_bits_to_f32(I.f32_to_bf16_bits(rng.standard_normal((rows, h_dim)).astype(np.float32)))
+    x *= np.float32(2.0) ** rng.integers(-3, 4, (rows, 1)).astype(np.float32)
+    wg = O.dequantize_128x128(*O.quantize_128x128(
+        (rng.standard_normal((i_dim, h_dim)) / 16).astype(np.float32)))
+    wu = O.dequantize_128x128(*O.quantize_128x128(
+        (rng.standard_normal((i_dim, h_dim)) / 16).astype(np.float32)))
+    wd = O.dequantize_128x128(*O.quantize_128x128(
+        (rng.standard_normal((h_dim, i_dim)) / 11).astype(np.float32)))
+    pick = rng.integers(0, rows, h_dim)
+    dy = np.zeros((rows, h_dim), np.float32)
+    dy[pick, np.arange(h_dim)] = 2.0 ** -5
+    xq, xs = O.quantize_1x128(x)
+    q = O.expert_ffn_backward_q(xq, xs, x, dy, wg, wu, wd)
+    # h from the forward's dequantised x, then the page's rule down each column
+    x_hat = O.dequantize_1x128(xq, xs)
+    h = (O.silu(x_hat @ wg.T) * (x_hat @ wu.T)).astype(np.float32)
+    h_hat = np.empty(h.shape)
+    for c in range(i_dim):
+        scale = np.float32(448.0) / np.max(np.abs(h[:, c]))
+        prod = (h[:, c] * scale).astype(np.float32).astype(np.float64)
+        h_hat[:, c] = _page_rounding_rule(prod) / np.float64(scale)
+    assert np.max(np.abs(h_hat - h)) > 1e-3 * np.max(np.abs(h))
+    assert np.array_equal(q["dwd"], 2.0 ** -5 * h_hat[pick])
+
+
+def test_wgrad_up_uses_x_quantised_down_its_columns():
+    """dW_up = Q(dU)^T . Q(x) and dW_gate = Q(dG)^T . Q(x), with x and dG/dU
+    in 128x1 tiles. With the lossless weights and x = 256 in channel c0
+    (the largest of every row, so G = 64 exactly) but Gaussian elsewhere, a
+    dy that selects one row per channel (a power of two) makes dU = 64 dh a
+    power-of-two selector (lossless), so dW_up exposes the column-quantised
+    x row by row: it must equal the page's per-tile rule applied to each
+    column of x. dG = dh U holds one Gaussian value per column (lossless up
+    to the float32 tile scale), so dW_gate = dG^T x_hat to 1e-6; tiling
+    dG or x along the rows instead fails."""
+    from tests.test_oracle_codec import _page_rounding_rule
+    rng = np.random.default_rng(54)
+    wg, wu, wd = _lossless_weights(54)
+    rows = 128
+    x = I.bf16_bits_to_f32(I.f32_to_bf16_bits(
+        (rng.standard_normal((rows, 128)) * 10.0 ** rng.uniform(-1, 1, (1, 128))).astype(np.float32)))
+    x[:, 5] = 256.0
+    assert np.all(np.abs(np.delete(x, 5, axis=1)) < 256.0)
+    pick = rng.integers(0, rows, 128)
+    dy = np.zeros((rows, 128), np.float32)
+    dy[pick, np.arange(128)] = 2.0 ** -3
+    xq, xs = O.quantize_1x128(x)
+    q = O.expert_ffn_backward_q(xq, xs, x, dy, wg, wu, wd)
+    x_col = np.empty(x.shape)
+    for c in range(128):
+        scale = np.float32(448.0) / np.max(np.abs(x[:, c]))
+        prod = (x[:, c] * scale).astype(np.float32).astype(np.float64)
+        x_col[:, c] = _page_rounding_rule(prod) / np.float64(scale)
+    assert np.max(np.abs(x_col - x)) > 1e-3 * np.max(np.abs(x))
+    # dU[r, i] = 64 * dh[r, i] = 64 * 2^-2 * dy[r, perm(i)]: one entry per column
+    du = q["d_u"]
+    row_of = np.argmax(np.abs(du), axis=0)
+    assert np.count_nonzero(du) == 128
+    assert np.array_equal(q["dwu"], du[row_of, np.arange(128)][:, None] * x_col[row_of])
+    dg = q["d_g"]
+    assert np.count_nonzero(dg) == 128
+    ref = dg[row_of, np.arange(128)][:, None] * x_col[row_of]
+    assert np.max(np.abs(q["dwg"] - ref)) <= 1e-6 * np.max(np.abs(ref))
+    wrong = O.dequantize_1x128(*O.quantize_1x128(x))
+    assert np.max(np.abs(wrong - x_col)) > 1e-3 * np.max(np.abs(x))

@@ -217,3 +217,20 @@ def test_block_quantiser_block_amax():
     assert s2[0, 1] * 8 == s[0, 1]
     assert np.array_equal(np.delete(s2, 1, axis=1), np.delete(s, 1, axis=1))
 
+
+
+def test_round_bf16_against_torch_and_ties():
+    """bf16 rounding of the expert outputs: torch's float -> bfloat16 cast on
+    values exactly representable in float32 (so torch rounds once), the
+    even significand on exact midpoints, and one rounding from the exact
+    float64 value (no double rounding through float32)."""
+    rng = np.random.default_rng(30)
+    v = (rng.standard_normal(50_000) * 10 ** rng.uniform(-6, 6, 50_000)).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.round_bf16(v.astype(np.float64)), ref)
+    assert O.round_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 1.0
+    assert O.round_bf16(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 1.0 + 2.0 ** -6
+    assert O.round_bf16(np.array([-(1.0 + 3 * 2.0 ** -8)]))[0] == -(1.0 + 2.0 ** -6)
+    # just above a midpoint rounds up even where float32 would land on it
+    assert O.round_bf16(np.array([1.0 + 2.0 ** -8 + 2.0 ** -40]))[0] == 1.0 + 2.0 ** -7
+    assert O.round_bf16(np.array([0.0]))[0] == 0.0

@@ -8,10 +8,14 @@ The sparse layer must equal the dense "run every expert, then mask" layer:
 the masked terms are exact zeros, so the two differ only by the summation
 order inside the float64 library matmuls (a few ulps).
 """
+import math
+
 import numpy as np
+import torch
 
 from oracle import moe_oracle as O
 from mixture_experts_layer_40_b200 import inputs as I
+from tests.test_oracle_codec import _page_rounding_rule
 
 
 def _tiny_all():
@@ -75,7 +79,72 @@ def test_quantised_ffn_uses_dequantised_operands():
     h = O.silu(xh @ dg.T) * (xh @ du.T)
     hq2, hs2 = O.quantize_1x128(h.astype(np.float32))
     assert np.array_equal(hq, hq2) and np.array_equal(hs, hs2)
-    assert np.allclose(y, O.dequantize_1x128(hq, hs) @ dd.T, rtol=1e-14, atol=0)
+    # bf16 outputs ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing...",
+    # section V, Figure 6): 8 significant bits, within half a step of the
+    # float64 sum, and torch's own bf16 cast of that sum (values exactly
+    # representable in float32 are compared, so torch rounds once)
+    y64 = O.dequantize_1x128(hq, hs) @ dd.T
+    assert np.all(np.abs(y - y64) <= 2.0 ** -8 * np.abs(y64))
+    y32 = y64.astype(np.float32)
+    exact = y32.astype(np.float64) == y64
+    ref = torch.from_numpy(y32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(y[exact], ref[exact])
+    assert np.mean(y != y64) > 0.9
+
+
+def _brute_h(x_hat, wg, wu):
+    """h = silu(x_hat . wg) * (x_hat . wu) with plain Python sums."""
+    rows, h_dim = x_hat.shape
+    out = np.empty((rows, wg.shape[0]))
+    for t in range(rows):
+        for j in range(wg.shape[0]):
+            gj = sum(float(x_hat[t, c]) * float(wg[j, c]) for c in range(h_dim))
+            uj = sum(float(x_hat[t, c]) * float(wu[j, c]) for c in range(h_dim))
+            out[t, j] = gj / (1.0 + math.exp(-gj)) * uj
+    return out
+
+
+def _page_tile_1x128(h):
+    """The per-tile rule of "DeepSeek-V3 Technical Report" (deepforge),
+    "Per-tile FP8 scaling", applied to rows of h in tiles of 128 channels:
+    scale = 448 / amax (float32), X_fp8 = round(X * scale) with the page's
+    E4M3 rounding, X_hat = X_fp8 / scale."""
+    h32 = np.asarray(h, np.float32)
+    out = np.empty(h32.shape)
+    for t in range(h32.shape[0]):
+        for c in range(0, h32.shape[1], 128):
+            tile = h32[t, c:c + 128]
+            scale = np.float32(448.0) / np.max(np.abs(tile))
+            prod = (tile * scale).astype(np.float32).astype(np.float64)
+            out[t, c:c + 128] = _page_rounding_rule(prod) / np.float64(scale)
+    return out
+
+
+def test_h_requantisation_seen_through_identity_down_weights():
+    """With W_down = 2^-3 times the identity (H = I = 128: one 128x128 block,
+    quantised losslessly: amax 2^-3, every diagonal code 448), Y = 2^-3 h_hat
+    before its bf16 rounding, so the oracle's down stage exposes the 1x128
+    re-quantised h element by element. It must equal the page's per-tile rule
+    applied to h computed by plain loops; an oracle that skipped the
+    re-quantisation of h, or tiled it another way, fails here."""
+    rng = np.random.default_rng(23)
+    x = rng.standard_normal((2, 128)).astype(np.float32)
+    wg = (rng.standard_normal((128, 128)) / 11).astype(np.float32)
+    wu = (rng.standard_normal((128, 128)) / 11).astype(np.float32)
+    wd = (np.eye(128) * 2.0 ** -3).astype(np.float32)
+    xq, xs = O.quantize_1x128(x)
+    dg = O.dequantize_128x128(*O.quantize_128x128(wg))
+    du = O.dequantize_128x128(*O.quantize_128x128(wu))
+    dd = O.dequantize_128x128(*O.quantize_128x128(wd))
+    assert np.array_equal(dd, wd.astype(np.float64))          # lossless block
+    h = _brute_h(O.dequantize_1x128(xq, xs), dg, du)
+    h_hat = _page_tile_1x128(h)
+    assert np.max(np.abs(h_hat - h)) > 1e-3 * np.max(np.abs(h))  # quantisation is visible
+    _, hq, hs = O.expert_up_q(xq, xs, dg, du)
+    y64 = O.expert_down_q(hq, hs, dd)
+    assert np.array_equal(y64, 2.0 ** -3 * h_hat)
+    y, _, _ = O.expert_ffn_q(xq, xs, dg, du, dd)
+    assert np.array_equal(y, O.round_bf16(2.0 ** -3 * h_hat))
 
 
 def test_sparse_equals_dense_then_mask():
