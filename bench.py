@@ -3,6 +3,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3_prefill]
                     [--impl ours|reference] [--no-cpu-baseline]
 
+With --gpus N > 1 and no rank environment (RANK / WORLD_SIZE), bench.py
+starts the N ranks itself under torchrun on 127.0.0.1.
+
 One step = one pass of the whole hot path on one batch of synthetic input:
 quantise x, route, permute, up/gate GEMM + SwiGLU + re-quantisation, down
 GEMM, combine, and the aux-loss-free bias update. With N > 1 ranks (torchrun,
@@ -58,6 +61,8 @@ def parse():
                         "buffers (CUDA IPC), no all-to-alls and no host synchronisation")
     p.add_argument("--backward", action="store_true",
                    help="also time the FP8 expert backward (Dgrad + Wgrad) after the forward")
+    p.add_argument("--launch-check", action="store_true",
+                   help="start the ranks, exchange one value, print n_gpus; no kernels")
     p.add_argument("--seq-len", type=int, default=0,
                    help="sequence length for the balance statistics (0: the whole batch)")
     return p.parse_args()
@@ -155,7 +160,10 @@ def algorithmic_work(w, counts: np.ndarray):
 
 GEMM_SOURCES = ["mixture_experts_layer_40_b200/csrc/gemm.cu",
                 "mixture_experts_layer_40_b200/csrc/common.cuh"]
-TRAFFIC_FILE = "profiles/grouped_gemm_v3_prefill_dram.md"
+# one line per recorded capture: "traffic <kernel> bytes=<B> workload=<name>
+# fingerprint=<gemm sources> [key=value ...]"; the summary beside it says how
+# each figure was taken
+TRAFFIC_FILE = "profiles/grouped_gemm_traffic.txt"
 
 
 def gemm_fingerprint() -> str:
@@ -181,8 +189,8 @@ def recorded_traffic(kernel: str, workload: str):
         return None
     for ln in lines:
         f = ln.split()
-        if len(f) == 5 and f[0] == "traffic" and f[1] == kernel:
-            kv = dict(x.split("=", 1) for x in f[2:])
+        if len(f) >= 5 and f[0] == "traffic" and f[1] == kernel:
+            kv = dict(x.split("=", 1) for x in f[2:] if "=" in x)
             if kv.get("workload") == workload and kv.get("fingerprint") == fp:
                 return int(kv["bytes"])
     return None
@@ -275,8 +283,19 @@ def oracle_setup(w, x_bits):
     from oracle import moe_oracle as O
     pool = I.make_weight_pool(w)
     ew = O.ExpertWeights(pool.pool13, pool.pool2, pool.slot_gate, pool.slot_up, pool.slot_down)
+    # the quantised and dequantised block pools are built once, untimed (the
+    # first dequantised() call builds the pool every expert is assembled from)
     ew.quantised_pools()
+    ew.dequantised(0)
     return I.bf16_bits_to_f32(x_bits), I.make_gate_w(w), I.make_bias(w), ew
+
+
+def oracle_sample_text(w, steps: int) -> str:
+    return (f"{steps} steps, each extrapolated from a sample: quantisation, routing, "
+            f"permutation and combine of 512 of the {w.T} tokens (scaled by T/512), 1 of the "
+            f"{w.N} routed experts on its sampled tokens (weight assembly + FFN, scaled by "
+            f"T/512 and N) and the shared expert on 64 tokens (scaled to T); block pools "
+            f"built before timing")
 
 
 # ---------------------------------------------------------------- ranks
@@ -333,9 +352,7 @@ def run_reference(args, w, rank):
              for s in range(args.steps)]
     ms = 1e3 * float(np.mean(times))
     value = w.T / (ms * 1e-3)
-    sample = (f"per step: quantisation, routing, permutation and combine of 512 of the {w.T} "
-              f"tokens, 1 of {w.N} routed experts on its sampled tokens and the shared expert on 64; "
-              f"scaled to all tokens and experts")
+    sample = oracle_sample_text(w, args.steps)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -573,14 +590,13 @@ def run_ours(args, w, rank, world, local_rank):
     }
     if world == 1 and not args.no_cpu_baseline:
         x32, gw, b0, ew = oracle_setup(w, x_bits)
-        t = [oracle_sample_step(w, x32, gw, b0, ew, s, node_limit=(args.groups, args.topk_groups))
-             for s in range(2)]
+        nl = (args.groups, args.topk_groups)
+        oracle_sample_step(w, x32, gw, b0, ew, 0, node_limit=nl)      # warm-up, untimed
+        t = [oracle_sample_step(w, x32, gw, b0, ew, 1 + s, node_limit=nl) for s in range(3)]
         v = w.T / float(np.mean(t))
         line["cpu_baseline"] = {
             "value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"2 steps; each: quantisation, routing, permutation and combine of 512 of "
-                      f"the {w.T} tokens, 1 of {w.N} routed experts on its sampled tokens and the "
-                      f"shared expert on 64, scaled to all tokens and experts"}
+            "sample": "after 1 untimed step, " + oracle_sample_text(w, 3)}
     print(json.dumps(line), flush=True)
 
 
@@ -707,15 +723,64 @@ def run_ep(args, w, rank, world, local_rank):
             dist.destroy_process_group()
 
 
+def launch_ranks(n: int) -> None:
+    """Re-runs this command as n ranks under torchrun (one process per GPU,
+    rendezvous on 127.0.0.1), bounded by an outer timeout well above the
+    process group's own; called when --gpus n > 1 and no rank environment
+    is set. Does not return."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run",
+           "--nnodes=1", f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    sys.stdout.flush()
+    os.execvp(cmd[0], cmd)
+
+
+def launch_check(world: int, rank: int) -> None:
+    """--launch-check: the rank plumbing alone (no kernels): every rank joins
+    the process group (gloo without a GPU), the ranks sum one int and take
+    the max of their times as the bench does, and rank 0 prints n_gpus."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if world > 1:
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        one = torch.ones(1, dtype=torch.int64)
+        if backend == "nccl":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+            one = one.cuda()
+        ranks = int(batch_counts(one, world).item())
+        t = torch.tensor([float(rank)], dtype=torch.float64, device=one.device)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        if rank == 0:
+            print(json.dumps({"launch_check": True, "n_gpus": world, "ranks_counted": ranks,
+                              "max_rank": float(t.item()), "backend": backend}), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
 def main():
     args = parse()
     from mixture_experts_layer_40_b200 import inputs as I
     w = I.WORKLOADS[args.workload]
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.impl == "ours":
+        launch_ranks(args.gpus)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, w, rank)
+        return
+    if args.launch_check:
+        launch_check(world, rank)
         return
     if world > 1:
         import datetime

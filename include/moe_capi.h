@@ -131,10 +131,12 @@ typedef struct {
   size_t a_s;           /* float [rows_total, H/128] */
   size_t h_q;           /* E4M3 [rows_total, I]: SwiGLU output, 1x128 re-quantised */
   size_t h_s;           /* float [rows_total, I/128] */
-  size_t y_rows;        /* float [rows_total, H]: expert outputs before the combine */
+  size_t y_rows;        /* bf16 [rows_total, H]: expert outputs before the combine */
   size_t gate_split;    /* bf16 [3, N, H]: the fp32 centroids as three bf16 terms */
   size_t bal_scratch;   /* moe_balance_stats scratch: float [T] token sums, then
                            float and int32 [T + ceil(T/128), N] chunk partials */
+  size_t perm_scratch;  /* int32 [ceil(T/128), N]: the permutation's per-chunk
+                           expert counts, then first rows */
   size_t total;         /* workspace bytes required */
 } moe_ws_layout;
 
@@ -187,15 +189,21 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
  * own pool and does not let plug-in libraries allocate, or a latency-critical
  * loop where a cudaMalloc (which may synchronise the device) is not allowed.
  *
- * Same work and outputs as moe_route (same kernels), but the T x N gate
- * logits live in a fixed array inside the library's device memory: 4 MiB,
+ * The same routing as moe_route, with two differences. The gate logits come
+ * from an fp32 SIMT kernel rather than moe_route's split-bf16 tensor-core
+ * kernel: both are fp32-accurate, so the ids, counts and gates agree with
+ * moe_route's except on tokens whose K-th and (K+1)-th biased scores are
+ * within about 1e-5 relative (near ties), and the gates within about 1e-6.
+ * And the T x N gate logits live in a fixed array inside the library's
+ * device memory: 4 MiB,
  * MOE_ROUTE_NOALLOC_MAX_LOGITS floats, present on every GPU that loads the
  * library until the process exits. Nothing is allocated; the caller passes
  * only inputs and outputs, as for moe_route. Returns MOE_ERR_WORKSPACE, before
  * enqueuing anything, when T * N exceeds MOE_ROUTE_NOALLOC_MAX_LOGITS.
  *
- * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress, no allocation); the first call on a device also
+ * loads the library's kernels there, so make it before any stream capture.
  * Every call uses the same array: calls whose work overlaps on the GPU (other
  * streams, other host threads on the same device) race on it, so the caller
  * must serialise them. The logits are fully rewritten by each call and
@@ -243,7 +251,7 @@ size_t moe_backward_workspace_size(moe_shape sh);
  *   dX rows    = dG . W_gate + dU . W_up per expert (FP8 grouped GEMM on w13t)
  *   dx[t]      = the sum of the token's K + 1 row gradients (shared first,
  *                then slots by ascending expert id), rounded once to bf16
- *   dgates[t,k] = dy[t] . Y_k[t] with the forward's fp32 expert output row
+ *   dgates[t,k] = dy[t] . Y_k[t] with the forward's bf16 expert output row
  *   dw2 [N+1, H, I] = per expert, dY^T . h over its rows (Wgrad), fp32
  *   dw13 [N+1, 2I, H] = per expert, [dG | dU]^T . x over its rows, in w13's
  *                row order (gate block c, then up block c), fp32
@@ -256,7 +264,7 @@ size_t moe_backward_workspace_size(moe_shape sh);
  *   (only read for the weight gradients; may be NULL without them)
  *   dy, dx: bf16 [T, H], 16-byte aligned; dgates: float [T, K]
  *   dw13, dw2: the weight gradients, or both NULL to skip them
- *   ws: the forward's workspace (its expert output rows are overwritten);
+ *   ws: the forward's workspace (read only, apart from its status word);
  *   bws: moe_backward_workspace_size(sh) bytes, 256-byte aligned.
  * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE; device
  * checks in ws's status word (moe_get_status).
@@ -345,9 +353,15 @@ int moe_update_bias(float* bias, const int32_t* counts, int32_t N, int32_t T, in
  *   h = silu(G) * U, h re-quantised 1x128.
  *   a_q [rows, H] E4M3, a_s [rows, H/128]; w13/s13 as in moe_weights with
  *   n_groups sets; h_q [rows, I] E4M3, h_s [rows, I/128].
- * moe_expert_down: per group, Y = h_hat W_down^T in fp32 (the expert outputs
- *   stay at accumulation precision until the combine rounds y once to bf16).
- *   h_q/h_s as above; w2/s2 as in moe_weights; y_rows float [rows, H].
+ * moe_expert_down: per group, Y = h_hat W_down^T, written as the fp32
+ *   totals (the accumulator before any output rounding; the backward's
+ *   GEMMs use this form). h_q/h_s as above; w2/s2 as in moe_weights;
+ *   y_rows float [rows, H].
+ * moe_expert_down_bf16: the same GEMM as the layer runs it, each fp32 total
+ *   rounded once to bf16 (round to nearest even): the FP8 GEMMs give BF16
+ *   outputs ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing, ...",
+ *   section V, Figure 6). Bit for bit the bf16 rounding of moe_expert_down's
+ *   output. y_rows bf16 [rows, H].
  * Rows outside every segment are not written.
  */
 int moe_expert_up(int32_t H, int32_t I, int32_t n_groups, const int32_t* group_rows,
@@ -359,6 +373,11 @@ int moe_expert_down(int32_t H, int32_t I, int32_t n_groups, const int32_t* group
                     const int32_t* group_start, int64_t rows, const uint8_t* h_q,
                     const float* h_s, const uint8_t* w2, const float* s2, void* y_rows,
                     uint32_t* status_ws, void* stream);
+
+int moe_expert_down_bf16(int32_t H, int32_t I, int32_t n_groups, const int32_t* group_rows,
+                         const int32_t* group_start, int64_t rows, const uint8_t* h_q,
+                         const float* h_s, const uint8_t* w2, const float* s2, void* y_rows,
+                         uint32_t* status_ws, void* stream);
 
 /*
  * Expert parallelism ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing,

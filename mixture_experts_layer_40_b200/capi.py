@@ -41,7 +41,7 @@ class moe_weights(ctypes.Structure):
 
 _LAYOUT_FIELDS = ["status", "counts", "offsets", "group_rows", "row_start", "row_token",
                   "token_row", "topk_ids", "topk_gates", "logits", "a_q", "a_s", "h_q", "h_s",
-                  "y_rows", "gate_split", "bal_scratch", "total"]
+                  "y_rows", "gate_split", "bal_scratch", "perm_scratch", "total"]
 
 
 class moe_ws_layout(ctypes.Structure):
@@ -74,6 +74,8 @@ SIGNATURES = {
     "moe_update_bias": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _F32, _P]),
     "moe_expert_up": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_down": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_expert_down_bf16": (ctypes.c_int, [_I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P, _P,
+                                            _P]),
     "moe_ep_row_bytes": (_I64, [moe_shape]),
     "moe_ep_dispatch_workspace_size": (_SZ, [moe_shape, _I32]),
     "moe_ep_dispatch": (ctypes.c_int, [moe_shape, _I32, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P,
@@ -266,6 +268,14 @@ def moe_expert_down(H, I, n_groups, group_rows, group_start, rows, h_q, h_s, w2,
         H, I, n_groups, _ptr(group_rows, torch.int32), _ptr(group_start, torch.int32), rows,
         _ptr(h_q, torch.uint8), _ptr(h_s, torch.float32), _ptr(w2, torch.uint8),
         _ptr(s2, torch.float32), _ptr(y_rows, torch.float32), _ptr(status), _stream(stream)))
+
+
+def moe_expert_down_bf16(H, I, n_groups, group_rows, group_start, rows, h_q, h_s, w2, s2, y_rows,
+                         status, stream=None):
+    _check("moe_expert_down_bf16", LIB.moe_expert_down_bf16(
+        H, I, n_groups, _ptr(group_rows, torch.int32), _ptr(group_start, torch.int32), rows,
+        _ptr(h_q, torch.uint8), _ptr(h_s, torch.float32), _ptr(w2, torch.uint8),
+        _ptr(s2, torch.float32), _ptr(y_rows, torch.bfloat16), _ptr(status), _stream(stream)))
 
 
 def moe_ep_row_bytes(sh: moe_shape) -> int:

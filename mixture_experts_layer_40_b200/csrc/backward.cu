@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(256) swiglu_backward_kernel(
 // One warp per (token, slot): dgates[t, k] = dy[t] . Y[token_row[t, k]] in fp32
 // (lane-strided partial sums, then a fixed butterfly).
 __global__ void __launch_bounds__(256) gate_grad_kernel(const __nv_bfloat16* __restrict__ dy,
-                                                        const float* __restrict__ y_rows,
+                                                        const __nv_bfloat16* __restrict__ y_rows,
                                                         const int32_t* __restrict__ token_row,
                                                         int T, int H, int K, int64_t routed_cap,
                                                         float* __restrict__ dgates,
@@ -182,15 +182,15 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const __nv_bfloat16* __r
       continue;
     }
     const uint2* d2 = reinterpret_cast<const uint2*>(dy + t * H);
-    const float4* y4 = reinterpret_cast<const float4*>(y_rows + r * H);
+    const uint2* y2 = reinterpret_cast<const uint2*>(y_rows + r * H);
     float acc = 0.0f;
     for (int i = lane; i < H / 4; i += 32) {
       const uint2 d = __ldg(d2 + i);
-      const float4 yv = __ldg(y4 + i);
-      acc = fmaf(bf16_lo(d.x), yv.x, acc);
-      acc = fmaf(bf16_hi(d.x), yv.y, acc);
-      acc = fmaf(bf16_lo(d.y), yv.z, acc);
-      acc = fmaf(bf16_hi(d.y), yv.w, acc);
+      const uint2 yv = __ldg(y2 + i);
+      acc = fmaf(bf16_lo(d.x), bf16_lo(yv.x), acc);
+      acc = fmaf(bf16_hi(d.x), bf16_hi(yv.x), acc);
+      acc = fmaf(bf16_lo(d.y), bf16_lo(yv.y), acc);
+      acc = fmaf(bf16_hi(d.y), bf16_hi(yv.y), acc);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -334,7 +334,7 @@ cudaError_t launch_swiglu_backward(const float* gu, const float* dh, int64_t row
   return cudaGetLastError();
 }
 
-cudaError_t launch_gate_grad(const void* dy, const float* y_rows, const int32_t* token_row, int T,
+cudaError_t launch_gate_grad(const void* dy, const __nv_bfloat16* y_rows, const int32_t* token_row, int T,
                              int H, int K, int64_t routed_cap, float* dgates, uint32_t* status,
                              cudaStream_t stream, int sm_count) {
   const int64_t pairs = (int64_t)T * K;

@@ -63,9 +63,10 @@ void layout_of(const moe_shape& s, moe_ws_layout* L) {
   L->a_s = take((size_t)L->rows_total * (H / kTile) * 4);
   L->h_q = take((size_t)L->rows_total * I);
   L->h_s = take((size_t)L->rows_total * (I / kTile) * 4);
-  L->y_rows = take((size_t)L->rows_total * H * 4);
+  L->y_rows = take((size_t)L->rows_total * H * 2);
   L->gate_split = take(router_split_bytes((int)N, (int)H));
   L->bal_scratch = take(balance_scratch_bytes(T, N));
+  L->perm_scratch = take(permute_scratch_bytes(T, (int)N));
   L->total = carve.off;
 }
 
@@ -187,6 +188,7 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
   layout_of(sh, &L);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  NvtxRange range("moe_route");
   uint32_t* status = at<uint32_t>(ws, L.status);
   cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
@@ -248,8 +250,17 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   uint8_t* a_q = at<uint8_t>(ws, L.a_q);
   float* a_s = at<float>(ws, L.a_s);
 
-  // optional stage events: recorded before each of the 6 stages and at the end
+  // optional stage events: recorded before each of the 6 stages and at the
+  // end; an NVTX range per stage in any case
+  static const char* const kStageNames[MOE_TRACE_EVENTS - 1] = {
+      "moe_forward/route", "moe_forward/permute", "moe_forward/quantize",
+      "moe_forward/expert_up", "moe_forward/expert_down", "moe_forward/combine"};
+  NvtxRange whole("moe_forward");
+  bool in_range = false;
   auto mark = [&](int i, cudaError_t e) {
+    if (in_range) nvtxRangePop();
+    in_range = i < MOE_TRACE_EVENTS - 1;
+    if (in_range) nvtxRangePushA(kStageNames[i]);
     if (events != nullptr && e == cudaSuccess)
       return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
     return e;
@@ -266,9 +277,10 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   // a6-a7: offsets, stable expert-major scatter of the (token, slot) pairs
   if (e == cudaSuccess)
     e = launch_permute(ids, counts, sh.T, sh.N, sh.K, (int64_t)sh.T * sh.K, L.routed_cap,
-                       at<int32_t>(ws, L.offsets),
+                       at<int32_t>(ws, L.perm_scratch), at<int32_t>(ws, L.offsets),
                        at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
-                       at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.token_row), status, s);
+                       at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.token_row), status, s,
+                       sms);
   e = mark(2, e);
   // a1 (+ a7's row copies): x -> 1x128 codes and scales, written to the
   // token's shared-expert row and its K routed rows
@@ -285,12 +297,12 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   e = mark(4, e);
   // a9: down GEMM -> bf16 expert outputs
   if (e == cudaSuccess)
-    e = launch_expert_down(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w->w2, w->s2,
-                           at<float>(ws, L.y_rows), s, sms);
+    e = launch_expert_down_bf16(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w->w2, w->s2,
+                                at<__nv_bfloat16>(ws, L.y_rows), s, sms);
   e = mark(5, e);
   // a10: weighted combine with the shared expert
   if (e == cudaSuccess)
-    e = launch_combine(at<float>(ws, L.y_rows), ids, gates, at<int32_t>(ws, L.token_row),
+    e = launch_combine(at<__nv_bfloat16>(ws, L.y_rows), ids, gates, at<int32_t>(ws, L.token_row),
                        sh.T, sh.H, sh.K, L.routed_cap, L.rows_total,
                        static_cast<__nv_bfloat16*>(y), status, s);
   e = mark(6, e);
@@ -357,6 +369,20 @@ int moe_expert_down(int32_t H, int32_t I, int32_t n_groups, const int32_t* group
                                         static_cast<cudaStream_t>(stream), sm_count()));
 }
 
+int moe_expert_down_bf16(int32_t H, int32_t I, int32_t n_groups, const int32_t* group_rows,
+                         const int32_t* group_start, int64_t rows, const uint8_t* h_q,
+                         const float* h_s, const uint8_t* w2, const float* s2, void* y_rows,
+                         uint32_t* status_ws, void* stream) {
+  const int r = expert_args_ok(H, I, n_groups, group_rows, group_start, rows);
+  if (r != MOE_OK) return r;
+  if (!h_q || !h_s || !w2 || !s2 || !y_rows) return MOE_ERR_NULL;
+  if (!aligned(h_q, 16) || !aligned(w2, 16) || !aligned(y_rows, 16)) return MOE_ERR_ALIGN;
+  GroupedGemm gg{H, I, n_groups, group_rows, group_start, rows, status_ws};
+  return cuda_status(launch_expert_down_bf16(gg, h_q, h_s, w2, s2,
+                                             static_cast<__nv_bfloat16*>(y_rows),
+                                             static_cast<cudaStream_t>(stream), sm_count()));
+}
+
 int moe_transpose_weights(moe_shape sh, const moe_weights* w, uint8_t* w13t, float* s13t,
                           uint8_t* w2t, float* s2t, void* stream) {
   if (!shape_ok(sh)) return MOE_ERR_SHAPE;
@@ -375,7 +401,7 @@ namespace moe {
 namespace {
 
 struct BackwardLayout {
-  size_t dy_q, dy_s, gu, dh, dgu_q, dgu_s;
+  size_t dy_q, dy_s, gu, dh, dgu_q, dgu_s, dx_rows;
   // weight gradients: row gates and the column-tile operands
   size_t row_gate, dyt_q, dyt_s, ht_q, ht_inv, dgut_q, dgut_s, xt_q, xt_inv;
   size_t total;
@@ -394,6 +420,7 @@ BackwardLayout backward_layout(const moe_shape& sh) {
   B.dh = take(R * I * 4);
   B.dgu_q = take(R * 2 * I);
   B.dgu_s = take(R * (2 * I / kTile) * 4);
+  B.dx_rows = take(R * H * 4);
   B.row_gate = take(R * 4);
   B.dyt_q = take(H * R);
   B.dyt_s = take(H * (R / kTile) * 4);
@@ -439,11 +466,12 @@ int moe_backward(moe_shape sh, const moe_weights* w, const moe_weights* wt,
       !aligned(wt->w2, 16))
     return MOE_ERR_ALIGN;
   const int sms = sm_count();
+  NvtxRange range("moe_backward");
   const int32_t* token_row = at<int32_t>(ws, L.token_row);
-  float* y_rows = at<float>(ws, L.y_rows);
+  const __nv_bfloat16* y_rows = at<__nv_bfloat16>(ws, L.y_rows);
+  float* dx_rows = at<float>(bws, B.dx_rows);
   cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
-  // gate gradients from the forward's fp32 expert output rows (before the
-  // rows buffer is reused for the input gradients)
+  // gate gradients from the forward's bf16 expert output rows
   if (e == cudaSuccess)
     e = launch_gate_grad(dy, y_rows, token_row, sh.T, sh.H, sh.K, L.routed_cap, dgates, status, s,
                          sms);
@@ -478,11 +506,11 @@ int moe_backward(moe_shape sh, const moe_weights* w, const moe_weights* wt,
   if (e == cudaSuccess) {
     GroupedGemm gg{sh.H, 2 * sh.I, sh.N + 1, gr, gs, L.rows_total, status};
     e = launch_expert_down(gg, at<uint8_t>(bws, B.dgu_q), at<float>(bws, B.dgu_s), wt->w13,
-                           wt->s13, y_rows, s, sms);
+                           wt->s13, dx_rows, s, sms);
   }
   // dx[t] = the token's K + 1 row gradients, fixed order, one bf16 rounding
   if (e == cudaSuccess)
-    e = launch_combine(y_rows, topk_ids, nullptr, token_row, sh.T, sh.H, sh.K, L.routed_cap,
+    e = launch_combine(dx_rows, topk_ids, nullptr, token_row, sh.T, sh.H, sh.K, L.routed_cap,
                        L.rows_total, static_cast<__nv_bfloat16*>(dx), status, s);
   if (!wgrad || e != cudaSuccess) return cuda_status(e);
   // Wgrad: operands in column tiles (128 rows x 1 channel), transposed

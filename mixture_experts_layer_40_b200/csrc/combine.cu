@@ -16,7 +16,20 @@ namespace {
 
 constexpr int kMaxK = 16;
 
-__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ y_rows,
+// 8 consecutive row elements as fp32
+MOE_DEV void load8(const __nv_bfloat16* p, int64_t c, float (&v)[8]) {
+  const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p) + c);
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+  v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+}
+MOE_DEV void load8(const float* p, int64_t c, float (&v)[8]) {
+  const float4 a = __ldcs(reinterpret_cast<const float4*>(p) + 2 * c);
+  const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 2 * c + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+template <typename Row>
+__global__ void __launch_bounds__(128) combine_kernel(const Row* __restrict__ y_rows,
                                                       const int32_t* __restrict__ ids,
                                                       const float* __restrict__ gates,
                                                       const int32_t* __restrict__ token_row,
@@ -58,16 +71,15 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   const int n = s_n;
   const int64_t shared_row = routed_cap + t;
   if (shared_row >= rows_total) return;
-  const float4* ys = reinterpret_cast<const float4*>(y_rows + shared_row * H);
+  const Row* ys = y_rows + shared_row * H;
   uint4* out = reinterpret_cast<uint4*>(y + (int64_t)t * H);
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
-    const float4 v0 = __ldcs(ys + 2 * c), v1 = __ldcs(ys + 2 * c + 1);
-    float acc[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float acc[8];
+    load8(ys, c, acc);
     for (int k = 0; k < n; ++k) {
-      const float4* yk = reinterpret_cast<const float4*>(y_rows + s_row[k] * H);
-      const float4 u0 = __ldcs(yk + 2 * c), u1 = __ldcs(yk + 2 * c + 1);
+      float f[8];
+      load8(y_rows + s_row[k] * H, c, f);
       const float g = s_gate[k];
-      const float f[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, f[i], acc[i]);
     }
@@ -89,16 +101,30 @@ __global__ void update_bias_kernel(float* __restrict__ bias, const int32_t* __re
   bias[i] = __fadd_rn(bias[i], step);
 }
 
+template <typename Row>
+cudaError_t combine(const Row* y_rows, const int32_t* ids, const float* gates,
+                    const int32_t* token_row, int T, int H, int K, int64_t routed_cap,
+                    int64_t rows_total, __nv_bfloat16* y, uint32_t* status, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  combine_kernel<Row><<<T, 128, 0, stream>>>(y_rows, ids, gates, token_row, T, H, K, routed_cap,
+                                             rows_total, y, status);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_combine(const __nv_bfloat16* y_rows, const int32_t* ids, const float* gates,
+                           const int32_t* token_row, int T, int H, int K, int64_t routed_cap,
+                           int64_t rows_total, __nv_bfloat16* y, uint32_t* status,
+                           cudaStream_t stream) {
+  return combine(y_rows, ids, gates, token_row, T, H, K, routed_cap, rows_total, y, status, stream);
+}
 
 cudaError_t launch_combine(const float* y_rows, const int32_t* ids, const float* gates,
                            const int32_t* token_row, int T, int H, int K, int64_t routed_cap,
                            int64_t rows_total, __nv_bfloat16* y, uint32_t* status,
                            cudaStream_t stream) {
-  if (T == 0) return cudaSuccess;
-  combine_kernel<<<T, 128, 0, stream>>>(y_rows, ids, gates, token_row, T, H, K, routed_cap,
-                                        rows_total, y, status);
-  return cudaGetLastError();
+  return combine(y_rows, ids, gates, token_row, T, H, K, routed_cap, rows_total, y, status, stream);
 }
 
 cudaError_t launch_update_bias(float* bias, const int32_t* counts, int N, int T, int K,

@@ -13,11 +13,11 @@
 //                       token ascending, one row per (token, rank) that holds
 //                       one of its experts), quantise x 1x128 once into the
 //                       send rows and into its shared-expert GEMM rows
-//   shared   (source) : the shared expert on its own tokens, fp32 rows
+//   shared   (source) : the shared expert on its own tokens, bf16 rows
 //   experts  (dest)   : received rows -> expert-major GEMM rows of its local
-//                       experts -> grouped FP8 up/down GEMMs -> per received
-//                       row, the gate-weighted sum over its local experts
-//                       (fp32, ascending expert id)
+//                       experts -> grouped FP8 up/down GEMMs (bf16 expert
+//                       outputs) -> per received row, the gate-weighted sum
+//                       over its local experts (fp32, ascending expert id)
 //   combine  (source) : y_t = shared_t + sum over ranks (ascending) of the
 //                       returned partial sums, rounded once to bf16
 // Every slot and row is fixed by the data, so results do not depend on timing.
@@ -84,7 +84,7 @@ SourceLayout source_layout(const moe_shape& sh, int W) {
   L.a_s = take((size_t)(L.rows * (H / kTile)) * 4);
   L.h_q = take((size_t)(L.rows * I));
   L.h_s = take((size_t)(L.rows * (I / kTile)) * 4);
-  L.y_shared = take((size_t)(L.rows * H) * 4);
+  L.y_shared = take((size_t)(L.rows * H) * 2);
   L.total = carve.off;
   return L;
 }
@@ -92,7 +92,7 @@ SourceLayout source_layout(const moe_shape& sh, int W) {
 struct ExpertLayout {
   int64_t routed_cap;
   size_t status, counts, offsets, group_rows, row_start, ids, gates, token_row, row_token;
-  size_t a_q, a_s, h_q, h_s, y_rows, total;
+  size_t a_q, a_s, h_q, h_s, y_rows, perm_scratch, total;
 };
 
 ExpertLayout expert_layout(const moe_shape& sh, int W, int64_t R, int64_t pairs) {
@@ -114,7 +114,8 @@ ExpertLayout expert_layout(const moe_shape& sh, int W, int64_t R, int64_t pairs)
   L.a_s = take((size_t)L.routed_cap * (H / kTile) * 4);
   L.h_q = take((size_t)L.routed_cap * I);
   L.h_s = take((size_t)L.routed_cap * (I / kTile) * 4);
-  L.y_rows = take((size_t)L.routed_cap * H * 4);
+  L.y_rows = take((size_t)L.routed_cap * H * 2);
+  L.perm_scratch = take(permute_scratch_bytes(R, (int)El));
   L.total = carve.off;
   return L;
 }
@@ -404,7 +405,7 @@ __global__ void __launch_bounds__(256) ep_gather_rows_kernel(
 // return buffer: row j = s seg_rows + i goes to peer_ret[s] at row
 // rank * seg_rows + i; rows without a slot are not written.
 __global__ void __launch_bounds__(128) ep_reduce_kernel(
-    const float* __restrict__ y_rows, const int32_t* __restrict__ ids,
+    const __nv_bfloat16* __restrict__ y_rows, const int32_t* __restrict__ ids,
     const float* __restrict__ gates, const int32_t* __restrict__ token_row, int H, int K,
     int64_t routed_cap, float* __restrict__ out, float* const* peer_ret, int rank,
     int64_t seg_rows, uint32_t* __restrict__ status) {
@@ -449,12 +450,12 @@ __global__ void __launch_bounds__(128) ep_reduce_kernel(
   for (int c = threadIdx.x; c < H / 4; c += blockDim.x) {
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     for (int k = 0; k < n; ++k) {
-      const float4 u = __ldcs(reinterpret_cast<const float4*>(y_rows + s_row[k] * H) + c);
+      const uint2 u = __ldcs(reinterpret_cast<const uint2*>(y_rows + s_row[k] * H) + c);
       const float g = s_gate[k];
-      acc.x = fmaf(g, u.x, acc.x);
-      acc.y = fmaf(g, u.y, acc.y);
-      acc.z = fmaf(g, u.z, acc.z);
-      acc.w = fmaf(g, u.w, acc.w);
+      acc.x = fmaf(g, bf16_lo(u.x), acc.x);
+      acc.y = fmaf(g, bf16_hi(u.x), acc.y);
+      acc.z = fmaf(g, bf16_lo(u.y), acc.z);
+      acc.w = fmaf(g, bf16_hi(u.y), acc.w);
     }
     o[c] = acc;
   }
@@ -466,7 +467,7 @@ __global__ void __launch_bounds__(128) ep_reduce_kernel(
 // ret[dest_off[d] + l] (all-to-all mode) or ret[d seg_rows + l] (peer mode,
 // seg_rows > 0).
 __global__ void __launch_bounds__(128) ep_combine_kernel(
-    const float* __restrict__ y_shared, const float* __restrict__ ret,
+    const __nv_bfloat16* __restrict__ y_shared, const float* __restrict__ ret,
     const int32_t* __restrict__ send_slot, const int32_t* __restrict__ dest_off, int H, int W,
     int64_t ret_rows, int64_t seg_rows, __nv_bfloat16* __restrict__ y,
     uint32_t* __restrict__ status) {
@@ -489,11 +490,12 @@ __global__ void __launch_bounds__(128) ep_combine_kernel(
   }
   __syncthreads();
   const int n = s_n;
-  const float4* ys = reinterpret_cast<const float4*>(y_shared + t * H);
+  const uint4* ys = reinterpret_cast<const uint4*>(y_shared + t * H);
   uint4* out = reinterpret_cast<uint4*>(y + t * H);
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
-    const float4 v0 = __ldcs(ys + 2 * c), v1 = __ldcs(ys + 2 * c + 1);
-    float acc[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const uint4 v = __ldcs(ys + c);
+    float acc[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                    bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
     for (int i = 0; i < n; ++i) {
       const float4* p = reinterpret_cast<const float4*>(ret + s_slot[i] * H);
       const float4 u0 = __ldcs(p + 2 * c), u1 = __ldcs(p + 2 * c + 1);
@@ -616,9 +618,9 @@ int experts_impl(const moe_shape& sh, int W, const moe_weights* w_local, const u
   e = cudaGetLastError();
   if (e == cudaSuccess)
     e = launch_permute(ids, counts, (int)R, El, sh.K, pairs, L.routed_cap,
-                       at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.group_rows),
-                       at<int32_t>(ws, L.row_start), at<int32_t>(ws, L.row_token), token_row,
-                       status, s);
+                       at<int32_t>(ws, L.perm_scratch), at<int32_t>(ws, L.offsets),
+                       at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
+                       at<int32_t>(ws, L.row_token), token_row, status, s, sms);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const int64_t n_tiles = R * (sh.H / kTile);
   ep_gather_rows_kernel<<<tile_grid(n_tiles), 256, 0, s>>>(recv, R, sh.H, sh.K, rb, token_row,
@@ -631,10 +633,10 @@ int experts_impl(const moe_shape& sh, int W, const moe_weights* w_local, const u
     e = launch_expert_up(gg, at<uint8_t>(ws, L.a_q), at<float>(ws, L.a_s), w_local->w13,
                          w_local->s13, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), s, sms);
   if (e == cudaSuccess)
-    e = launch_expert_down(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w_local->w2,
-                           w_local->s2, at<float>(ws, L.y_rows), s, sms);
+    e = launch_expert_down_bf16(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w_local->w2,
+                                w_local->s2, at<__nv_bfloat16>(ws, L.y_rows), s, sms);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  ep_reduce_kernel<<<(unsigned)R, 128, 0, s>>>(at<float>(ws, L.y_rows), ids, gates, token_row,
+  ep_reduce_kernel<<<(unsigned)R, 128, 0, s>>>(at<__nv_bfloat16>(ws, L.y_rows), ids, gates, token_row,
                                                sh.H, sh.K, L.routed_cap, out, peer_ret, rank,
                                                seg_rows, status);
   return cuda_status(cudaGetLastError());
@@ -650,7 +652,7 @@ int combine_impl(const moe_shape& sh, int W, const float* ret, int64_t ret_rows,
   if (!y || (ret_rows > 0 && !ret)) return MOE_ERR_NULL;
   if (!aligned(y, 16) || !aligned(ret, 16)) return MOE_ERR_ALIGN;
   ep_combine_kernel<<<(unsigned)sh.T, 128, 0, s>>>(
-      at<float>(ws, L.y_shared), ret, at<int32_t>(ws, L.send_slot), at<int32_t>(ws, L.dest_off),
+      at<__nv_bfloat16>(ws, L.y_shared), ret, at<int32_t>(ws, L.send_slot), at<int32_t>(ws, L.dest_off),
       sh.H, W, ret_rows, seg_rows, static_cast<__nv_bfloat16*>(y), at<uint32_t>(ws, L.status));
   return cuda_status(cudaGetLastError());
 }
@@ -720,8 +722,8 @@ int moe_ep_shared(moe_shape sh, int32_t W, const moe_weights* w_local, void* ws,
   cudaError_t e = launch_expert_up(gg, at<uint8_t>(ws, L.a_q), at<float>(ws, L.a_s), w13, s13,
                                    at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), s, sms);
   if (e == cudaSuccess)
-    e = launch_expert_down(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w2, s2,
-                           at<float>(ws, L.y_shared), s, sms);
+    e = launch_expert_down_bf16(gg, at<uint8_t>(ws, L.h_q), at<float>(ws, L.h_s), w2, s2,
+                                at<__nv_bfloat16>(ws, L.y_shared), s, sms);
   return cuda_status(e);
 }
 

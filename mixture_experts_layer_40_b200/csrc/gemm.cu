@@ -57,15 +57,23 @@ constexpr uint32_t kIdesc = make_idesc(kBM, kBN, 0u, 0u);  // E4M3 x E4M3 -> fp3
 #endif
 constexpr int kYCols = MOE_YCOLS;
 constexpr int kYBufBytes = 32 * kYCols * 4;
+// What the epilogue makes of a finished tile:
+//   kEpiUp    SwiGLU of the gate/up halves, then the 1x128 E4M3 requant of h
+//   kEpiF32   fp32 rows (the backward's GEMMs, and the stage entry point that
+//             pins the accumulation against float64)
+//   kEpiBf16  bf16 rows, rounded once from the fp32 totals (the layer's
+//             expert outputs)
+enum Epi : int { kEpiUp = 0, kEpiF32 = 1, kEpiBf16 = 2 };
 // the up GEMM (56 k-blocks per tile at H = 7168) keeps a 4-stage ring; the
-// down GEMM gives one stage to the output staging buffers
-template <bool kUp>
+// down GEMMs give one stage to the output staging buffers
+template <int kEpi>
 struct Cfg {
-  static constexpr int stages = kUp ? kMaxStages : MOE_DOWN_STAGES;
+  static constexpr bool up = kEpi == kEpiUp;
+  static constexpr int stages = up ? kMaxStages : MOE_DOWN_STAGES;
   static constexpr size_t dyn_smem =
-      (size_t)stages * kStageBytes + (kUp ? 0 : 8 * 2 * kYBufBytes) + 1024;
+      (size_t)stages * kStageBytes + (up ? 0 : 8 * 2 * kYBufBytes) + 1024;
 };
-static_assert(Cfg<false>::dyn_smem + 8192 <= 232448, "shared memory");
+static_assert(Cfg<kEpiF32>::dyn_smem + 8192 <= 232448, "shared memory");
 // Register split: launched at kLaunchRegs per thread (384 x 168 = 64512);
 // warpgroup 0 drops to kRegsCtl, the two epilogue warpgroups rise to kRegsEpi.
 // 128 * kRegsCtl + 256 * kRegsEpi must not exceed 384 * kLaunchRegs.
@@ -87,7 +95,8 @@ struct GemmArgs {
   uint8_t* h_q;           // up: [rows, I]
   float* h_s;             // up: [rows, I / 128]
   int32_t I;
-  float* y;               // down: [rows, H] fp32
+  float* y;               // kEpiF32: [rows, H] fp32
+  __nv_bfloat16* yb;      // kEpiBf16: [rows, H] bf16
   int32_t H;
   uint32_t* status;
 };
@@ -122,12 +131,13 @@ MOE_DEV void decode_tile(int tile, const int* prefix, int n_groups, int n_tiles,
 // For a < -88, exp(-a) is +inf and the quotient is -0.
 MOE_DEV float silu(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
-template <bool kUp>
+template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
-  constexpr int kSt = Cfg<kUp>::stages;
+  constexpr bool kUp = kEpi == kEpiUp;
+  constexpr int kSt = Cfg<kEpi>::stages;
   __shared__ GemmShared sh;
   extern __shared__ uint8_t dyn_smem[];
   const uint32_t ring = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -356,6 +366,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (eg == 0) p.h_s[grow * (p.I / kBM) + n] = s;
         }
+      } else if (kEpi == kEpiBf16) {
+        // bf16 rows (one rounding of the fp32 totals) out through shared
+        // memory and TMA stores, 64 columns (128 bytes) of the warp's 32 rows
+        // at a time, when all 32 rows belong to the group; a group's last,
+        // partial 32 rows are stored directly, row by row, and padding rows
+        // are never written
+        const int q_live = valid - quarter * 32;
+        const int y0 = p.group_start[g] + m * kBM + quarter * 32;
+        const int x0 = n * kBN + 128 * eg;
+        const uint32_t swz = (uint32_t)(lane & 7);
+        if (q_live < 32) {
+          if (live) {
+            uint4* dst = reinterpret_cast<uint4*>(p.yb + grow * p.H + x0);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              dst[j] = make_uint4(pack_bf16x2(acc[8 * j + 0], acc[8 * j + 1]),
+                                  pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]),
+                                  pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]),
+                                  pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t buf_j = ybuf + (uint32_t)(j * kYBufBytes);
+            // the store that last read this buffer (two chunks ago) is done
+            if (lane == 0) bulk_wait_read_1();
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t dst = buf_j + (uint32_t)lane * 128u + (((uint32_t)c ^ swz) << 4);
+              const int a0 = 64 * j + 8 * c;
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                           "r"(pack_bf16x2(acc[a0 + 0], acc[a0 + 1])),
+                           "r"(pack_bf16x2(acc[a0 + 2], acc[a0 + 3])),
+                           "r"(pack_bf16x2(acc[a0 + 4], acc[a0 + 5])),
+                           "r"(pack_bf16x2(acc[a0 + 6], acc[a0 + 7]))
+                           : "memory");
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_y, buf_j, x0 + 64 * j, y0);
+              bulk_commit();
+            }
+          }
+        }
       } else {
         // fp32 rows out through shared memory and TMA stores, 8 columns of
         // the warp's 32 rows at a time, when all 32 rows belong to the group;
@@ -409,26 +465,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, 512);
 }
 
-template <bool kUp>
+template <int kEpi>
 cudaError_t launch(const GemmArgs& a, const CUtensorMap& ma, const CUtensorMap& mb,
                    const CUtensorMap& my,
                    cudaStream_t stream, int sm_count, int64_t tile_bound) {
-  static bool configured = false;
-  if (!configured) {
-    // the register split above is only safe if the kernel really was built
-    // with kLaunchRegs registers per thread
+  // once per device: the register split above is only safe if the kernel
+  // really was built with kLaunchRegs registers per thread, and the large
+  // dynamic shared memory must be allowed on each device the kernel runs on
+  static DeviceOnce once;
+  cudaError_t e = once.run([] {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<kUp>);
-    if (e != cudaSuccess) return e;
+    cudaError_t r = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<kEpi>);
+    if (r != cudaSuccess) return r;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<kUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Cfg<kUp>::dyn_smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+    return cudaFuncSetAttribute(grouped_gemm_kernel<kEpi>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Cfg<kEpi>::dyn_smem);
+  });
+  if (e != cudaSuccess) return e;
   int grid = sm_count;
   if (tile_bound < grid) grid = (int)(tile_bound > 0 ? tile_bound : 1);
-  grouped_gemm_kernel<kUp><<<grid, kThreads, Cfg<kUp>::dyn_smem, stream>>>(ma, mb, my, a);
+  grouped_gemm_kernel<kEpi><<<grid, kThreads, Cfg<kEpi>::dyn_smem, stream>>>(ma, mb, my, a);
   return cudaGetLastError();
 }
 
@@ -458,8 +515,29 @@ cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const fl
   a.H = gg.H;
   a.status = gg.status;
   const int64_t bound = (gg.rows / kBM + gg.n_groups) * (int64_t)a.n_tiles;
-  return launch<true>(a, ma, mb, ma, stream, sm_count, bound);
+  return launch<kEpiUp>(a, ma, mb, ma, stream, sm_count, bound);
 }
+
+namespace {
+
+GemmArgs down_args(const GroupedGemm& gg, const float* h_s, const float* s2) {
+  GemmArgs a{};
+  a.group_rows = gg.group_rows;
+  a.group_start = gg.group_start;
+  a.n_groups = gg.n_groups;
+  a.kblocks = gg.I / kBK;
+  a.n_tiles = gg.H / kBN;
+  a.b_rows = gg.H;
+  a.rows = gg.rows;
+  a.a_s = h_s;
+  a.b_s = s2;
+  a.I = gg.I;
+  a.H = gg.H;
+  a.status = gg.status;
+  return a;
+}
+
+}  // namespace
 
 cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const float* h_s,
                                const uint8_t* w2, const float* s2, float* y,
@@ -471,22 +549,26 @@ cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const 
   if (e != cudaSuccess) return e;
   e = make_tmap_f32(&my, y, gg.H, gg.rows, kYCols, 32);
   if (e != cudaSuccess) return e;
-  GemmArgs a{};
-  a.group_rows = gg.group_rows;
-  a.group_start = gg.group_start;
-  a.n_groups = gg.n_groups;
-  a.kblocks = gg.I / kBK;
-  a.n_tiles = gg.H / kBN;
-  a.b_rows = gg.H;
-  a.rows = gg.rows;
-  a.a_s = h_s;
-  a.b_s = s2;
+  GemmArgs a = down_args(gg, h_s, s2);
   a.y = y;
-  a.I = gg.I;
-  a.H = gg.H;
-  a.status = gg.status;
   const int64_t bound = (gg.rows / kBM + gg.n_groups) * (int64_t)a.n_tiles;
-  return launch<false>(a, ma, mb, my, stream, sm_count, bound);
+  return launch<kEpiF32>(a, ma, mb, my, stream, sm_count, bound);
+}
+
+cudaError_t launch_expert_down_bf16(const GroupedGemm& gg, const uint8_t* h_q, const float* h_s,
+                                    const uint8_t* w2, const float* s2, __nv_bfloat16* y,
+                                    cudaStream_t stream, int sm_count) {
+  CUtensorMap ma, mb, my;
+  cudaError_t e = make_tmap_u8(&ma, h_q, gg.I, gg.rows, kBK, kBM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_u8(&mb, w2, gg.I, (int64_t)gg.n_groups * gg.H, kBK, kBN);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16(&my, y, gg.H, gg.rows, 1, 64, 32);
+  if (e != cudaSuccess) return e;
+  GemmArgs a = down_args(gg, h_s, s2);
+  a.yb = y;
+  const int64_t bound = (gg.rows / kBM + gg.n_groups) * (int64_t)a.n_tiles;
+  return launch<kEpiBf16>(a, ma, mb, my, stream, sm_count, bound);
 }
 
 }  // namespace moe

@@ -6,6 +6,11 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
+#include <atomic>
+#include <mutex>
+
 #include "../../include/moe_capi.h"
 
 namespace moe {
@@ -32,6 +37,45 @@ struct Carver {
     off = (size_t)round_up((int64_t)(off + bytes), 256);
     return a;
   }
+};
+
+// An NVTX range over a host scope (entry points and the forward's stages), for
+// timeline profilers; without a profiler attached the calls do nothing. The
+// range covers the host-side enqueue, not the kernels' execution.
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// A set-up step (kernel attributes) done once per device: the first call
+// with a device current runs it, later calls on that device skip it. A step
+// that fails is retried by the next call. Safe to use from several host
+// threads. Function attributes belong to the device's context, so a process
+// that resets a device (cudaDeviceReset) must not call the library on that
+// device again.
+class DeviceOnce {
+ public:
+  template <typename F>
+  cudaError_t run(F&& setup) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    e = setup();
+    if (e == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+    return e;
+  }
+
+ private:
+  static constexpr int kMaxDevices = 64;
+  std::mutex mu_;
+  std::atomic<bool> done_[kMaxDevices] = {};
 };
 
 }  // namespace moe

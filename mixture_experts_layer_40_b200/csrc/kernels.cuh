@@ -3,6 +3,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "host_util.h"
 
 namespace moe {
 
@@ -74,7 +75,7 @@ cudaError_t launch_wgrad(const int32_t* group_rows, const int32_t* group_start, 
                          cudaStream_t stream, int sm_count);
 cudaError_t launch_swiglu_backward(const float* gu, const float* dh, int64_t rows, int I,
                                    uint8_t* q, float* qs, cudaStream_t stream, int sm_count);
-cudaError_t launch_gate_grad(const void* dy, const float* y_rows, const int32_t* token_row, int T,
+cudaError_t launch_gate_grad(const void* dy, const __nv_bfloat16* y_rows, const int32_t* token_row, int T,
                              int H, int K, int64_t routed_cap, float* dgates, uint32_t* status,
                              cudaStream_t stream, int sm_count);
 
@@ -85,14 +86,18 @@ cudaError_t launch_balance_stats(const float* logits, const int32_t* ids, int T,
                                  int seq_len, float alpha, uint8_t* scratch, float* f, float* P,
                                  float* loss, cudaStream_t stream);
 
-// Permutation: scan of counts into group tables, stable scatter of the
-// (token, slot) pairs into expert-major GEMM rows. Slots whose id is
-// negative are skipped (their token_row entries are left as they are);
-// `pairs` is the number of slots with an id, checked against the counts.
+// Permutation: per-chunk ranks and counts, a scan of the counts into group
+// tables and per-chunk base rows, and the stable placement of the (token,
+// slot) pairs into expert-major GEMM rows. Slots whose id is negative are
+// skipped (their token_row entries are left as they are); `pairs` is the
+// number of slots with an id, checked against the counts. `hist` is scratch
+// of permute_scratch_bytes(T, N) bytes.
+size_t permute_scratch_bytes(int64_t T, int N);
 cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K,
-                           int64_t pairs, int64_t routed_cap, int32_t* offsets, int32_t* group_rows,
-                           int32_t* row_start, int32_t* row_token, int32_t* token_row,
-                           uint32_t* status, cudaStream_t stream);
+                           int64_t pairs, int64_t routed_cap, int32_t* hist, int32_t* offsets,
+                           int32_t* group_rows, int32_t* row_start, int32_t* row_token,
+                           int32_t* token_row, uint32_t* status, cudaStream_t stream,
+                           int sm_count);
 // 1x128 quantisation of x written to each token's shared-expert row
 // (routed_cap + t) and to its K routed rows token_row[t, k].
 cudaError_t launch_quantize_scatter(const void* x, int T, int H, int K, const int32_t* token_row,
@@ -102,10 +107,23 @@ cudaError_t launch_quantize_scatter(const void* x, int T, int H, int K, const in
 cudaError_t launch_expert_up(const GroupedGemm& gg, const uint8_t* a_q, const float* a_s,
                              const uint8_t* w13, const float* s13, uint8_t* h_q, float* h_s,
                              cudaStream_t stream, int sm_count);
+// Down GEMM with fp32 output rows (the backward's GEMMs; the accumulation
+// pin) and with bf16 output rows (the layer's expert outputs).
 cudaError_t launch_expert_down(const GroupedGemm& gg, const uint8_t* h_q, const float* h_s,
                                const uint8_t* w2, const float* s2, float* y,
                                cudaStream_t stream, int sm_count);
+cudaError_t launch_expert_down_bf16(const GroupedGemm& gg, const uint8_t* h_q, const float* h_s,
+                                    const uint8_t* w2, const float* s2, __nv_bfloat16* y,
+                                    cudaStream_t stream, int sm_count);
 
+// Combine of the layer (bf16 expert rows) and of the backward's input
+// gradients (fp32 rows): y[t] = row[shared] + sum_k g[t,k] row[token_row[t,k]]
+// in fp32, slots by ascending expert id, one rounding to bf16 (gates null:
+// every weight 1).
+cudaError_t launch_combine(const __nv_bfloat16* y_rows, const int32_t* ids, const float* gates,
+                           const int32_t* token_row, int T, int H, int K, int64_t routed_cap,
+                           int64_t rows_total, __nv_bfloat16* y, uint32_t* status,
+                           cudaStream_t stream);
 cudaError_t launch_combine(const float* y_rows, const int32_t* ids, const float* gates,
                            const int32_t* token_row, int T, int H, int K, int64_t routed_cap,
                            int64_t rows_total, __nv_bfloat16* y, uint32_t* status,

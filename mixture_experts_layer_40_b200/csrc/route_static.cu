@@ -9,14 +9,16 @@
 // scratch in a fixed array in the library's own device memory instead, so the
 // caller passes only the inputs and outputs and nothing is allocated.
 //
+// The logits come from the fp32 SIMT kernel (launch_router), not from the
+// split-bf16 tensor-core kernel of moe_route: the top-K, gates and counts are
+// moe_route's up to near ties of the K-th score and fp32 logit rounding.
+//
 // The array exists once per GPU that loads the library and stays resident
 // until the process exits. Every call shares it: two calls whose kernels
 // overlap on the GPU (different streams, or different host threads on one
 // device) race on it and must be serialised by the caller. The logits are
 // fully rewritten by each call, so no part of the array needs clearing; the
 // counts output is zeroed by the call itself.
-#include <mutex>
-
 #include "kernels.cuh"
 
 namespace moe {
@@ -25,23 +27,15 @@ namespace {
 // Scratch for the gate logits: T * N floats at most (4 MiB).
 __device__ __align__(256) float g_route_scratch[MOE_ROUTE_NOALLOC_MAX_LOGITS];
 
-constexpr int kMaxDevices = 64;
-
-// Device address of g_route_scratch on each device. Host code cannot use the
-// array's name as a device pointer (it names a host-side stand-in), so the
-// address is looked up once per device, with that device current.
+// Device address of g_route_scratch on the current device. Host code cannot
+// use the array's name as a device pointer (it names a host-side stand-in),
+// so the address is looked up, with the device current, on every call: the
+// lookup is cheap, and an address cached across calls would go stale if the
+// device's context were reset.
 float* scratch_on_current_device() {
-  static float* addr[kMaxDevices] = {nullptr};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<float*>(p);
-  }
-  return addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
+  return static_cast<float*>(p);
 }
 
 }  // namespace

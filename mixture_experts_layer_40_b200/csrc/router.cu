@@ -528,13 +528,12 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&mw, wsplit, H, N, 3, kRK, kRN);
   if (e != cudaSuccess) return e;
-  static bool configured = false;
-  if (!configured) {
-    e = cudaFuncSetAttribute(logits_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kRDynSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static DeviceOnce once;  // the shared-memory limit is raised once per device
+  e = once.run([] {
+    return cudaFuncSetAttribute(logits_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kRDynSmem);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((T + kRM - 1) / kRM), (unsigned)((N + kRN - 1) / kRN));
   logits_tc_kernel<<<grid, kRThreads, kRDynSmem, stream>>>(mx, mw, T, H, N, logits, status);
   e = cudaGetLastError();

@@ -267,19 +267,20 @@ cudaError_t launch_wgrad(const int32_t* group_rows, const int32_t* group_start, 
                          const uint8_t* b_t, const float* b_inv, float* c, uint32_t* status,
                          cudaStream_t stream, int sm_count) {
   if (M % kBM != 0 || N % kBN != 0 || gemm_rows % kBM != 0) return cudaErrorInvalidValue;
-  static bool configured = false;
-  if (!configured) {
+  // once per device: the register split needs the launch register count it
+  // was written for, and the large dynamic shared memory must be allowed
+  static DeviceOnce once;
+  cudaError_t e = once.run([] {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, wgrad_gemm_kernel);
-    if (e != cudaSuccess) return e;
+    cudaError_t r = cudaFuncGetAttributes(&fa, wgrad_gemm_kernel);
+    if (r != cudaSuccess) return r;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(wgrad_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kDynSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+    return cudaFuncSetAttribute(wgrad_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kDynSmem);
+  });
+  if (e != cudaSuccess) return e;
   CUtensorMap ma, mb, mc;
-  cudaError_t e = make_tmap_u8(&ma, a_t, gemm_rows, M, kBK, kBM);
+  e = make_tmap_u8(&ma, a_t, gemm_rows, M, kBK, kBM);
   if (e != cudaSuccess) return e;
   e = make_tmap_u8(&mb, b_t, gemm_rows, N, kBK, kBN);
   if (e != cudaSuccess) return e;

@@ -10,6 +10,7 @@ indexing, which moves bytes and computes nothing.
 from __future__ import annotations
 
 import dataclasses
+import struct
 
 import numpy as np
 import torch
@@ -153,3 +154,39 @@ class MoELayer:
         off = getattr(self.layout, name)
         n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
         return self.ws[off:off + n].view(dtype).view(*shape)
+
+
+# ---------------------------------------------------------------- controller state
+#
+# The routing bias is the layer's only state that changes during training
+# (the aux-loss-free controller, "DeepSeek-V3: Auxiliary-Loss-Free MoE Load
+# Balancing...", section III). It is saved with its exact float32 bits, so a
+# run resumed from the file takes the same routing decisions and bias steps
+# as one that never stopped.
+BIAS_MAGIC = b"MOEBIAS1"
+
+
+def save_bias(path: str, bias: torch.Tensor, step: int, gamma: float) -> None:
+    """Writes the bias (float32 [N], device or host) and the controller's step
+    count and gamma: magic, then N and step (int64), gamma (float32), then
+    the N float32 values, all little-endian."""
+    b = bias.detach().to("cpu", torch.float32).contiguous().numpy()
+    with open(path, "wb") as f:
+        f.write(BIAS_MAGIC)
+        f.write(struct.pack("<qqf", b.shape[0], int(step), float(gamma)))
+        f.write(b.astype("<f4").tobytes())
+
+
+def load_bias(path: str, device="cpu") -> tuple[torch.Tensor, int, float]:
+    """Reads a file written by save_bias: (bias float32 [N] on `device`, step,
+    gamma). Raises ValueError on a file of another format or a short file."""
+    with open(path, "rb") as f:
+        data = f.read()
+    head = len(BIAS_MAGIC) + struct.calcsize("<qqf")
+    if len(data) < head or data[:len(BIAS_MAGIC)] != BIAS_MAGIC:
+        raise ValueError(f"{path}: not a routing-bias file")
+    n, step, gamma = struct.unpack("<qqf", data[len(BIAS_MAGIC):head])
+    if n < 0 or len(data) != head + 4 * n:
+        raise ValueError(f"{path}: {len(data) - head} bytes of values for N = {n}")
+    vals = np.frombuffer(data[head:], dtype="<f4").astype(np.float32)
+    return torch.from_numpy(vals.copy()).to(device), int(step), float(gamma)

@@ -61,3 +61,27 @@ def test_recorded_traffic_follows_the_sources(tmp_path, monkeypatch):
     assert bench.recorded_traffic("expert_up", "v3_prefill") == 123
     assert bench.recorded_traffic("expert_up", "decode") is None
     assert bench.recorded_traffic("expert_down", "v3_prefill") is None   # stale capture
+
+
+def test_gpus_flag_starts_the_ranks():
+    """bench.py --gpus 2 without a rank environment starts two ranks itself
+    (torchrun on 127.0.0.1); they meet in a process group (gloo here, no GPU)
+    and rank 0 reports n_gpus = 2."""
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                          "--launch-check"], capture_output=True, text=True, timeout=300,
+                         cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["ranks_counted"] == 2 and d["max_rank"] == 1.0
+
+
+def test_cpu_baseline_builds_the_pools_before_timing():
+    """The oracle's dequantised block pool is built in the set-up, so no
+    timed sample step pays for it."""
+    w = I.WORKLOADS["tiny"]
+    _, _, _, ew = bench.oracle_setup(w, I.make_x(w))
+    assert getattr(ew, "_deq", None) is not None

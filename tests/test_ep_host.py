@@ -168,7 +168,8 @@ def test_row_bytes_and_workspace_sizes(capi):
     assert capi.moe_ep_row_bytes(capi.shape_of(10, 256, 16, 3, 128)) == 288
     # 256 + 8 + 5 * 8 = 304
     assert capi.moe_ep_row_bytes(capi.shape_of(10, 256, 16, 5, 128)) == 304
-    assert capi.moe_ep_dispatch_workspace_size(sh, 8) > 4096 * 7168 * 4
+    # at least the shared expert's bf16 output rows
+    assert capi.moe_ep_dispatch_workspace_size(sh, 8) > 4096 * 7168 * 2
     for bad_w in [0, 3, 17, 32]:  # 256/3 not whole; more than 16 ranks; 256/32 < 16
         assert capi.moe_ep_dispatch_workspace_size(sh, bad_w) == 0
     assert capi.moe_ep_expert_workspace_size(sh, 8, 100, 801) == 0  # pairs > R K

@@ -81,7 +81,8 @@ def _bws_views(layer, w):
     dh = take(R * w.I * 4, torch.float32, (R, w.I))
     dgu_q = take(R * 2 * w.I, torch.uint8, (R, 2 * w.I))
     dgu_s = take(R * (2 * w.I // 128) * 4, torch.float32, (R, 2 * w.I // 128))
-    return dy_q, dy_s, dh, dgu_q, dgu_s
+    dx_rows = take(R * w.H * 4, torch.float32, (R, w.H))
+    return dy_q, dy_s, dh, dgu_q, dgu_s, dx_rows
 
 
 def test_transposed_weights_bit_exact():
@@ -105,7 +106,7 @@ def test_backward_small(t):
     case, layer, dy, dx, dgates = _run(w, 3)
     _check(w, case, layer, dy, dx, dgates)
     L = layer.layout
-    dy_q, dy_s, dh, dgu_q, dgu_s = _bws_views(layer, w)
+    dy_q, dy_s, dh, dgu_q, dgu_s, dx_rows = _bws_views(layer, w)
     sh = slice(L.routed_cap, L.routed_cap + w.T)
     # the shared expert's dY rows are dy itself, 1x128-quantised: bit-exact
     rq, rs = O.quantize_1x128(dy)
@@ -122,8 +123,7 @@ def test_backward_small(t):
     d_g = O.dequantize_1x128(codes[:, :, 0].reshape(w.T, w.I), scales[:, :, 0])
     d_u = O.dequantize_1x128(codes[:, :, 1].reshape(w.T, w.I), scales[:, :, 1])
     dxr_ref = d_g @ wg + d_u @ wu
-    y_rows = layer.view("y_rows", torch.float32, (L.rows_total, w.H))
-    got = y_rows[sh].cpu().numpy().astype(np.float64)
+    got = dx_rows[sh].cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - dxr_ref) <= 1e-5 * np.sqrt(np.mean(dxr_ref ** 2, axis=1, keepdims=True)))
 
 
@@ -147,7 +147,7 @@ def _bws_wgrad_views(layer, w):
     """The weight-gradient part of the backward workspace (after _bws_views)."""
     R = layer.layout.rows_total
     sizes = [R * w.H, R * (w.H // 128) * 4, R * 2 * w.I * 4, R * w.I * 4, R * 2 * w.I,
-             R * (2 * w.I // 128) * 4]
+             R * (2 * w.I // 128) * 4, R * w.H * 4]
     off = 0
     for n in sizes:
         off = (off + n + 255) // 256 * 256

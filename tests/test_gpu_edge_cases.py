@@ -72,8 +72,7 @@ def test_every_expert_selected():
     assert np.array_equal(layer.counts.cpu().numpy(), np.full(16, w.T, np.int32))
     r_ids, _, _, score = O.route(case.x, case.gate_w, case.bias, w.K)
     use, _, _ = H.reconcile_ids(gid, r_ids, score, w.K)
-    ref = O.moe_forward(case.x, case.gate_w, case.bias, w.K, case.ew, mode="Q", ids=use)
-    H.check_rows(y, ref["y"])
+    H.expert_path_parity(w, case, layer, y, use, np.arange(w.T))
 
 
 def test_largest_expert_count_and_k():
@@ -86,5 +85,56 @@ def test_largest_expert_count_and_k():
     r_ids, _, _, score = O.route(case.x, case.gate_w, case.bias, w.K)
     use, _, _ = H.reconcile_ids(gid, r_ids, score, w.K)
     assert np.array_equal(layer.counts.cpu().numpy(), O.expert_counts(use, w.N))
-    ref = O.moe_forward(case.x, case.gate_w, case.bias, w.K, case.ew, mode="Q", ids=use)
-    H.check_rows(y, ref["y"])
+    H.expert_path_parity(w, case, layer, y, use, np.arange(w.T))
+
+
+_TWO_THREADS = r"""
+import sys, threading
+import numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+from mixture_experts_layer_40_b200 import inputs as I
+from mixture_experts_layer_40_b200.layer import MoELayer, device_weights
+w = I.Workload("threads", T=200, H=512, N=32, K=4, I=256, bias_range=0.1, seed=77)
+xb = I.make_x(w)
+pool = I.make_weight_pool(w)
+layers = [MoELayer(w.T, w.H, w.N, w.K, w.I, device_weights(w, pool, I.make_gate_w(w), "cuda"))
+          for _ in range(2)]
+x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+bias = torch.from_numpy(I.make_bias(w)).cuda()
+torch.cuda.synchronize()
+start = threading.Barrier(2)
+out, errors = [None, None], []
+def run(i):
+    try:
+        torch.cuda.set_device(0)
+        s = torch.cuda.Stream()
+        start.wait()
+        with torch.cuda.stream(s):
+            out[i] = layers[i].forward(x, bias, stream=s)
+            out[i] = out[i].clone()
+        s.synchronize()
+        assert layers[i].status(s) == 0
+    except Exception as e:
+        errors.append(repr(e))
+ts = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+[t.start() for t in ts]
+[t.join() for t in ts]
+assert not errors, errors
+assert torch.equal(out[0], out[1])
+assert torch.equal(out[0], layers[0].forward(x, bias))
+print("ok")
+"""
+
+
+def test_first_calls_from_two_host_threads():
+    """The once-per-device set-up of the kernels (shared-memory limits, the
+    register-count check) is taken under a lock: in a fresh process, two host
+    threads whose first library calls run at the same time on one device
+    both get the layer's result, bit for bit."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _TWO_THREADS, root], capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr

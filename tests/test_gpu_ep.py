@@ -15,8 +15,12 @@ Checks, per rank:
     output is the same GEMM result, only the order of the fp32 additions in
     the combine differs, so values agree to one bf16 ulp (plus a 4e-6 RMS
     allowance for cancellation) and almost all are identical;
-  * the output against the oracle (small shapes), as for the forward.
+  * the output against the oracle (small shapes): the one-GPU layer on the
+    rank's tokens stage by stage (tests/helpers.py expert_path_parity), and
+    the expert-parallel output the rounding of the oracle's combine of those
+    expert outputs, up to near ties, within the layer output's tier.
 The product's ExpertParallelMoE is also run over a real one-rank NCCL group."""
+import dataclasses
 import socket
 
 import numpy as np
@@ -149,16 +153,22 @@ def check_against_forward(w: I.Workload, st, dw, bias, G=0, M=0):
     diff = np.abs(a - b)
     assert np.all(diff <= ulp + 4e-6 * rms), float(np.max(diff / (ulp + 4e-6 * rms)))
     assert np.mean(a == b) >= 0.95
-    return layer
+    return layer, b
 
 
-def check_against_oracle(w: I.Workload, st, case_gate_w, ew, bias):
+def check_against_oracle(w: I.Workload, st, case, one_gpu):
     if st["T"] == 0:
         return
+    layer, y_one = one_gpu
+    wr = dataclasses.replace(w, T=st["T"])
     x = I.bf16_bits_to_f32(st["x_bits"])
-    ids = st["ids"].cpu().numpy()
-    ref = O.moe_forward(x, case_gate_w, bias, w.K, ew, mode="Q", ids=ids)
-    H.check_rows(st["y"].float().cpu().numpy(), ref["y"])
+    rcase = dataclasses.replace(case, w=wr, x_bits=st["x_bits"], x=x)
+    r_ids, _, _, score = O.route(x, case.gate_w, case.bias, w.K)
+    use, _, _ = H.reconcile_ids(st["ids"].cpu().numpy(), r_ids, score, w.K)
+    stats = H.expert_path_parity(wr, rcase, layer, y_one, use, np.arange(st["T"]))
+    y_ep = st["y"].float().cpu().numpy().astype(np.float64)
+    H.check_bf16(y_ep, stats["y_ref"], "expert-parallel combine")
+    H.check_rows(y_ep, stats["y_ref"])
 
 
 def _setup(w: I.Workload):
@@ -175,8 +185,8 @@ def test_ep_two_ranks(W, Ts):
     ranks = emulate(w, W, xs, dw, case.bias)
     for st in ranks:
         check_plan(w, W, st)
-        check_against_forward(w, st, dw, case.bias)
-        check_against_oracle(w, st, case.gate_w, case.ew, case.bias)
+        one = check_against_forward(w, st, dw, case.bias)
+        check_against_oracle(w, st, case, one)
 
 
 def test_ep_four_ranks_node_limited():

@@ -1,9 +1,11 @@
 """GPU parity of the whole layer forward (moe_forward through the C ABI)
 against the oracle: intermediates that are integer or byte work are compared
 bit-exactly (x codes and scales, counts, offsets, the permutation), routing
-with the near-tie rule, and the output rows within 2e-2 of their RMS. Small
-workloads are checked on every token; the V3-shape ones on a seeded sample
-of tokens (routing, counts and the permutation always on every token)."""
+with the near-tie rule, the expert path stage by stage (h codes, the bf16
+expert outputs, the combine; tests/helpers.py expert_path_parity) and the
+output rows within 2e-2 of their RMS. Small workloads are checked on every
+token; the V3-shape ones on a seeded sample of 512 tokens (routing, counts
+and the permutation always on every token)."""
 import numpy as np
 import pytest
 import torch
@@ -76,14 +78,14 @@ def check_intermediates(w, case, layer, bias, sample_rows=None):
 
 
 def check_output(w, case, layer, bias, y, use_ids, tokens=None):
-    ref = O.moe_forward(case.x, case.gate_w, bias, w.K, case.ew, mode="Q", tokens=tokens,
-                        ids=use_ids)
-    yg = y if tokens is None else y[tokens]
-    worst = H.check_rows(yg, ref["y"])
-    gates = layer.gates.cpu().numpy()
-    sel = ref["gates"] if tokens is None else ref["gates"]
-    assert np.max(np.abs(gates - sel)) < 1e-5
-    return worst
+    tokens = np.arange(w.T) if tokens is None else np.asarray(tokens)
+    stats = H.expert_path_parity(w, case, layer, y[tokens], use_ids, tokens)
+    # gates of the GPU's ids from the oracle's unbiased affinities
+    s = O.sigmoid(O.gate_logits(case.x, case.gate_w))
+    sel = np.take_along_axis(s, use_ids.astype(np.int64), axis=1)
+    ref_gates = sel / sel.sum(axis=1, keepdims=True)
+    assert np.max(np.abs(layer.gates.cpu().numpy() - ref_gates)) < 1e-5
+    return stats
 
 
 def test_forward_tiny_all_tokens():
@@ -135,14 +137,36 @@ def test_forward_decode_v3_shape():
     w = I.WORKLOADS["decode"]
     case, layer, bias, y = run_forward(w)
     use_ids, _ = check_intermediates(w, case, layer, bias)
-    tokens = np.random.default_rng(0).choice(w.T, 24, replace=False)
-    check_output(w, case, layer, bias, y, use_ids, tokens=np.sort(tokens))
+    check_output(w, case, layer, bias, y, use_ids)
+
+
+def _sampled(w, seed, n=512):
+    return np.sort(np.random.default_rng(seed).choice(w.T, min(n, w.T), replace=False))
 
 
 def test_forward_v3_prefill_sampled():
     w = I.WORKLOADS["v3_prefill"]
     case, layer, bias, y = run_forward(w)
-    rows = np.random.default_rng(1).choice(w.T, 256, replace=False)
-    use_ids, _ = check_intermediates(w, case, layer, bias, sample_rows=rows)
-    tokens = np.sort(np.random.default_rng(2).choice(w.T, 16, replace=False))
-    check_output(w, case, layer, bias, y, use_ids, tokens=tokens)
+    use_ids, _ = check_intermediates(w, case, layer, bias, sample_rows=_sampled(w, 1))
+    check_output(w, case, layer, bias, y, use_ids, tokens=_sampled(w, 2))
+
+
+def test_forward_large_prefill_outliers_sampled():
+    """T = 32768 with 1% of the channels scaled x20 (the outliers that stress
+    the 1x128 tiles): routing, counts and the permutation on every token; x
+    codes and scales, h codes, expert outputs and y on 512 seeded tokens."""
+    w = I.WORKLOADS["large_prefill"]
+    case, layer, bias, y = run_forward(w)
+    use_ids, _ = check_intermediates(w, case, layer, bias, sample_rows=_sampled(w, 3))
+    check_output(w, case, layer, bias, y, use_ids, tokens=_sampled(w, 4))
+
+
+def test_forward_skewed_sampled():
+    """T = 8192 with Zipf-ranked gate logits: a few experts receive most of
+    the tokens (the largest groups of the grouped GEMMs)."""
+    w = I.WORKLOADS["skewed"]
+    case, layer, bias, y = run_forward(w)
+    counts = layer.counts.cpu().numpy()
+    assert counts.max() > 4 * counts.mean()
+    use_ids, _ = check_intermediates(w, case, layer, bias, sample_rows=_sampled(w, 5))
+    check_output(w, case, layer, bias, y, use_ids, tokens=_sampled(w, 6))

@@ -243,3 +243,50 @@ def test_expert_down_parity(capi, h_dim, i_dim, group_rows):
         rel = np.sqrt(np.mean((got - ref) ** 2) / np.mean(ref ** 2))
         assert rel < 1e-6, rel
     assert np.all(yg[~written] == 3.0)
+
+
+@pytest.mark.parametrize("h_dim,i_dim,group_rows", [
+    (256, 128, [5, 0, 128, 129, 300, 1, 31, 32, 33]),
+    (7168, 2048, [130, 0, 7, 256]),
+])
+def test_expert_down_bf16_is_the_rounded_fp32_gemm(capi, h_dim, i_dim, group_rows):
+    """The layer's down GEMM writes bf16 expert outputs ("DeepSeek-V3:
+    Auxiliary-Loss-Free MoE Load Balancing...", section V, Figure 6): bit for
+    bit the round-to-nearest-even of the fp32 GEMM's totals (same kernel,
+    other epilogue), and the bf16 rounding of the float64 sums of the same
+    operands up to the near-midpoint rule. Groups of 31, 32 and 33 rows cover
+    the direct stores of a partial 32-row quarter and the staged TMA stores."""
+    rng = np.random.default_rng(h_dim + 2)
+    starts, r = [], 0
+    for n in group_rows:
+        starts.append(r)
+        r += (n + 127) // 128 * 128 + 128
+    rows, n_groups = r, len(group_rows)
+    h = (rng.standard_normal((rows, i_dim)) * rng.uniform(0.1, 10, (rows, 1))).astype(np.float32)
+    h_q, h_s = O.quantize_1x128(h)
+    w2 = (rng.standard_normal((n_groups, h_dim, i_dim)) / np.sqrt(i_dim)).astype(np.float32)
+    q2 = np.empty(w2.shape, np.uint8)
+    s2 = np.empty((n_groups, h_dim // 128, i_dim // 128), np.float32)
+    for g in range(n_groups):
+        q2[g], s2[g] = O.quantize_128x128(w2[g])
+    args = (h_dim, i_dim, n_groups, _dev(np.array(group_rows, np.int32)),
+            _dev(np.array(starts, np.int32)), rows, _dev(h_q), _dev(h_s), _dev(q2), _dev(s2))
+    y32 = torch.full((rows, h_dim), 3.0, dtype=torch.float32, device="cuda")
+    y16 = torch.full((rows, h_dim), 3.0, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    capi.moe_expert_down(*args, y32, status)
+    capi.moe_expert_down_bf16(*args, y16, status)
+    assert capi.moe_get_status(status) == 0
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+    got = y16.float().cpu().numpy().astype(np.float64)
+    h_hat = O.dequantize_1x128(h_q, h_s)
+    written = np.zeros(rows, bool)
+    flips = 0
+    for g in range(n_groups):
+        st, n = starts[g], group_rows[g]
+        written[st:st + n] = True
+        if n == 0:
+            continue
+        ref = h_hat[st:st + n] @ O.dequantize_128x128(q2[g], s2[g]).T
+        flips += H.check_bf16(got[st:st + n], ref, f"group {g}")
+    assert np.all(got[~written] == 3.0)

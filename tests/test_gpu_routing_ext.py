@@ -106,8 +106,7 @@ def test_forward_with_node_limited_routing():
     gid = layer.ids.cpu().numpy()
     o_ids, _, _, score, gscore = O.route_grouped(case.x, case.gate_w, case.bias, w.K, 8, 4)
     _reconcile_grouped(gid, o_ids, score, gscore, w.K, 8, 4)
-    ref = O.moe_forward(case.x, case.gate_w, case.bias, w.K, case.ew, mode="Q", ids=gid)
-    H.check_rows(y, ref["y"])
+    H.expert_path_parity(w, case, layer, y, gid, np.arange(w.T))
 
 
 @pytest.mark.parametrize("t_count,seq_len", [(1000, 300), (4096, 4096), (77, 1)])
@@ -159,3 +158,76 @@ def test_bias_controller_trajectory():
         assert np.array_equal(bd.cpu().numpy(), bias), step
     # the oracle alone on this router goes from 5.8 to 1.1 in 30 steps
     assert ratios[0] > 3.0 and ratios[-1] < 0.4 * ratios[0], ratios
+
+
+def test_bias_controller_v3_skewed_50_steps():
+    """The skewed workload at the V3 shape (T = 8192, N = 256, K = 8, Zipf-
+    ranked logits), 50 route + bias-update steps from b = 0 with gamma = 1e-3
+    on the same batch, as the benchmark's controller trace runs them
+    ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing...", section III,
+    "How the bias is set"). At every step the GPU bias equals the oracle's
+    fp32 update of the previous bias with the GPU's counts, bit for bit; at
+    the first, a middle and the last step the counts are those of the
+    oracle's routing under the current bias (near-tie rule); the max/mean
+    load falls."""
+    w = I.WORKLOADS["skewed"]
+    xb = I.make_x(w)
+    x, gw = I.bf16_bits_to_f32(xb), I.make_gate_w(w)
+    sh = capi.shape_of(w.T, w.H, w.N, w.K, w.I)
+    ws = torch.empty(capi.moe_workspace_size(sh), dtype=torch.uint8, device="cuda")
+    ids = torch.empty((w.T, w.K), dtype=torch.int32, device="cuda")
+    gates = torch.empty((w.T, w.K), dtype=torch.float32, device="cuda")
+    counts = torch.empty((w.N,), dtype=torch.int32, device="cuda")
+    gwd, xd = torch.from_numpy(gw).cuda(), H.x_to_device(xb)
+    bias = np.zeros(w.N, np.float32)
+    bd = torch.from_numpy(bias).cuda()
+    ratios = []
+    for step in range(w.steps):
+        capi.moe_route(sh, gwd, xd, bd, ids, gates, counts, ws)
+        c = counts.cpu().numpy()
+        assert c.sum() == w.T * w.K
+        if step in (0, w.steps // 2, w.steps - 1):
+            o_ids, _, _, score = O.route(x, gw, bias, w.K)
+            use, _, _ = H.reconcile_ids(ids.cpu().numpy(), o_ids, score, w.K)
+            assert np.array_equal(c, O.expert_counts(use, w.N)), step
+        ratios.append(c.max() / c.mean())
+        capi.moe_update_bias(bd, counts, w.N, w.T, w.K, w.gamma)
+        bias = O.update_bias(bias, c, w.T, w.K, w.gamma)
+        assert np.array_equal(bd.cpu().numpy(), bias), step
+    assert capi.moe_get_status(ws) == 0
+    assert ratios[-1] < ratios[0], ratios
+
+
+def test_bias_controller_resumes_from_a_saved_bias(tmp_path):
+    """Route + update 8 steps on the GPU in one go, and again with the bias
+    saved to a file after step 3 and loaded into a fresh device tensor: the
+    final bias and the last step's ids agree bit for bit."""
+    from mixture_experts_layer_40_b200.layer import load_bias, save_bias
+    w = I.Workload("resume", T=1024, H=512, N=32, K=4, I=128, bias_range=0.0, seed=31,
+                   zipf_s=1.2, zipf_alpha=4.0)
+    xb = I.make_x(w)
+    gw = torch.from_numpy(I.make_gate_w(w)).cuda()
+    xd = H.x_to_device(xb)
+    sh = capi.shape_of(w.T, w.H, w.N, w.K, w.I)
+    ws = torch.empty(capi.moe_workspace_size(sh), dtype=torch.uint8, device="cuda")
+    ids = torch.empty((w.T, w.K), dtype=torch.int32, device="cuda")
+    gates = torch.empty((w.T, w.K), dtype=torch.float32, device="cuda")
+    counts = torch.empty((w.N,), dtype=torch.int32, device="cuda")
+
+    def steps(bias, n):
+        for _ in range(n):
+            capi.moe_route(sh, gw, xd, bias, ids, gates, counts, ws)
+            capi.moe_update_bias(bias, counts, w.N, w.T, w.K, 5e-3)
+
+    b1 = torch.zeros(w.N, dtype=torch.float32, device="cuda")
+    steps(b1, 8)
+    ids1 = ids.clone()
+    b2 = torch.zeros(w.N, dtype=torch.float32, device="cuda")
+    steps(b2, 3)
+    save_bias(str(tmp_path / "b.bin"), b2, 3, 5e-3)
+    b3, step, _ = load_bias(str(tmp_path / "b.bin"), "cuda")
+    assert step == 3
+    steps(b3, 5)
+    assert torch.equal(b1.view(torch.int32), b3.view(torch.int32))
+    assert torch.equal(ids1, ids)
+    assert capi.moe_get_status(ws) == 0
