@@ -85,3 +85,18 @@ def test_cpu_baseline_builds_the_pools_before_timing():
     w = I.WORKLOADS["tiny"]
     _, _, _, ew = bench.oracle_setup(w, I.make_x(w))
     assert getattr(ew, "_deq", None) is not None
+
+
+def test_roofline_bound_follows_the_ridge():
+    """An HBM-bound launch (V3 prefill's up GEMM: about 300 FLOP per byte,
+    below the ridge of 3160 TFLOP/s over 6650 GB/s) is reported in GB/s; a
+    compute-bound one (the same GEMM at T = 32768, about 1900 FLOP per byte)
+    in TFLOP/s against the FP8 peak."""
+    up = bench.algorithmic_work(I.WORKLOADS["v3_prefill"], np.ones(256))["expert_up"]
+    r = bench.roofline_of(up, 1.0, 6650.0, 3160.0)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - up["bytes"] / 1e-3 / 1e9) < 1e-6 * r["achieved"]
+    big = bench.algorithmic_work(I.WORKLOADS["large_prefill"], np.ones(256))["expert_up"]
+    r = bench.roofline_of(big, 10.0, 6650.0, 3160.0)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["frac"] - big["flops"] / 1e-2 / 1e12 / 3160.0) < 1e-9
