@@ -115,19 +115,21 @@ cudaError_t make_tmap_f32(CUtensorMap* map, const void* base, int64_t inner, int
 }
 
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
-                           int64_t depth, int box_inner, int box_rows) {
+                           int64_t depth, int box_inner, int box_rows, int box_depth) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return cudaErrorNotSupported;
   const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)(rows > 0 ? rows : 1),
                               (cuuint64_t)(depth > 0 ? depth : 1)};
   const cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)(inner * 2 * (rows > 0 ? rows : 1))};
-  const cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+  const cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows,
+                             (cuuint32_t)(box_depth > 0 ? box_depth : 1)};
   const cuuint32_t estr[3] = {1, 1, 1};
   const cuuint32_t rank = depth > 1 ? 3 : 2;
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        box_inner * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 

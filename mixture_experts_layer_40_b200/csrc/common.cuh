@@ -122,6 +122,15 @@ MOE_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_
       : "memory");
 }
 
+// Prefetch of a tensor-map tile into L2 (no shared memory, no completion):
+// a later tma_load_2d of the same tile then finds it in L2.
+MOE_DEV void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // TMA tile store from shared memory (bulk-group completion). The writing
 // threads must have made their shared-memory stores visible to the async
 // proxy (fence_proxy_async_smem) before one thread issues the copy.
@@ -242,6 +251,18 @@ MOE_DEV uint64_t smem_desc_sw128(uint32_t smem_addr) {
   d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: 8 rows x 128 B
   d |= (uint64_t)1 << 46;                        // descriptor version for sm_100
   d |= (uint64_t)2 << 61;                        // 128-byte swizzle
+  return d;
+}
+
+// The same for tiles written by TMA with 64-byte swizzling: rows of 64 bytes,
+// 8-row groups 512 bytes apart.
+MOE_DEV uint64_t smem_desc_sw64(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);  // start address
+  d |= (uint64_t)1 << 16;                        // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(512 >> 4) << 32;               // stride byte offset: 8 rows x 64 B
+  d |= (uint64_t)1 << 46;                        // descriptor version for sm_100
+  d |= (uint64_t)4 << 61;                        // 64-byte swizzle
   return d;
 }
 

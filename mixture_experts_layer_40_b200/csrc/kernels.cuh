@@ -20,14 +20,16 @@ struct GroupedGemm {
 // box_inner bytes x box_rows rows, 128-byte swizzle (host side).
 cudaError_t make_tmap_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
                          int box_inner, int box_rows);
-// bf16 tensor map over [depth, rows, inner] (depth 1: 2-D), box of box_inner
-// elements x box_rows rows x 1, 128-byte swizzle (host side).
+
 // fp32 [rows, inner] row-major; the swizzle span is the box row (box_inner * 4
 // bytes: 32, 64 or 128)
 cudaError_t make_tmap_f32(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
                           int box_inner, int box_rows);
+// bf16 tensor map over [depth, rows, inner] (depth 1: 2-D), box of box_inner
+// elements x box_rows rows x box_depth; 64-byte swizzle for 32-element box
+// rows, 128-byte swizzle otherwise (host side).
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t rows,
-                           int64_t depth, int box_inner, int box_rows);
+                           int64_t depth, int box_inner, int box_rows, int box_depth = 1);
 
 // The sizes every entry point accepts (see moe_shape in moe_capi.h).
 bool shape_ok(const moe_shape& s);

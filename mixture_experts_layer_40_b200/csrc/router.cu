@@ -102,6 +102,9 @@ MOE_DEV void warp_argmax(float& best, int& bid) {
 // the sum of its K/M highest biased scores (taken in descending order), the
 // M best groups are kept (lower group id on ties) and every expert outside
 // them is masked out of the selection.
+// kPerLane: a compile-time bound on the scores each lane holds (N <= 32 *
+// kPerLane), so that the per-lane arrays stay in registers.
+template <int kPerLane>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
                                                    const float* __restrict__ bias, int T, int N,
                                                    int K, int G, int M,
@@ -112,9 +115,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
   const int warps = blockDim.x >> 5;
   const int per_lane = (N + 31) >> 5;
   for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
-    float sc[kMaxPerLane], sv[kMaxPerLane];
+    float sc[kPerLane], sv[kPerLane];
 #pragma unroll
-    for (int j = 0; j < kMaxPerLane; ++j) {
+    for (int j = 0; j < kPerLane; ++j) {
       sc[j] = -INFINITY;
       sv[j] = 0.0f;
       const int e = lane + 32 * j;
@@ -135,7 +138,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
           float best = -INFINITY;
           int bid = N, bj = -1;
 #pragma unroll
-          for (int j = 0; j < kMaxPerLane; ++j) {
+          for (int j = 0; j < kPerLane; ++j) {
             const int e = lane + 32 * j;
             if (j < per_lane && e < N && e / size == g && !((used >> j) & 1u) &&
                 (sc[j] > best || (sc[j] == best && e < bid))) {
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
         keep |= 1u << bid;
       }
 #pragma unroll
-      for (int j = 0; j < kMaxPerLane; ++j) {
+      for (int j = 0; j < kPerLane; ++j) {
         const int e = lane + 32 * j;
         if (j < per_lane && e < N && !((keep >> (e / size)) & 1u)) sc[j] = -INFINITY;
       }
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
       float best = -INFINITY, best_s = 0.0f;
       int bid = N, bj = -1;
 #pragma unroll
-      for (int j = 0; j < kMaxPerLane; ++j) {
+      for (int j = 0; j < kPerLane; ++j) {
         const int e = lane + 32 * j;
         if (j < per_lane && e < N && !((taken >> j) & 1u) && (sc[j] > best || (sc[j] == best && e < bid))) {
           best = sc[j];
@@ -206,6 +209,25 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
       atomicAdd(&counts[my_id], 1);
     }
   }
+}
+
+// Top-K over the logits with the smallest per-lane bound that holds N.
+cudaError_t launch_topk(const float* logits, const float* bias, int T, int N, int K, int G, int M,
+                        int32_t* ids, float* gates, int32_t* counts, cudaStream_t stream,
+                        int sm_count) {
+  int blocks = (T + 7) / 8;
+  if (blocks > sm_count * 8) blocks = sm_count * 8;
+  const int per_lane = (N + 31) / 32;
+  if (per_lane <= 4)
+    topk_kernel<4><<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, G, M, ids, gates, counts);
+  else if (per_lane <= 8)
+    topk_kernel<8><<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, G, M, ids, gates, counts);
+  else if (per_lane <= 16)
+    topk_kernel<16><<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, G, M, ids, gates, counts);
+  else
+    topk_kernel<kMaxPerLane><<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, G, M, ids, gates,
+                                                        counts);
+  return cudaGetLastError();
 }
 
 // Sequence-wise balance statistics in three passes, every sum in a fixed
@@ -338,10 +360,7 @@ cudaError_t launch_router(const void* x, const float* gate_w, const float* bias,
                                         logits);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  int blocks = (T + 7) / 8;
-  if (blocks > sm_count * 8) blocks = sm_count * 8;
-  topk_kernel<<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, G, M, ids, gates, counts);
-  return cudaGetLastError();
+  return launch_topk(logits, bias, T, N, K, G, M, ids, gates, counts, stream, sm_count);
 }
 
 }  // namespace moe
@@ -509,9 +528,170 @@ __global__ void __launch_bounds__(kRThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, kRN);
 }
 
+// Wide tiles for large batches: one CTA computes 256 tokens x 256 experts
+// (two 128-row fp32 accumulators in TMEM, 512 columns, sharing each k-block's
+// centroid tile), so the split centroids are streamed once per 256 tokens
+// instead of once per 128 tokens and 64 experts. k-blocks are 32 bf16 wide
+// (64-byte rows, 64-byte swizzle) to fit three stages of x (16 KB) and the
+// three centroid terms (48 KB).
+constexpr int kWM = 256;                  // tokens per tile (two accumulators)
+constexpr int kWN = 256;                  // experts per tile
+constexpr int kWK = 32;                   // bf16 elements per k-block (64 bytes)
+constexpr int kWStages = 3;
+constexpr int kWABytes = kWM * kWK * 2;   // 16 KB
+constexpr int kWBBytes = kWN * kWK * 2;   // 16 KB per split term
+constexpr int kWStageBytes = kWABytes + 3 * kWBBytes;
+constexpr int kWThreads = 384;
+constexpr uint32_t kWIdesc = make_idesc(128, kWN, 1u, 1u);  // BF16 x BF16 -> fp32
+constexpr size_t kWDynSmem = (size_t)kWStages * kWStageBytes + 1024;
+
+struct alignas(8) WideShared {
+  uint64_t full[kWStages];
+  uint64_t empty[kWStages];
+  uint64_t tfull;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Warps: 0 TMA producer, 1 TMEM allocator and MMA issuer, 2-3 idle, 4-11
+// epilogue (warpgroup h reads accumulator h: tokens 128h .. 128h + 127).
+__global__ void __launch_bounds__(kWThreads, 1)
+    logits_tc_wide_kernel(const __grid_constant__ CUtensorMap tm_x,
+                          const __grid_constant__ CUtensorMap tm_w, int T, int H, int N,
+                          float* __restrict__ z, uint32_t* __restrict__ status) {
+  __shared__ WideShared sh;
+  extern __shared__ uint8_t dyn_smem[];
+  const uint32_t ring = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kWM;
+  const int n0 = blockIdx.y * kWN;
+  const int kb_n = H / kWK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kWStages; ++s) {
+      mbar_init(smem_u32(&sh.full[s]), 1);
+      mbar_init(smem_u32(&sh.empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sh.tfull), 1);
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tm_x);
+    prefetch_tensormap(&tm_w);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(&sh.tmem_base), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sh.tmem_base;
+  volatile int* abort = &sh.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // producer: 256 rows of x and the three centroid terms of every k-block
+      int kb = 0;
+      for (; kb < kb_n; ++kb) {
+        const int s = kb % kWStages;
+        const uint32_t ph = (uint32_t)(kb / kWStages) & 1u;
+        if (!mbar_wait(smem_u32(&sh.empty[s]), ph ^ 1u, abort, status)) break;
+        const uint32_t full = smem_u32(&sh.full[s]);
+        mbar_arrive_expect_tx(full, kWStageBytes);
+        const uint32_t sa = ring + s * kWStageBytes;
+        tma_load_2d(sa, &tm_x, kb * kWK, m0, full);
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(sa + kWABytes),
+            "l"(reinterpret_cast<uint64_t>(&tm_w)), "r"(kb * kWK), "r"(n0), "r"(0), "r"(full)
+            : "memory");
+      }
+      if (kb < kb_n) {
+        for (int s = 0; s < kWStages && s < kb; ++s) {
+          const int last = s + ((kb - 1 - s) / kWStages) * kWStages;
+          mbar_wait(smem_u32(&sh.full[s]), (uint32_t)(last / kWStages) & 1u, nullptr, status);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // MMA issuer: per k-block, each 128-token half against the three terms,
+      // two K=16 steps each, all into that half's fp32 accumulator
+      bool ok = true;
+      bool issued = false;
+      for (int kb = 0; kb < kb_n; ++kb) {
+        const int s = kb % kWStages;
+        const uint32_t ph = (uint32_t)(kb / kWStages) & 1u;
+        if (!mbar_wait(smem_u32(&sh.full[s]), ph, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = ring + s * kWStageBytes;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int t = 0; t < 3; ++t) {
+#pragma unroll
+            for (int k = 0; k < kWK / 16; ++k) {
+              mma_bf16(tmem_base + (uint32_t)(h * kWN),
+                       smem_desc_sw64(sa + h * (kWABytes / 2) + k * 32),
+                       smem_desc_sw64(sa + kWABytes + t * kWBBytes + k * 32), kWIdesc,
+                       (kb | t | k) != 0 ? 1u : 0u);
+            }
+          }
+        }
+        issued = true;
+        mma_commit(smem_u32(&sh.empty[s]));
+      }
+      if (issued) mma_commit(smem_u32(&sh.tfull));
+      if (!ok && issued) mbar_wait(smem_u32(&sh.tfull), 0u, nullptr, status);
+    }
+  } else if (warp >= 4) {
+    // epilogue: each thread one token's 256 fp32 logits -> z
+    const int h = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int t = m0 + h * 128 + quarter * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh.tfull), 0u, abort, status));
+    if (ok) {
+      tc_fence_after();
+      const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(h * kWN);
+      const int cols = min(kWN, N - n0);
+      float* dst = z + (int64_t)t * N + n0;
+#pragma unroll 1
+      for (int c = 0; c < kWN; c += 32) {
+        float v[32];
+        tmem_ld32(t0 + (uint32_t)c, v);
+        tmem_wait_ld();
+        if (t < T) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c + 4 * j < cols)
+              reinterpret_cast<float4*>(dst + c)[j] =
+                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
 }  // namespace
 
 size_t router_split_bytes(int N, int H) { return (size_t)3 * N * H * sizeof(__nv_bfloat16); }
+
+// Wide tiles move about 3.2x the bytes of a 128 x 64 tile through L2 for 8x
+// its logits; they pay off once the small tiles would need more than 3.2
+// times as many waves as the wide ones (T = 32768 at N = 256: 7 against 1).
+static bool use_wide_logits(int64_t T, int64_t N, int sm_count) {
+  if (N % kWN != 0) return false;  // whole 256-expert tiles only
+  const int64_t sms = sm_count > 0 ? sm_count : 148;
+  const int64_t small = ((T + kRM - 1) / kRM) * ((N + kRN - 1) / kRN);
+  const int64_t wide = ((T + kWM - 1) / kWM) * ((N + kWN - 1) / kWN);
+  const int64_t small_waves = (small + sms - 1) / sms;
+  const int64_t wide_waves = (wide + sms - 1) / sms;
+  return 10 * small_waves > 32 * wide_waves;
+}
 
 cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
                              int N, int K, int G, int M, __nv_bfloat16* wsplit, float* logits,
@@ -523,25 +703,36 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
                       stream>>>(gate_w, nw, wsplit);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap mx, mw;
-  e = make_tmap_bf16(&mx, x, H, T, 1, kRK, kRM);
-  if (e != cudaSuccess) return e;
-  e = make_tmap_bf16(&mw, wsplit, H, N, 3, kRK, kRN);
-  if (e != cudaSuccess) return e;
-  static DeviceOnce once;  // the shared-memory limit is raised once per device
+  static DeviceOnce once;  // the shared-memory limits are raised once per device
   e = once.run([] {
-    return cudaFuncSetAttribute(logits_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kRDynSmem);
+    cudaError_t r = cudaFuncSetAttribute(logits_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kRDynSmem);
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(logits_tc_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kWDynSmem);
   });
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((T + kRM - 1) / kRM), (unsigned)((N + kRN - 1) / kRN));
-  logits_tc_kernel<<<grid, kRThreads, kRDynSmem, stream>>>(mx, mw, T, H, N, logits, status);
+  CUtensorMap mx, mw;
+  if (use_wide_logits(T, N, sm_count)) {
+    e = make_tmap_bf16(&mx, x, H, T, 1, kWK, kWM);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_bf16(&mw, wsplit, H, N, 3, kWK, kWN, 3);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((T + kWM - 1) / kWM), (unsigned)((N + kWN - 1) / kWN));
+    logits_tc_wide_kernel<<<grid, kWThreads, kWDynSmem, stream>>>(mx, mw, T, H, N, logits,
+                                                                  status);
+  } else {
+    e = make_tmap_bf16(&mx, x, H, T, 1, kRK, kRM);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_bf16(&mw, wsplit, H, N, 3, kRK, kRN);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((T + kRM - 1) / kRM), (unsigned)((N + kRN - 1) / kRN));
+    logits_tc_kernel<<<grid, kRThreads, kRDynSmem, stream>>>(mx, mw, T, H, N, logits, status);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  int blocks = (T + 7) / 8;
-  if (blocks > sm_count * 8) blocks = sm_count * 8;
-  topk_kernel<<<blocks, 256, 0, stream>>>(logits, bias, T, N, K, G, M, ids, gates, counts);
-  return cudaGetLastError();
+  return launch_topk(logits, bias, T, N, K, G, M, ids, gates, counts, stream, sm_count);
 }
 
 }  // namespace moe

@@ -96,8 +96,10 @@ def _route(capi, w, x_bits, gate_w, bias):
     return ids.cpu().numpy(), gates.cpu().numpy(), counts.cpu().numpy()
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "v3_prefill", "skewed"])
+@pytest.mark.parametrize("name", ["tiny", "decode", "v3_prefill", "skewed", "large_prefill"])
 def test_route_parity(capi, name):
+    """large_prefill (T = 32768) takes the wide-tile logits kernel (256 tokens x
+    256 experts per CTA), the others the 128 x 64 tiles."""
     w = I.WORKLOADS[name]
     xb = I.make_x(w)
     gate_w, bias = I.make_gate_w(w), I.make_bias(w)
