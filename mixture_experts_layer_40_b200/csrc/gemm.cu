@@ -8,8 +8,8 @@
 // while a second WGMMA group computes; here every 128-deep k-block is
 // accumulated by the tensor core into its own TMEM buffer (two buffers, ping-
 // pong) and eight epilogue warps read it back with tcgen05.ld and add
-// partial * 1/(s_a s_b) into fp32 register totals while the tensor core fills
-// the other buffer.
+// partial * 1/(s_a s_b) into fp32 register totals (packed in pairs, two-lane
+// FMAs) while the tensor core fills the other buffer.
 //
 // One persistent CTA per SM, 384 threads (three warpgroups):
 //   warp 0     TMA producer: A (128 rows x 128 B) and B (256 rows x 128 B)
@@ -21,7 +21,7 @@
 //              so each warpgroup covers the 128 rows of a tile and owns half
 //              of its 256 columns
 // The first warpgroup gives registers back (setmaxnreg) so that each epilogue
-// thread can hold 128 fp32 totals plus two 32-column partial chunks.
+// thread can hold 128 fp32 totals plus a 64-column partial chunk.
 // Tiles are (group, m-tile, n-tile) with n fastest: the n-tiles of one row
 // tile run on neighbouring CTAs at the same time and share its A rows in L2.
 // Both operands load with the default L2 policy: with the weight stream
@@ -246,13 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t sa = ring + s * kStageBytes;
           const uint32_t d = tmem_base + (uint32_t)(buf * kBN);
+          const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sa + kABytes);
 #pragma unroll
           for (int k4 = 0; k4 < kBK / 32; ++k4) {
-            mma_f8(d, smem_desc_sw128(sa + k4 * 32), smem_desc_sw128(sa + kABytes + k4 * 32), kIdesc,
-                   k4 > 0 ? 1u : 0u);
+            // +32 bytes along K = +2 in the descriptor's 16-byte address field
+            mma_f8(d, da + (uint64_t)(2 * k4), db + (uint64_t)(2 * k4), kIdesc, k4 > 0 ? 1u : 0u);
           }
-          mma_commit(smem_u32(&sh.empty[s]));
           mma_commit(smem_u32(&sh.tfull[buf]));
+          mma_commit(smem_u32(&sh.empty[s]));
         }
       }
       if (!ok && kbi > 0) {
@@ -273,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kbi = 0;
     uint32_t xchg_phase = 0;
     int tile_count = 0;
-    float acc[128];
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tile_count) {
+      uint64_t acc2[64];  // the 128 fp32 totals as packed pairs
       int g, n, m;
       decode_tile(tile, sh.prefix, p.n_groups, p.n_tiles, g, n, m);
       const int valid = p.group_rows[g] - m * kBM;
@@ -284,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* sb0 = p.b_s + ((int64_t)g * b_blocks + 2 * n + (kUp ? 0 : eg)) * kb_n;
       const float* sb1 = p.b_s + ((int64_t)g * b_blocks + 2 * n + 1) * kb_n;
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      for (int i = 0; i < 64; ++i) acc2[i] = 0ull;
       float sa_next = ldg_early(sa_ptr);
       float sb0_next = ldg_early(sb0);
       float sb1_next = kUp ? ldg_early(sb1) : 0.0f;
@@ -311,26 +312,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // [128+64eg, ...); down -> [128eg, 128eg+128)
         const uint32_t c0 = kUp ? (uint32_t)(64 * eg) : (uint32_t)(128 * eg);
         const uint32_t c2 = kUp ? (uint32_t)(128 + 64 * eg) : (uint32_t)(128 * eg + 64);
-        float v0[32], v1[32];
-        tmem_ld32(t0 + c0, v0);
-        tmem_ld32(t0 + c0 + 32, v1);
+        float v[64];
+        tmem_ld64(t0 + c0, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) fma_f32x2(acc[i], acc[i + 1], v0[i], v0[i + 1], inv0x2);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) fma_f32x2(acc[32 + i], acc[33 + i], v1[i], v1[i + 1], inv0x2);
-        tmem_ld32(t0 + c2, v0);
-        tmem_ld32(t0 + c2 + 32, v1);
+        for (int i = 0; i < 64; i += 2) fma_f32x2(acc2[i / 2], v[i], v[i + 1], inv0x2);
+        tmem_ld64(t0 + c2, v);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sh.tempty[buf]));
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) fma_f32x2(acc[64 + i], acc[65 + i], v0[i], v0[i + 1], inv1x2);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) fma_f32x2(acc[96 + i], acc[97 + i], v1[i], v1[i + 1], inv1x2);
+        for (int i = 0; i < 64; i += 2) fma_f32x2(acc2[32 + i / 2], v[i], v[i + 1], inv1x2);
       }
       if (!ok) break;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) unpack_f32x2(acc2[i], acc[2 * i], acc[2 * i + 1]);
 
       if (kUp) {
         // h = silu(G) * U for this thread's 64 channels, then 1x128 re-quantisation;
