@@ -96,7 +96,12 @@ typedef struct {
  *   s13    [N+1, 2I/128, H/128] float32 block scales of w13 (same row order)
  *   w2     [N+1, H, I]         E4M3 W_down
  *   s2     [N+1, H/128, I/128] float32 block scales of w2
- * w13 and w2 must be 16-byte aligned.
+ *   gate_split  optional (NULL: made on every call): bf16 [3, N, H], gate_w
+ *               split exactly into three bf16 terms by moe_split_gate. The
+ *               tensor-core router multiplies these; with them given,
+ *               moe_forward skips the split. The caller re-splits whenever
+ *               gate_w changes (after every optimiser step, in training).
+ * w13 and w2 must be 16-byte aligned; gate_split 16-byte aligned.
  */
 typedef struct {
   const float* gate_w;
@@ -104,6 +109,7 @@ typedef struct {
   const float* s13;
   const uint8_t* w2;
   const float* s2;
+  const void* gate_split;
 } moe_weights;
 
 /*
@@ -161,6 +167,15 @@ int moe_quantize_1x128(const void* x, int64_t rows, int64_t cols, uint8_t* q, fl
  */
 int moe_quantize_128x128(const float* w, int64_t rows, int64_t cols, uint8_t* q, float* scales,
                          void* stream);
+
+/*
+ * The fp32 centroids as three bf16 terms, hi + mid + lo == gate_w exactly
+ * (each term the bf16 rounding of what the previous ones leave), for
+ * moe_weights.gate_split: gate_w float [N, H] -> gate_split bf16 [3, N, H]
+ * (term-major). Done once at set-up, or after every change of gate_w.
+ * Both 16-byte aligned; N >= 1, H >= 1.
+ */
+int moe_split_gate(const float* gate_w, int32_t N, int32_t H, void* gate_split, void* stream);
 
 /* Workspace bytes needed by moe_route / moe_forward for `sh` (0 if invalid). */
 size_t moe_workspace_size(moe_shape sh);

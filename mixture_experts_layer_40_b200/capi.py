@@ -36,7 +36,7 @@ class moe_shape(ctypes.Structure):
 
 class moe_weights(ctypes.Structure):
     _fields_ = [("gate_w", ctypes.c_void_p), ("w13", ctypes.c_void_p), ("s13", ctypes.c_void_p),
-                ("w2", ctypes.c_void_p), ("s2", ctypes.c_void_p)]
+                ("w2", ctypes.c_void_p), ("s2", ctypes.c_void_p), ("gate_split", ctypes.c_void_p)]
 
 
 _LAYOUT_FIELDS = ["status", "counts", "offsets", "group_rows", "row_start", "row_token",
@@ -57,6 +57,7 @@ SIGNATURES = {
     "moe_quantize_128x128": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "moe_workspace_size": (_SZ, [moe_shape]),
     "moe_workspace_layout": (ctypes.c_int, [moe_shape, ctypes.POINTER(moe_ws_layout)]),
+    "moe_split_gate": (ctypes.c_int, [_P, _I32, _I32, _P, _P]),
     "moe_route": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_route_noalloc": (ctypes.c_int, [moe_shape, _P, _P, _P, _P, _P, _P, _P]),
     "moe_balance_stats": (ctypes.c_int, [moe_shape, ctypes.c_int32, ctypes.c_float, _P, _SZ, _P,
@@ -216,10 +217,19 @@ def moe_route_noalloc(sh: moe_shape, gate_w, x, bias, topk_ids, topk_gates, coun
         _stream(stream)))
 
 
-def make_weights(gate_w, w13, s13, w2, s2) -> moe_weights:
+def make_weights(gate_w, w13, s13, w2, s2, gate_split=None) -> moe_weights:
     return moe_weights(_ptr(gate_w, torch.float32, "gate_w"), _ptr(w13, torch.uint8, "w13"),
                        _ptr(s13, torch.float32, "s13"), _ptr(w2, torch.uint8, "w2"),
-                       _ptr(s2, torch.float32, "s2"))
+                       _ptr(s2, torch.float32, "s2"),
+                       None if gate_split is None else _ptr(gate_split, torch.bfloat16,
+                                                            "gate_split"))
+
+
+def moe_split_gate(gate_w, gate_split, stream=None):
+    N, H = gate_w.shape
+    _check("moe_split_gate", LIB.moe_split_gate(
+        _ptr(gate_w, torch.float32, "gate_w"), N, H, _ptr(gate_split, torch.bfloat16, "gate_split"),
+        _stream(stream)))
 
 
 def moe_forward(sh: moe_shape, w: moe_weights, x, bias, y, topk_ids=None, topk_gates=None,

@@ -161,6 +161,14 @@ int moe_quantize_128x128(const float* w, int64_t rows, int64_t cols, uint8_t* q,
       launch_quantize_128x128(w, rows, cols, q, scales, static_cast<cudaStream_t>(stream)));
 }
 
+int moe_split_gate(const float* gate_w, int32_t N, int32_t H, void* gate_split, void* stream) {
+  if (!gate_w || !gate_split) return MOE_ERR_NULL;
+  if (N < 1 || H < 1) return MOE_ERR_SHAPE;
+  if (!aligned(gate_w, 16) || !aligned(gate_split, 16)) return MOE_ERR_ALIGN;
+  return cuda_status(launch_split_gate(gate_w, N, H, static_cast<__nv_bfloat16*>(gate_split),
+                                       static_cast<cudaStream_t>(stream), sm_count()));
+}
+
 size_t moe_workspace_size(moe_shape sh) {
   if (!shape_ok(sh)) return 0;
   moe_ws_layout L;
@@ -238,7 +246,7 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   if (!w || !x || !bias || !y || !ws) return MOE_ERR_NULL;
   if (!w->gate_w || !w->w13 || !w->s13 || !w->w2 || !w->s2) return MOE_ERR_NULL;
   if (!aligned(x, 16) || !aligned(y, 16) || !aligned(w->gate_w, 16) || !aligned(w->w13, 16) ||
-      !aligned(w->w2, 16) || !aligned(ws, 256))
+      !aligned(w->w2, 16) || !aligned(ws, 256) || !aligned(w->gate_split, 16))
     return MOE_ERR_ALIGN;
   moe_ws_layout L;
   layout_of(sh, &L);
@@ -274,7 +282,8 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   if (e == cudaSuccess)
     e = launch_router_tc(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                          at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
-                         counts, status, s, sms);
+                         counts, status, s, sms,
+                         static_cast<const __nv_bfloat16*>(w->gate_split));
   e = mark(1, e);
   // a6-a7: offsets, stable expert-major scatter of the (token, slot) pairs
   if (e == cudaSuccess)

@@ -49,11 +49,16 @@ cudaError_t launch_router(const void* x, const float* gate_w, const float* bias,
 // Router on tensor cores: splits the fp32 centroids into three bf16 terms in
 // `wsplit` (router_split_bytes), computes the logits with BF16 tcgen05 MMAs
 // and fp32 accumulation, then the same top-K as launch_router.
+// presplit: the three terms made earlier (launch_split_gate); NULL: split
+// into wsplit first.
 size_t router_split_bytes(int N, int H);
+cudaError_t launch_split_gate(const float* gate_w, int N, int H, __nv_bfloat16* wsplit,
+                              cudaStream_t stream, int sm_count);
 cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
                              int N, int K, int G, int M, __nv_bfloat16* wsplit, float* logits,
                              int32_t* ids, float* gates, int32_t* counts, uint32_t* status,
-                             cudaStream_t stream, int sm_count);
+                             cudaStream_t stream, int sm_count,
+                             const __nv_bfloat16* presplit = nullptr);
 
 // Backward of the expert path (backward.cu).
 cudaError_t launch_transpose_blocks(const uint8_t* w, const float* s, int64_t groups, int64_t rows,

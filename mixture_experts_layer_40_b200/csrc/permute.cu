@@ -94,11 +94,18 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
     offsets[e] = off;
     group_rows[e] = c;
     row_start[e] = start;
+    // eight chunks' counts are fetched before any is used, so the loads
+    // overlap instead of costing one memory latency per chunk
     int run = start;
-    for (int ch = 0; ch < n_chunks; ++ch) {
-      const int v = hist[(int64_t)ch * N + e];
-      hist[(int64_t)ch * N + e] = run;
-      run += v;
+    for (int ch0 = 0; ch0 < n_chunks; ch0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = ch0 + j < n_chunks ? hist[(int64_t)(ch0 + j) * N + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (ch0 + j < n_chunks) hist[(int64_t)(ch0 + j) * N + e] = run;
+        run += v[j];
+      }
     }
     if (run != start + c) flag_status(status, kStatusBounds);
   }

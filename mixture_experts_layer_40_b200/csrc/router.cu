@@ -693,16 +693,26 @@ static bool use_wide_logits(int64_t T, int64_t N, int sm_count) {
   return 10 * small_waves > 32 * wide_waves;
 }
 
+cudaError_t launch_split_gate(const float* gate_w, int N, int H, __nv_bfloat16* wsplit,
+                              cudaStream_t stream, int sm_count) {
+  const int64_t nw = (int64_t)N * H;
+  if (nw == 0) return cudaSuccess;
+  split_gate_kernel<<<(unsigned)std::min<int64_t>((nw + 255) / 256, (int64_t)sm_count * 8), 256, 0,
+                      stream>>>(gate_w, nw, wsplit);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
                              int N, int K, int G, int M, __nv_bfloat16* wsplit, float* logits,
                              int32_t* ids, float* gates, int32_t* counts, uint32_t* status,
-                             cudaStream_t stream, int sm_count) {
+                             cudaStream_t stream, int sm_count, const __nv_bfloat16* presplit) {
   if (T == 0) return cudaSuccess;
-  const int64_t nw = (int64_t)N * H;
-  split_gate_kernel<<<(unsigned)std::min<int64_t>((nw + 255) / 256, (int64_t)sm_count * 8), 256, 0,
-                      stream>>>(gate_w, nw, wsplit);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (presplit == nullptr) {
+    e = launch_split_gate(gate_w, N, H, wsplit, stream, sm_count);
+    if (e != cudaSuccess) return e;
+  }
+  const __nv_bfloat16* terms = presplit != nullptr ? presplit : wsplit;
   static DeviceOnce once;  // the shared-memory limits are raised once per device
   e = once.run([] {
     cudaError_t r = cudaFuncSetAttribute(logits_tc_kernel,
@@ -717,7 +727,7 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
   if (use_wide_logits(T, N, sm_count)) {
     e = make_tmap_bf16(&mx, x, H, T, 1, kWK, kWM);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16(&mw, wsplit, H, N, 3, kWK, kWN, 3);
+    e = make_tmap_bf16(&mw, terms, H, N, 3, kWK, kWN, 3);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((T + kWM - 1) / kWM), (unsigned)((N + kWN - 1) / kWN));
     logits_tc_wide_kernel<<<grid, kWThreads, kWDynSmem, stream>>>(mx, mw, T, H, N, logits,
@@ -725,7 +735,7 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
   } else {
     e = make_tmap_bf16(&mx, x, H, T, 1, kRK, kRM);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16(&mw, wsplit, H, N, 3, kRK, kRN);
+    e = make_tmap_bf16(&mw, terms, H, N, 3, kRK, kRN);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((T + kRM - 1) / kRM), (unsigned)((N + kRN - 1) / kRN));
     logits_tc_kernel<<<grid, kRThreads, kRDynSmem, stream>>>(mx, mw, T, H, N, logits, status);

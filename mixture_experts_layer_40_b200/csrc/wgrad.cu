@@ -10,7 +10,9 @@
 // The expert segments start 128-aligned and their padding rows hold zeros.
 //
 // Same machinery as the forward's grouped GEMM: one persistent CTA per SM,
-// warp 0 TMA producer (3-stage ring of 128x128 A and 256x128 B k-blocks),
+// warp 0 TMA producer (3-stage ring of 128x128 A and 256x128 B k-blocks and
+// B's 256 inverse column scales of the k-block; a stage is free again once
+// the MMA and the promotion warps have both used it),
 // warp 1 TMEM allocator and single-thread tcgen05 MMA issuer (two 256-column
 // TMEM buffers), warps 4-11 promotion and fp32 output through shared memory
 // and TMA stores. Every wait is bounded.
@@ -22,20 +24,24 @@ namespace moe {
 
 namespace {
 
-// 128-bit read-only load issued where it stands (the volatile asm keeps the
-// compiler from sinking it towards its first use).
-MOE_DEV float4 ldg_early4(const float4* p) {
-  float4 v;
-  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "l"(p));
-  return v;
+// Plain bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global to shared memory, completing on `bar`.
+MOE_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
 }
+
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
 constexpr int kStages = 3;  // two stages' worth of smem goes to output staging
 constexpr int kABytes = kBM * kBK, kBBytes = kBN * kBK;
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kSBytes = kBN * 4;  // the k-block's inverse column scales of B
+// a stage: A tile, B tile, then B's 256 inverse column scales (so that the
+// promotion reads them from shared memory, not with L2 latency per k-block)
+constexpr int kStageBytes = kABytes + kBBytes + 1024;
 constexpr int kThreads = 384;
 constexpr int kYCols = 32;                       // fp32 columns per TMA store
 constexpr int kYBufBytes = 32 * kYCols * 4;      // 32 rows x 128 bytes
@@ -92,7 +98,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&sh.full[s]), 1);
-      mbar_init(smem_u32(&sh.empty[s]), 1);
+      // released by the MMA's commit and by the 8 promotion warps once they
+      // have read the stage's column scales
+      mbar_init(smem_u32(&sh.empty[s]), 1 + 8);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&sh.tfull[b]), 1);
@@ -126,10 +134,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
           if (!mbar_wait(smem_u32(&sh.empty[s]), ph ^ 1u, abort, p.status)) { ok = false; break; }
           const uint32_t full = smem_u32(&sh.full[s]);
-          mbar_arrive_expect_tx(full, kStageBytes);
+          mbar_arrive_expect_tx(full, kABytes + kBBytes + kSBytes);
           const uint32_t sa = ring + s * kStageBytes;
           tma_load_2d(sa, &tm_a, (kb0 + kb) * kBK, m * kBM, full);
           tma_load_2d(sa + kABytes, &tm_b, (kb0 + kb) * kBK, n * kBN, full);
+          bulk_load(sa + kABytes + kBBytes, p.b_inv + (int64_t)(kb0 + kb) * p.N + n * kBN,
+                    kSBytes, full);
         }
       }
       if (!ok) {
@@ -192,32 +202,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int kb = 0; kb < kbn; ++kb, ++kbi) {
         const float inv_a = __fdividef(1.0f, ldg_early(sa_row + kb));
-        const float4* binv = reinterpret_cast<const float4*>(p.b_inv + (int64_t)(kb0 + kb) * p.N + x0);
-        // the column scales of each 32-column group (the same addresses in every
-        // lane) are requested before that group's accumulator load, the first
-        // group's before the wait for the accumulator, so their latency overlaps
-        float4 b[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) b[q] = ldg_early4(binv + q);
         const int buf = kbi & 1;
         ok = __all_sync(0xffffffffu,
                         mbar_wait(smem_u32(&sh.tfull[buf]), (uint32_t)(kbi >> 1) & 1u, abort, p.status));
         if (!ok) break;
         tc_fence_after();
+        // the MMA of this k-block has completed, so its stage is still held
+        // (the producer refills it only after these warps release it); the
+        // wait on its full barrier, long complete, makes the column scales'
+        // bulk copy visible to these threads
+        const int stage = kbi % kStages;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh.full[stage]),
+                                               (uint32_t)(kbi / kStages) & 1u, abort, p.status));
+        if (!ok) break;
+        const float4* binv = reinterpret_cast<const float4*>(
+            dyn_smem + (ring - smem_u32(dyn_smem)) + stage * kStageBytes + kABytes + kBBytes) +
+            (128 * eg) / 4;
         const uint32_t t0 = lane_addr + (uint32_t)(buf * kBN + 128 * eg);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if (j > 0) {
+          float4 b[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) b[q] = ldg_early4(binv + 8 * j + q);
-          }
+          for (int q = 0; q < 8; ++q) b[q] = binv[8 * j + q];
           float v[32];
           tmem_ld32(t0 + 32 * j, v);
           tmem_wait_ld();
           if (j == 3) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sh.tempty[buf]));
+            if (lane == 0) {
+              mbar_arrive(smem_u32(&sh.tempty[buf]));
+              mbar_arrive(smem_u32(&sh.empty[stage]));  // its column scales are read
+            }
           }
 #pragma unroll
           for (int q = 0; q < 8; ++q) {

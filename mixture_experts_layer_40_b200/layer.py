@@ -71,7 +71,7 @@ class MoELayer:
     """One layer: forward(x, bias) -> y through moe_forward."""
 
     def __init__(self, T: int, H: int, N: int, K: int, I: int, weights: DeviceWeights,
-                 device="cuda", groups: int = 0, topk_groups: int = 0):
+                 device="cuda", groups: int = 0, topk_groups: int = 0, presplit_gate: bool = True):
         self.T, self.H, self.N, self.K, self.I = T, H, N, K, I
         self.shape = capi.shape_of(T, H, N, K, I, groups, topk_groups)
         nbytes = capi.moe_workspace_size(self.shape)
@@ -82,8 +82,14 @@ class MoELayer:
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.ws[:16].zero_()
         self.weights = weights
+        # the centroids' three bf16 terms, made once here (resplit_gate after
+        # changing weights.gate_w); without them every forward splits again
+        self.gate_split = None
+        if presplit_gate:
+            self.gate_split = torch.empty((3, N, H), dtype=torch.bfloat16, device=self.device)
+            capi.moe_split_gate(weights.gate_w, self.gate_split)
         self._cw = capi.make_weights(weights.gate_w, weights.w13, weights.s13, weights.w2,
-                                     weights.s2)
+                                     weights.s2, self.gate_split)
         self.layout = capi.moe_workspace_layout(self.shape)
         self.ids = torch.empty((T, K), dtype=torch.int32, device=self.device)
         self.gates = torch.empty((T, K), dtype=torch.float32, device=self.device)
@@ -96,6 +102,11 @@ class MoELayer:
         capi.moe_forward(self.shape, self._cw, x, bias, y, self.ids, self.gates, self.counts,
                          self.ws, stream)
         return y
+
+    def resplit_gate(self, stream=None) -> None:
+        """Re-make the centroids' bf16 terms after weights.gate_w changed."""
+        if self.gate_split is not None:
+            capi.moe_split_gate(self.weights.gate_w, self.gate_split, stream)
 
     def route(self, x: torch.Tensor, bias: torch.Tensor, stream=None):
         capi.moe_route(self.shape, self.weights.gate_w, x, bias, self.ids, self.gates,

@@ -170,3 +170,26 @@ def test_forward_skewed_sampled():
     assert counts.max() > 4 * counts.mean()
     use_ids, _ = check_intermediates(w, case, layer, bias, sample_rows=_sampled(w, 5))
     check_output(w, case, layer, bias, y, use_ids, tokens=_sampled(w, 6))
+
+
+def test_forward_with_and_without_presplit_gate():
+    """The centroids' bf16 terms made once (moe_split_gate, moe_weights.gate_split)
+    or on every call give the same routing and output bits; after the
+    centroids change, resplit_gate follows them."""
+    w = I.Workload("split", T=333, H=512, N=32, K=4, I=256, bias_range=0.1, seed=17)
+    case = H.make_case(w)
+    dw = device_weights(w, case.pool, case.gate_w, "cuda")
+    xd = H.x_to_device(case.x_bits)
+    bd = torch.from_numpy(case.bias).cuda()
+    a = MoELayer(w.T, w.H, w.N, w.K, w.I, dw, presplit_gate=True)
+    b = MoELayer(w.T, w.H, w.N, w.K, w.I, dw, presplit_gate=False)
+    ya, yb = a.forward(xd, bd), b.forward(xd, bd)
+    assert a.status() == 0 and b.status() == 0
+    assert torch.equal(ya, yb) and torch.equal(a.ids, b.ids) and torch.equal(a.gates, b.gates)
+    # the split terms sum back to the centroids exactly
+    t = a.gate_split.double()
+    assert torch.equal(t[0] + t[1] + t[2], dw.gate_w.double())
+    dw.gate_w.mul_(-1.0)
+    a.resplit_gate()
+    ya, yb = a.forward(xd, bd), b.forward(xd, bd)
+    assert torch.equal(ya, yb) and torch.equal(a.ids, b.ids)

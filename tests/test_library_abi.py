@@ -109,3 +109,16 @@ def test_null_and_alignment_rejected(capi):
     assert capi.LIB.moe_quantize_128x128(16, 100, 128, 16, 16, None) == -1
     assert capi.LIB.moe_update_bias(None, 16, 16, 4, 2, 0.001, None) == -2
     assert capi.LIB.moe_expert_up(256, 128, 0, 16, 16, 128, 16, 16, 16, 16, 16, 16, None, None) == -1
+
+
+def test_split_gate_rejects_bad_arguments(capi):
+    lib = capi.LIB
+    # MOE_ERR_NULL = -2, MOE_ERR_SHAPE = -1, MOE_ERR_ALIGN = -7
+    assert lib.moe_split_gate(None, 16, 256, 16, None) == -2
+    assert lib.moe_split_gate(16, 16, 256, None, None) == -2
+    assert lib.moe_split_gate(16, 0, 256, 16, None) == -1
+    assert lib.moe_split_gate(8, 16, 256, 16, None) == -7
+    # a misaligned pre-split buffer in the weights is refused before any work
+    sh = capi.shape_of(64, 256, 16, 4, 128)
+    w = capi.moe_weights(16, 16, 16, 16, 16, 8)
+    assert lib.moe_forward(sh, ctypes.byref(w), 16, 16, 16, None, None, None, 256, 1 << 30, None) == -7
