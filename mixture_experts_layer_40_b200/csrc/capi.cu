@@ -277,17 +277,17 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
   };
   cudaError_t e = mark(0, cudaSuccess);
   if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, 4, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)sh.N * 4, s);
-  // a2-a5: gate logits, sigmoid, biased top-K, gates, counts (from bf16 x)
+  // a2-a5: gate logits, sigmoid, biased top-K, gates (from bf16 x)
   if (e == cudaSuccess)
     e = launch_router_tc(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                          at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
-                         counts, status, s, sms,
+                         nullptr, status, s, sms,
                          static_cast<const __nv_bfloat16*>(w->gate_split));
   e = mark(1, e);
-  // a6-a7: offsets, stable expert-major scatter of the (token, slot) pairs
+  // a6-a7: counts from per-chunk histograms, offsets, stable expert-major
+  // placement of the (token, slot) pairs
   if (e == cudaSuccess)
-    e = launch_permute(ids, counts, sh.T, sh.N, sh.K, (int64_t)sh.T * sh.K, L.routed_cap,
+    e = launch_permute(ids, counts, true, sh.T, sh.N, sh.K, (int64_t)sh.T * sh.K, L.routed_cap,
                        at<int32_t>(ws, L.perm_scratch), at<int32_t>(ws, L.offsets),
                        at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
                        at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.token_row), status, s,

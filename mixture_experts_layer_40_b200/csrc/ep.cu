@@ -617,7 +617,7 @@ int experts_impl(const moe_shape& sh, int W, const moe_weights* w_local, const u
       recv, R, sh.K, sh.H, rb, El, seg_rows, seg_counts, ids, gates, counts, status);
   e = cudaGetLastError();
   if (e == cudaSuccess)
-    e = launch_permute(ids, counts, (int)R, El, sh.K, pairs, L.routed_cap,
+    e = launch_permute(ids, counts, false, (int)R, El, sh.K, pairs, L.routed_cap,
                        at<int32_t>(ws, L.perm_scratch), at<int32_t>(ws, L.offsets),
                        at<int32_t>(ws, L.group_rows), at<int32_t>(ws, L.row_start),
                        at<int32_t>(ws, L.row_token), token_row, status, s, sms);

@@ -41,14 +41,16 @@ cudaError_t launch_quantize_128x128(const float* w, int64_t rows, int64_t cols, 
 
 // Router: gate logits (fp32 SIMT GEMM), then sigmoid, biased top-K (node-
 // limited to the M best of G expert groups when G > 1), gates and counts
-// (counts must be zero on entry).
+// (counts must be zero on entry; null: not counted).
 cudaError_t launch_router(const void* x, const float* gate_w, const float* bias, int T, int H,
                           int N, int K, int G, int M, float* logits, int32_t* ids, float* gates,
                           int32_t* counts, uint32_t* status, cudaStream_t stream, int sm_count);
 
 // Router on tensor cores: splits the fp32 centroids into three bf16 terms in
 // `wsplit` (router_split_bytes), computes the logits with BF16 tcgen05 MMAs
-// and fp32 accumulation, then the same top-K as launch_router.
+// and fp32 accumulation, then the same top-K as launch_router (for large T
+// at N = 256 and K <= 8 inside the logits kernel's epilogue; the logits are
+// written in every case).
 // presplit: the three terms made earlier (launch_split_gate); NULL: split
 // into wsplit first.
 size_t router_split_bytes(int N, int H);
@@ -97,14 +99,16 @@ cudaError_t launch_balance_stats(const float* logits, const int32_t* ids, int T,
 // tables and per-chunk base rows, and the stable placement of the (token,
 // slot) pairs into expert-major GEMM rows. Slots whose id is negative are
 // skipped (their token_row entries are left as they are); `pairs` is the
-// number of slots with an id, checked against the counts. `hist` is scratch
-// of permute_scratch_bytes(T, N) bytes.
+// number of slots with an id, checked against the counts. With count_out the
+// per-expert counts are written from the chunks' histograms, else they are
+// read and checked against them. `hist` is scratch of
+// permute_scratch_bytes(T, N) bytes.
 size_t permute_scratch_bytes(int64_t T, int N);
-cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K,
-                           int64_t pairs, int64_t routed_cap, int32_t* hist, int32_t* offsets,
-                           int32_t* group_rows, int32_t* row_start, int32_t* row_token,
-                           int32_t* token_row, uint32_t* status, cudaStream_t stream,
-                           int sm_count);
+cudaError_t launch_permute(const int32_t* ids, int32_t* counts, bool count_out, int T, int N,
+                           int K, int64_t pairs, int64_t routed_cap, int32_t* hist,
+                           int32_t* offsets, int32_t* group_rows, int32_t* row_start,
+                           int32_t* row_token, int32_t* token_row, uint32_t* status,
+                           cudaStream_t stream, int sm_count);
 // 1x128 quantisation of x written to each token's shared-expert row
 // (routed_cap + t) and to its K routed rows token_row[t, k].
 cudaError_t launch_quantize_scatter(const void* x, int T, int H, int K, const int32_t* token_row,

@@ -6,8 +6,10 @@
 //           chunk's earlier pairs with the same expert (per-warp lane masks of
 //           each expert, then a scan over the chunk's four warps), and the
 //           chunk's count of each expert
-//   scan  : counts -> offsets, GEMM group rows and 128-aligned row starts, and
-//           for every (chunk, expert) the first GEMM row of that chunk's pairs
+//   scan  : the per-chunk counts summed into each expert's count (written, or
+//           checked against the router's), offsets, GEMM group rows and
+//           128-aligned row starts, and for every (chunk, expert) the first
+//           GEMM row of that chunk's pairs
 //   place : row = chunk base + rank for every pair; records row_token and
 //           token_row (the activation quantiser then writes every token's
 //           codes straight into its rows)
@@ -72,20 +74,38 @@ __global__ void __launch_bounds__(kChunk) rank_kernel(const int32_t* __restrict_
       ranks[t * K + k] = base[warp * N + e[k]] + __popc(mask[warp * N + e[k]] & below);
 }
 
-// One CTA of 1024 threads; N <= 1024. Group tables as before, then for every
-// chunk c: hist[c, e] <- row_start[e] + the pairs of e in chunks before c.
-// `pairs` is the number of (token, slot) pairs the counts must add up to
-// (negative: not checked).
-__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ counts, int N,
-                                                    int T, int64_t pairs, int64_t routed_cap,
-                                                    int n_chunks, int32_t* __restrict__ hist,
+// One CTA of 1024 threads; N <= 1024. Each expert's count is the sum of its
+// per-chunk counts; with count_out the counts are written from them, else
+// they are read from `counts` and checked against them. Then the group
+// tables, and for every chunk c: hist[c, e] <- row_start[e] + the pairs of e
+// in chunks before c. `pairs` is the number of (token, slot) pairs the counts
+// must add up to (negative: not checked). Eight chunks' counts are fetched
+// before any is used, so the loads overlap.
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts, bool count_out,
+                                                    int N, int T, int64_t pairs,
+                                                    int64_t routed_cap, int n_chunks,
+                                                    int32_t* __restrict__ hist,
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ group_rows,
                                                     int32_t* __restrict__ row_start,
                                                     uint32_t* __restrict__ status) {
   __shared__ int sums[33];
   const int e = threadIdx.x;
-  const int c = e < N ? counts[e] : 0;
+  int c = 0;
+  if (e < N) {
+    for (int ch0 = 0; ch0 < n_chunks; ch0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = ch0 + j < n_chunks ? hist[(int64_t)(ch0 + j) * N + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) c += v[j];
+    }
+    if (count_out) {
+      counts[e] = c;
+    } else if (counts[e] != c) {
+      flag_status(status, kStatusBounds);
+    }
+  }
   const int padded = (c + kTile - 1) / kTile * kTile;
   int total_c, total_p;
   const int off = block_scan_int(c, sums, &total_c);
@@ -94,8 +114,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
     offsets[e] = off;
     group_rows[e] = c;
     row_start[e] = start;
-    // eight chunks' counts are fetched before any is used, so the loads
-    // overlap instead of costing one memory latency per chunk
     int run = start;
     for (int ch0 = 0; ch0 < n_chunks; ch0 += 8) {
       int v[8];
@@ -107,7 +125,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
         run += v[j];
       }
     }
-    if (run != start + c) flag_status(status, kStatusBounds);
   }
   if (e == 0) {
     offsets[N] = total_c;
@@ -152,11 +169,11 @@ size_t permute_scratch_bytes(int64_t T, int N) {
   return (size_t)((T + kChunk - 1) / kChunk) * (size_t)N * 4;
 }
 
-cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int N, int K,
-                           int64_t pairs, int64_t routed_cap, int32_t* hist, int32_t* offsets,
-                           int32_t* group_rows, int32_t* row_start, int32_t* row_token,
-                           int32_t* token_row, uint32_t* status, cudaStream_t stream,
-                           int sm_count) {
+cudaError_t launch_permute(const int32_t* ids, int32_t* counts, bool count_out, int T, int N,
+                           int K, int64_t pairs, int64_t routed_cap, int32_t* hist,
+                           int32_t* offsets, int32_t* group_rows, int32_t* row_start,
+                           int32_t* row_token, int32_t* token_row, uint32_t* status,
+                           cudaStream_t stream, int sm_count) {
   const int n_chunks = (T + kChunk - 1) / kChunk;
   // at most 2 * 4 * 1024 ints = 32 KB (N <= 1024): under the default limit
   const size_t smem = (size_t)2 * kChunkWarps * N * sizeof(int);
@@ -166,8 +183,8 @@ cudaError_t launch_permute(const int32_t* ids, const int32_t* counts, int T, int
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  scan_kernel<<<1, 1024, 0, stream>>>(counts, N, T, pairs, routed_cap, n_chunks, hist, offsets,
-                                      group_rows, row_start, status);
+  scan_kernel<<<1, 1024, 0, stream>>>(counts, count_out, N, T, pairs, routed_cap, n_chunks, hist,
+                                      offsets, group_rows, row_start, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(row_token, 0xFF, (size_t)routed_cap * sizeof(int32_t), stream);

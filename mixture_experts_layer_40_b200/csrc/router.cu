@@ -81,6 +81,18 @@ __global__ void __launch_bounds__(256) logits_kernel(const __nv_bfloat16* __rest
 
 constexpr int kMaxPerLane = 32;  // N <= 1024
 
+// The affinity s = sigmoid(z) and the biased selection score s + b (a NaN
+// score ranks below every number). Every top-K path uses these two, so that
+// equal logits give equal choices whichever kernel made them.
+// The reciprocal is the hardware one (__fdividef: within 2 ulp, no branch,
+// and 0 once exp(-z) overflows), so that the 32 affinities of a chunk can be
+// scheduled together; the exact quotient's slow-path branch serialised them.
+MOE_DEV float affinity(float z) { return __fdividef(1.0f, 1.0f + expf(-z)); }
+MOE_DEV float biased_score(float s, float b) {
+  const float v = s + b;
+  return v == v ? v : -INFINITY;
+}
+
 // Warp arg-max of (score, id) pairs: the highest score, the lower id on ties.
 MOE_DEV void warp_argmax(float& best, int& bid) {
 #pragma unroll
@@ -96,7 +108,9 @@ MOE_DEV void warp_argmax(float& best, int& bid) {
 
 // One warp per token: sigmoid, biased scores, K rounds of a warp arg-max
 // (highest score, lower id on ties), gates from the unbiased affinities,
-// counts by integer atomics (exact, order-independent).
+// counts by integer atomics (exact, order-independent) unless counts is null
+// (the layer forward takes them from the permutation's histograms instead:
+// at T = 32768 the atomics on N counters cost about 0.1 ms).
 // Node-limited routing (G > 1, "DeepSeek-V3, explained", recipe step 5):
 // before the K rounds, each of the G contiguous expert groups is scored by
 // the sum of its K/M highest biased scores (taken in descending order), the
@@ -122,10 +136,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
       sv[j] = 0.0f;
       const int e = lane + 32 * j;
       if (j < per_lane && e < N) {
-        const float s = 1.0f / (1.0f + expf(-z[(int64_t)t * N + e]));
-        const float v = s + bias[e];
+        const float s = affinity(z[(int64_t)t * N + e]);
         sv[j] = s;
-        sc[j] = (v == v) ? v : -INFINITY;
+        sc[j] = biased_score(s, bias[e]);
       }
     }
     if (G > 1 && M < G) {
@@ -206,7 +219,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ z,
     if (lane < K) {
       ids[(int64_t)t * K + lane] = my_id;
       gates[(int64_t)t * K + lane] = my_s / sum;
-      atomicAdd(&counts[my_id], 1);
+      if (counts != nullptr) atomicAdd(&counts[my_id], 1);
     }
   }
 }
@@ -240,8 +253,6 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int N, in
 //   3. one CTA per sequence: chunk partials added in chunk order, then f, P
 //      and alpha * sum_i f_i P_i (expert order).
 constexpr int kBalChunk = 128;
-
-MOE_DEV float affinity(float z) { return 1.0f / (1.0f + expf(-z)); }
 
 __global__ void __launch_bounds__(256) token_sum_kernel(const float* __restrict__ z, int T, int N,
                                                         float* __restrict__ denom) {
@@ -551,14 +562,43 @@ struct alignas(8) WideShared {
   uint64_t tfull;
   uint32_t tmem_base;
   int abort;
+  float bias[kWN];
+};
+
+// Selection fused into the wide tiles' epilogue when one tile holds all of a
+// token's scores (N = 256) and K <= kFuseL: each epilogue thread owns one
+// token (one TMEM lane) and keeps its best kFuseL (score, id, affinity)
+// triples in registers, sorted, while the 256 columns stream past in chunks
+// of 32. Candidates arrive in ascending id, so a candidate ties with a kept
+// entry only to lose (the lower id wins), exactly as in topk_kernel; the
+// first K entries of the sorted list are topk_kernel's K choices in its
+// order. Node-limited routing is fused for G = 8 groups of 32 experts (one
+// chunk each): a first pass sums each group's K/M highest scores (highest
+// first), the M best groups are kept (lower group on ties) and the other
+// groups' experts enter the second pass with score -inf.
+constexpr int kFuseL = 8;
+constexpr int kStashStride = 256;  // one float per epilogue thread per row
+static_assert(64 * kStashStride * 4 <= kWStages * kWStageBytes, "stash fits in the ring");
+
+MOE_DEV bool ranks_above(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+struct FuseArgs {
+  const float* bias;
+  int K, G, M;
+  int32_t* ids;
+  float* gates;
+  int32_t* counts;  // null: not counted
 };
 
 // Warps: 0 TMA producer, 1 TMEM allocator and MMA issuer, 2-3 idle, 4-11
 // epilogue (warpgroup h reads accumulator h: tokens 128h .. 128h + 127).
+template <bool kFuse>
 __global__ void __launch_bounds__(kWThreads, 1)
     logits_tc_wide_kernel(const __grid_constant__ CUtensorMap tm_x,
                           const __grid_constant__ CUtensorMap tm_w, int T, int H, int N,
-                          float* __restrict__ z, uint32_t* __restrict__ status) {
+                          float* __restrict__ z, uint32_t* __restrict__ status, FuseArgs fa) {
   __shared__ WideShared sh;
   extern __shared__ uint8_t dyn_smem[];
   const uint32_t ring = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -582,6 +622,10 @@ __global__ void __launch_bounds__(kWThreads, 1)
     prefetch_tensormap(&tm_w);
   }
   if (warp == 1) tmem_alloc(smem_u32(&sh.tmem_base), 512);
+  if (kFuse && warp >= 4) {
+    const int i = threadIdx.x - 128;
+    sh.bias[i] = fa.bias[n0 + i];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -655,6 +699,81 @@ __global__ void __launch_bounds__(kWThreads, 1)
       const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(h * kWN);
       const int cols = min(kWN, N - n0);
       float* dst = z + (int64_t)t * N + n0;
+      // this thread's column of the stash: 32 (affinity, score) pairs
+      float* stash = reinterpret_cast<float*>(dyn_smem + (ring - smem_u32(dyn_smem))) +
+                     (threadIdx.x - 128);
+      // node-limited routing: which of the 8 groups this token keeps
+      uint32_t keep = 0xffffffffu;
+      if (kFuse && fa.G > 1 && fa.M < fa.G) {
+        const int per_group = fa.K / fa.M;
+        float gs[8];
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          float v[32];
+          tmem_ld32(t0 + (uint32_t)(32 * c), v);
+          tmem_wait_ld();
+          if (per_group <= 2) {
+            // the two highest, branch-free: t0 >= t1 throughout
+            float h0 = -INFINITY, h1 = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float sc = biased_score(affinity(v[j]), sh.bias[32 * c + j]);
+              h1 = fmaxf(h1, fminf(h0, sc));
+              h0 = fmaxf(h0, sc);
+            }
+            const float gsum = per_group == 1 ? 0.0f + h0 : (0.0f + h0) + h1;
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+              if (g == c) gs[g] = gsum;
+            continue;
+          }
+          float top[kFuseL];
+#pragma unroll
+          for (int i = 0; i < kFuseL; ++i) top[i] = -INFINITY;
+          // the chunk's scores first (independent: no branch between them)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = biased_score(affinity(v[j]), sh.bias[32 * c + j]);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float sc = v[j];
+            if (sc > top[kFuseL - 1]) {
+              bool b[kFuseL];
+#pragma unroll
+              for (int i = 0; i < kFuseL; ++i) b[i] = sc > top[i];
+#pragma unroll
+              for (int i = kFuseL - 1; i > 0; --i) top[i] = b[i - 1] ? top[i - 1] : (b[i] ? sc : top[i]);
+              top[0] = b[0] ? sc : top[0];
+            }
+          }
+          float gsum = 0.0f;
+#pragma unroll
+          for (int i = 0; i < kFuseL; ++i)
+            if (i < per_group) gsum += top[i];
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            if (g == c) gs[g] = gsum;
+        }
+        keep = 0;
+        for (int r = 0; r < fa.M; ++r) {
+          float best = -INFINITY;
+          int bid = 32;
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            if (!((keep >> g) & 1u) && ranks_above(gs[g], g, best, bid)) {
+              best = gs[g];
+              bid = g;
+            }
+          keep |= 1u << bid;
+        }
+      }
+      float lv[kFuseL], ls[kFuseL];
+      int li[kFuseL];
+#pragma unroll
+      for (int i = 0; i < kFuseL; ++i) {
+        lv[i] = -INFINITY;
+        li[i] = kWN;  // beaten by every real expert
+        ls[i] = 0.0f;
+      }
 #pragma unroll 1
       for (int c = 0; c < kWN; c += 32) {
         float v[32];
@@ -666,6 +785,64 @@ __global__ void __launch_bounds__(kWThreads, 1)
             if (c + 4 * j < cols)
               reinterpret_cast<float4*>(dst + c)[j] =
                   make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+        if (kFuse) {
+          // a masked group's experts score -inf: they matter only while the
+          // list still holds a -inf entry
+          const bool masked = !((keep >> (c / 32)) & 1u);
+          if (!masked || lv[kFuseL - 1] == -INFINITY) {
+            // the chunk's affinities and scores (independent, no branches),
+            // stashed in the idle operand ring; the candidates that beat the
+            // list's last entry as it stood before the chunk are marked, and
+            // only those are inserted, in ascending id: a warp then runs as
+            // many insertions as its busiest lane, not one per column that
+            // any lane wants
+            uint32_t pass = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float a = affinity(v[j]);
+              const float sc = masked ? -INFINITY : biased_score(a, sh.bias[c + j]);
+              stash[(2 * j) * kStashStride] = a;
+              stash[(2 * j + 1) * kStashStride] = sc;
+              pass |= (uint32_t)ranks_above(sc, c + j, lv[kFuseL - 1], li[kFuseL - 1]) << j;
+            }
+            while (pass != 0u) {
+              const int j = __ffs(pass) - 1;
+              pass &= pass - 1u;
+              const int e = c + j;
+              const float s = stash[(2 * j) * kStashStride];
+              const float sc = stash[(2 * j + 1) * kStashStride];
+              if (ranks_above(sc, e, lv[kFuseL - 1], li[kFuseL - 1])) {
+                bool b[kFuseL];
+#pragma unroll
+                for (int i = 0; i < kFuseL; ++i) b[i] = ranks_above(sc, e, lv[i], li[i]);
+#pragma unroll
+                for (int i = kFuseL - 1; i > 0; --i) {
+                  lv[i] = b[i - 1] ? lv[i - 1] : (b[i] ? sc : lv[i]);
+                  li[i] = b[i - 1] ? li[i - 1] : (b[i] ? e : li[i]);
+                  ls[i] = b[i - 1] ? ls[i - 1] : (b[i] ? s : ls[i]);
+                }
+                lv[0] = b[0] ? sc : lv[0];
+                li[0] = b[0] ? e : li[0];
+                ls[0] = b[0] ? s : ls[0];
+              }
+            }
+          }
+        }
+      }
+      if (kFuse && t < T) {
+        // gates from the unbiased affinities, normalised in selection order
+        float sum = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kFuseL; ++i)
+          if (i < fa.K) sum += ls[i];
+#pragma unroll
+        for (int i = 0; i < kFuseL; ++i) {
+          if (i < fa.K) {
+            fa.ids[(int64_t)t * fa.K + i] = li[i];
+            fa.gates[(int64_t)t * fa.K + i] = ls[i] / sum;
+            if (fa.counts != nullptr) atomicAdd(&fa.counts[li[i]], 1);
+          }
         }
       }
     }
@@ -719,8 +896,11 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kRDynSmem);
     if (r != cudaSuccess) return r;
-    return cudaFuncSetAttribute(logits_tc_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kWDynSmem);
+    r = cudaFuncSetAttribute(logits_tc_wide_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWDynSmem);
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(logits_tc_wide_kernel<true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWDynSmem);
   });
   if (e != cudaSuccess) return e;
   CUtensorMap mx, mw;
@@ -730,8 +910,16 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
     e = make_tmap_bf16(&mw, terms, H, N, 3, kWK, kWN, 3);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((T + kWM - 1) / kWM), (unsigned)((N + kWN - 1) / kWN));
-    logits_tc_wide_kernel<<<grid, kWThreads, kWDynSmem, stream>>>(mx, mw, T, H, N, logits,
-                                                                  status);
+    const bool grouped = G > 1 && M < G;
+    FuseArgs fa{bias, K, G, M, ids, gates, counts};
+    if (N == kWN && K <= kFuseL && (!grouped || G == 8)) {
+      // the selection runs in the tiles' epilogue
+      logits_tc_wide_kernel<true><<<grid, kWThreads, kWDynSmem, stream>>>(mx, mw, T, H, N, logits,
+                                                                          status, fa);
+      return cudaGetLastError();
+    }
+    logits_tc_wide_kernel<false><<<grid, kWThreads, kWDynSmem, stream>>>(mx, mw, T, H, N, logits,
+                                                                         status, fa);
   } else {
     e = make_tmap_bf16(&mx, x, H, T, 1, kRK, kRM);
     if (e != cudaSuccess) return e;

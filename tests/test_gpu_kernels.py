@@ -117,6 +117,23 @@ def test_route_parity(capi, name):
     assert np.allclose(gates.sum(axis=1), 1.0, atol=GATE_TOL)
 
 
+@pytest.mark.parametrize("k", [1, 4])
+def test_route_parity_wide_tiles_fewer_slots(capi, k):
+    """The selection fused into the wide logits tiles keeps a sorted list of
+    eight; with K < 8 its first K entries are the choices. T = 16384 with a
+    ragged last tile (T - 100)."""
+    w = I.Workload("wide", T=16384 - 100, H=7168, N=256, K=k, I=2048, bias_range=0.05,
+                   seed=21)
+    xb = I.make_x(w)
+    gate_w, bias = I.make_gate_w(w), I.make_bias(w)
+    ids, gates, counts = _route(capi, w, xb, gate_w, bias)
+    r_ids, _, s, score = O.route(I.bf16_bits_to_f32(xb), gate_w, bias, w.K)
+    use_ids, _, _ = H.reconcile_ids(ids, r_ids, score, w.K)
+    assert np.array_equal(counts, O.expert_counts(use_ids, w.N))
+    sel = np.take_along_axis(s, ids.astype(np.int64), axis=1)
+    assert np.max(np.abs(gates - sel / sel.sum(axis=1, keepdims=True))) < GATE_TOL
+
+
 def test_route_ragged_tokens_and_hot_expert(capi):
     w = I.Workload("hot", T=333, H=512, N=32, K=4, I=128, bias_range=0.1)
     xb = I.make_x(w)

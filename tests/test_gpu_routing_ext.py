@@ -80,16 +80,19 @@ def _reconcile_grouped(gpu_ids, o_ids, score, gscore, k, groups, top):
     return int(differ.sum())
 
 
-@pytest.mark.parametrize("t_count", [4096, 333])
-def test_node_limited_v3_shape(t_count):
-    w = I.Workload("g", T=t_count, H=7168, N=256, K=8, I=2048, bias_range=0.05, seed=11)
+@pytest.mark.parametrize("t_count,k,top", [(4096, 8, 4), (333, 8, 4), (16384, 8, 4),
+                                           (16384, 6, 3)])
+def test_node_limited_v3_shape(t_count, k, top):
+    """T = 16384 takes the wide logits tiles, whose epilogue also makes the
+    selection (group scores, kept groups, top-K) for each of its tokens."""
+    w = I.Workload("g", T=t_count, H=7168, N=256, K=k, I=2048, bias_range=0.05, seed=11)
     xb = I.make_x(w)
     x, gw, b = I.bf16_bits_to_f32(xb), I.make_gate_w(w), I.make_bias(w)
-    _, _, ids, gates, counts = _route(w, xb, gw, b, 8, 4)
+    _, _, ids, gates, counts = _route(w, xb, gw, b, 8, top)
     gid = ids.cpu().numpy()
-    o_ids, o_gates, s, score, gscore = O.route_grouped(x, gw, b, w.K, 8, 4)
-    assert np.all([len(set((gid[t] // 32).tolist())) <= 4 for t in range(w.T)])
-    ndiff = _reconcile_grouped(gid, o_ids, score, gscore, w.K, 8, 4)
+    o_ids, o_gates, s, score, gscore = O.route_grouped(x, gw, b, w.K, 8, top)
+    assert np.all([len(set((gid[t] // 32).tolist())) <= top for t in range(w.T)])
+    ndiff = _reconcile_grouped(gid, o_ids, score, gscore, w.K, 8, top)
     assert ndiff <= max(2, w.T // 500)
     same = np.all(gid == o_ids, axis=1)
     assert np.max(np.abs(gates.cpu().numpy()[same] - o_gates[same])) < 1e-5
