@@ -178,10 +178,16 @@ def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-@pytest.mark.parametrize("h_dim,i_dim,group_rows", [
+# Group sizes: empty groups, whole 128-row tiles, last row tiles of 1, 3, 5,
+# 44, 64 and 65 rows.
+TAIL_CASES = [
     (256, 128, [5, 0, 128, 129, 300, 1]),
+    (256, 128, [64, 65, 192, 3, 0, 0, 64]),
     (7168, 2048, [130, 0, 7, 256]),
-])
+]
+
+
+@pytest.mark.parametrize("h_dim,i_dim,group_rows", TAIL_CASES)
 def test_expert_up_parity(capi, h_dim, i_dim, group_rows):
     c = _gemm_case(h_dim, i_dim, group_rows, seed=h_dim)
     n_groups, rows = len(group_rows), c["rows"]
@@ -220,10 +226,7 @@ def test_expert_up_parity(capi, h_dim, i_dim, group_rows):
     assert np.all(hq[~written] == 0x5A) and np.all(hs[~written] == -7.0)
 
 
-@pytest.mark.parametrize("h_dim,i_dim,group_rows", [
-    (256, 128, [5, 0, 128, 129, 300, 1]),
-    (7168, 2048, [130, 0, 7, 256]),
-])
+@pytest.mark.parametrize("h_dim,i_dim,group_rows", TAIL_CASES)
 def test_expert_down_parity(capi, h_dim, i_dim, group_rows):
     rng = np.random.default_rng(h_dim + 1)
     starts, r = [], 0
@@ -266,6 +269,7 @@ def test_expert_down_parity(capi, h_dim, i_dim, group_rows):
 
 @pytest.mark.parametrize("h_dim,i_dim,group_rows", [
     (256, 128, [5, 0, 128, 129, 300, 1, 31, 32, 33]),
+    (256, 128, [64, 65, 192, 3, 0, 0, 64]),
     (7168, 2048, [130, 0, 7, 256]),
 ])
 def test_expert_down_bf16_is_the_rounded_fp32_gemm(capi, h_dim, i_dim, group_rows):
