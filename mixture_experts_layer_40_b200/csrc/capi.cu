@@ -205,7 +205,8 @@ int moe_route(moe_shape sh, const float* gate_w, const void* x, const float* bia
   if (e == cudaSuccess)
     e = launch_router_tc(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                          at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), topk_ids,
-                         topk_gates, counts, status, s, sm_count());
+                         topk_gates, counts, status, s, sm_count(), nullptr,
+                         at<float>(ws, L.a_q), (size_t)L.rows_total * sh.H);
   return cuda_status(e);
 }
 
@@ -282,7 +283,10 @@ static int forward_impl(moe_shape sh, const moe_weights* w, const void* x, const
     e = launch_router_tc(x, w->gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                          at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
                          nullptr, status, s, sms,
-                         static_cast<const __nv_bfloat16*>(w->gate_split));
+                         static_cast<const __nv_bfloat16*>(w->gate_split),
+                         // the activation rows are written after the routing:
+                         // their region holds the partial logits meanwhile
+                         reinterpret_cast<float*>(a_q), (size_t)L.rows_total * sh.H);
   e = mark(1, e);
   // a6-a7: counts from per-chunk histograms, offsets, stable expert-major
   // placement of the (token, slot) pairs

@@ -60,7 +60,7 @@ struct SourceLayout {
   int64_t rows;  // shared-expert GEMM rows (T rounded up to 128)
   size_t status, counts, topk_ids, topk_gates, logits, gate_split, send_slot, grp, plan, dest_off;
   size_t send_counts;
-  size_t a_q, a_s, h_q, h_s, y_shared, total;
+  size_t a_q, a_s, h_q, h_s, y_shared, splitk, total;
 };
 
 SourceLayout source_layout(const moe_shape& sh, int W) {
@@ -85,6 +85,9 @@ SourceLayout source_layout(const moe_shape& sh, int W) {
   L.h_q = take((size_t)(L.rows * I));
   L.h_s = take((size_t)(L.rows * (I / kTile)) * 4);
   L.y_shared = take((size_t)(L.rows * H) * 2);
+  // the router's partial logits, so that the dispatch routes the rank's
+  // tokens exactly as the one-GPU layer does
+  L.splitk = take(router_splitk_bytes(T, (int)N, (int)H));
   L.total = carve.off;
   return L;
 }
@@ -561,7 +564,8 @@ int dispatch_impl(const moe_shape& sh, int W, int rank, const float* gate_w, con
   float* gates = topk_gates_opt ? topk_gates_opt : at<float>(ws, L.topk_gates);
   e = launch_router_tc(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                        at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
-                       counts, status, s, sms);
+                       counts, status, s, sms, nullptr, at<float>(ws, L.splitk),
+                       router_splitk_bytes(sh.T, sh.N, sh.H));
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   int32_t* send_slot = at<int32_t>(ws, L.send_slot);
   int32_t* dest_off = at<int32_t>(ws, L.dest_off);

@@ -50,17 +50,24 @@ cudaError_t launch_router(const void* x, const float* gate_w, const float* bias,
 // `wsplit` (router_split_bytes), computes the logits with BF16 tcgen05 MMAs
 // and fp32 accumulation, then the same top-K as launch_router (for large T
 // at N = 256 and K <= 8 inside the logits kernel's epilogue; the logits are
-// written in every case).
+// written in every case). splitk_scratch (splitk_bytes, 16-byte aligned; may
+// be NULL): room for partial logits, so that batches too small to fill the
+// GPU with whole-depth tiles split the reduction over several CTAs.
 // presplit: the three terms made earlier (launch_split_gate); NULL: split
 // into wsplit first.
 size_t router_split_bytes(int N, int H);
+// Bytes of partial logits launch_router_tc needs as splitk_scratch to split
+// the reduction for this shape (0: no split). With less it computes the
+// logits with whole-depth tiles, whose fp32 sums round differently.
+size_t router_splitk_bytes(int64_t T, int N, int H);
 cudaError_t launch_split_gate(const float* gate_w, int N, int H, __nv_bfloat16* wsplit,
                               cudaStream_t stream, int sm_count);
 cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
                              int N, int K, int G, int M, __nv_bfloat16* wsplit, float* logits,
                              int32_t* ids, float* gates, int32_t* counts, uint32_t* status,
                              cudaStream_t stream, int sm_count,
-                             const __nv_bfloat16* presplit = nullptr);
+                             const __nv_bfloat16* presplit = nullptr,
+                             float* splitk_scratch = nullptr, size_t splitk_bytes = 0);
 
 // Backward of the expert path (backward.cu).
 cudaError_t launch_transpose_blocks(const uint8_t* w, const float* s, int64_t groups, int64_t rows,

@@ -594,7 +594,13 @@ struct FuseArgs {
 
 // Warps: 0 TMA producer, 1 TMEM allocator and MMA issuer, 2-3 idle, 4-11
 // epilogue (warpgroup h reads accumulator h: tokens 128h .. 128h + 127).
-template <bool kFuse>
+// kMode: kWideLogits writes the logits; kWideSelect also makes the selection
+// (above); kWideSplit covers the slice blockIdx.z of gridDim.z equal slices
+// of the reduction and writes its fp32 partial sums to z + blockIdx.z * T * N
+// (summed in slice order by splitk_reduce_kernel).
+enum WideMode : int { kWideLogits = 0, kWideSelect = 1, kWideSplit = 2 };
+
+template <int kMode>
 __global__ void __launch_bounds__(kWThreads, 1)
     logits_tc_wide_kernel(const __grid_constant__ CUtensorMap tm_x,
                           const __grid_constant__ CUtensorMap tm_w, int T, int H, int N,
@@ -604,9 +610,13 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const uint32_t ring = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  constexpr bool kFuse = kMode == kWideSelect;
+  constexpr bool kSplit = kMode == kWideSplit;
   const int m0 = blockIdx.x * kWM;
   const int n0 = blockIdx.y * kWN;
-  const int kb_n = H / kWK;
+  const int kb_all = H / kWK;
+  const int kb_lo = kSplit ? (int)((int64_t)kb_all * blockIdx.z / gridDim.z) : 0;
+  const int kb_n = (kSplit ? (int)((int64_t)kb_all * (blockIdx.z + 1) / gridDim.z) : kb_all) - kb_lo;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kWStages; ++s) {
@@ -643,11 +653,12 @@ __global__ void __launch_bounds__(kWThreads, 1)
         const uint32_t full = smem_u32(&sh.full[s]);
         mbar_arrive_expect_tx(full, kWStageBytes);
         const uint32_t sa = ring + s * kWStageBytes;
-        tma_load_2d(sa, &tm_x, kb * kWK, m0, full);
+        tma_load_2d(sa, &tm_x, (kb_lo + kb) * kWK, m0, full);
         asm volatile(
             "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
             " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(sa + kWABytes),
-            "l"(reinterpret_cast<uint64_t>(&tm_w)), "r"(kb * kWK), "r"(n0), "r"(0), "r"(full)
+            "l"(reinterpret_cast<uint64_t>(&tm_w)), "r"((kb_lo + kb) * kWK), "r"(n0), "r"(0),
+            "r"(full)
             : "memory");
       }
       if (kb < kb_n) {
@@ -698,7 +709,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
       tc_fence_after();
       const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(h * kWN);
       const int cols = min(kWN, N - n0);
-      float* dst = z + (int64_t)t * N + n0;
+      float* dst = z + (kSplit ? (int64_t)blockIdx.z * T * N : 0) + (int64_t)t * N + n0;
       // this thread's column of the stash: 32 (affinity, score) pairs
       float* stash = reinterpret_cast<float*>(dyn_smem + (ring - smem_u32(dyn_smem))) +
                      (threadIdx.x - 128);
@@ -853,7 +864,42 @@ __global__ void __launch_bounds__(kWThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, 512);
 }
 
+// z = the sum of the S slices' partial logits, added in slice order.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ part,
+                                                           int64_t n4, int S,
+                                                           float4* __restrict__ z) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 a = part[i];
+    for (int s = 1; s < S; ++s) {
+      const float4 b = part[(int64_t)s * n4 + i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    z[i] = a;
+  }
+}
+
+// Slices of the reduction for wide tiles when neither tile shape alone fills
+// the GPU (batches below the wide tiles' threshold): as many as keep the 148
+// SMs of a B200 busy, each at least 8 k-blocks (256 channels) deep; 0 = none.
+// The count depends on the shape only (not on the device or on the scratch
+// given), so every path that routes the same tokens sums the same slices.
+int splitk_slices(int64_t T, int64_t N, int64_t H) {
+  constexpr int64_t kSms = 148;
+  if (N % kWN != 0 || T <= 0) return 0;
+  const int64_t tiles = ((T + kWM - 1) / kWM) * (N / kWN);
+  const int64_t s = std::min<int64_t>(kSms / tiles, (H / kWK) / 8);
+  return s >= 2 ? (int)s : 0;
+}
+
 }  // namespace
+
+size_t router_splitk_bytes(int64_t T, int N, int H) {
+  return (size_t)splitk_slices(T, N, H) * (size_t)T * (size_t)N * sizeof(float);
+}
 
 size_t router_split_bytes(int N, int H) { return (size_t)3 * N * H * sizeof(__nv_bfloat16); }
 
@@ -882,7 +928,8 @@ cudaError_t launch_split_gate(const float* gate_w, int N, int H, __nv_bfloat16* 
 cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bias, int T, int H,
                              int N, int K, int G, int M, __nv_bfloat16* wsplit, float* logits,
                              int32_t* ids, float* gates, int32_t* counts, uint32_t* status,
-                             cudaStream_t stream, int sm_count, const __nv_bfloat16* presplit) {
+                             cudaStream_t stream, int sm_count, const __nv_bfloat16* presplit,
+                             float* splitk_scratch, size_t splitk_bytes) {
   if (T == 0) return cudaSuccess;
   cudaError_t e = cudaSuccess;
   if (presplit == nullptr) {
@@ -896,10 +943,13 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kRDynSmem);
     if (r != cudaSuccess) return r;
-    r = cudaFuncSetAttribute(logits_tc_wide_kernel<false>,
+    r = cudaFuncSetAttribute(logits_tc_wide_kernel<kWideLogits>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWDynSmem);
     if (r != cudaSuccess) return r;
-    return cudaFuncSetAttribute(logits_tc_wide_kernel<true>,
+    r = cudaFuncSetAttribute(logits_tc_wide_kernel<kWideSplit>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWDynSmem);
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(logits_tc_wide_kernel<kWideSelect>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWDynSmem);
   });
   if (e != cudaSuccess) return e;
@@ -914,12 +964,30 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, const float* bi
     FuseArgs fa{bias, K, G, M, ids, gates, counts};
     if (N == kWN && K <= kFuseL && (!grouped || G == 8)) {
       // the selection runs in the tiles' epilogue
-      logits_tc_wide_kernel<true><<<grid, kWThreads, kWDynSmem, stream>>>(mx, mw, T, H, N, logits,
-                                                                          status, fa);
+      logits_tc_wide_kernel<kWideSelect><<<grid, kWThreads, kWDynSmem, stream>>>(
+          mx, mw, T, H, N, logits, status, fa);
       return cudaGetLastError();
     }
-    logits_tc_wide_kernel<false><<<grid, kWThreads, kWDynSmem, stream>>>(mx, mw, T, H, N, logits,
-                                                                         status, fa);
+    logits_tc_wide_kernel<kWideLogits><<<grid, kWThreads, kWDynSmem, stream>>>(
+        mx, mw, T, H, N, logits, status, fa);
+  } else if (const int S = splitk_slices(T, N, H);
+             S >= 2 && splitk_scratch != nullptr &&
+             (size_t)S * (size_t)T * (size_t)N * sizeof(float) <= splitk_bytes) {
+    // wide tiles over S slices of the reduction, then the slices' sum
+    e = make_tmap_bf16(&mx, x, H, T, 1, kWK, kWM);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_bf16(&mw, terms, H, N, 3, kWK, kWN, 3);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((T + kWM - 1) / kWM), (unsigned)(N / kWN), (unsigned)S);
+    FuseArgs fa{};
+    logits_tc_wide_kernel<kWideSplit><<<grid, kWThreads, kWDynSmem, stream>>>(
+        mx, mw, T, H, N, splitk_scratch, status, fa);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t n4 = (int64_t)T * N / 4;
+    const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count * 8);
+    splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(splitk_scratch), n4, S, reinterpret_cast<float4*>(logits));
   } else {
     e = make_tmap_bf16(&mx, x, H, T, 1, kRK, kRM);
     if (e != cudaSuccess) return e;
