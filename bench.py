@@ -236,6 +236,30 @@ def measure_fp8_peak(torch, device):
 
 # ---------------------------------------------------------------- CPU oracle
 
+def router_launches(T: int, N: int, K: int, G: int, M: int, H: int, sms: int = 148) -> int:
+    """Kernels the router launches per forward (the centroids are split once
+    at set-up), following launch_router_tc in csrc/router.cu: wide tiles
+    (`use_wide_logits`) make the selection in their epilogue at N = 256,
+    K <= 8 (plain, or node-limited with 8 groups), else logits + top-K;
+    smaller batches split the reduction (`splitk_slices`: logits, slice sum,
+    top-K) or run 128 x 64 tiles (logits, top-K)."""
+    small = -(-T // 128) * -(-N // 64)
+    wide = -(-T // 256) * -(-N // 256)
+    if N % 256 == 0 and 10 * -(-small // sms) > 32 * -(-wide // sms):
+        grouped = G > 1 and M < G
+        return 1 if N == 256 and K <= 8 and (not grouped or G == 8) else 2
+    if N % 256 == 0 and T > 0 and min(148 // wide, (H // 32) // 8) >= 2:
+        return 3
+    return 2
+
+
+def step_launches(T: int, N: int, K: int, G: int, M: int, H: int) -> int:
+    """The library's kernels in one timed step: the router's, rank + scan +
+    place (the permutation), quantise-and-scatter, up GEMM, down GEMM,
+    combine, bias update."""
+    return router_launches(T, N, K, G, M, H) + 3 + 5
+
+
 def oracle_sample_step(w, x, gate_w, bias, ew, step: int, sample_tokens: int = 512,
                        groups: int = 1, shared_rows: int = 64, node_limit: tuple = (0, 0)):
     """One bounded sample of the layer on the CPU oracle; returns its time
@@ -417,9 +441,7 @@ def run_ours(args, w, rank, world, local_rank):
     for evs in events:
         for ev in evs:
             ev.record(stream)
-    # split gate, logits, top-K, scan, scatter, quantise-and-scatter, up, down,
-    # combine, bias update
-    launches_per_step = 10
+    launches_per_step = step_launches(w.T, w.N, w.K, args.groups, args.topk_groups, w.H)
 
     def step(traced_events=None, x_in=x, y_out=y):
         if traced_events is None:

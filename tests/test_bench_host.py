@@ -100,3 +100,17 @@ def test_roofline_bound_follows_the_ridge():
     r = bench.roofline_of(big, 10.0, 6650.0, 3160.0)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert abs(r["frac"] - big["flops"] / 1e-2 / 1e12 / 3160.0) < 1e-9
+
+
+def test_launch_count_follows_the_router_path():
+    """The `gpu_launches` claim: per step the router's kernels (1 with the
+    selection in the wide tiles' epilogue, 3 with a split reduction, 2
+    otherwise), the permutation's 3, and quantise, up, down, combine, bias
+    update. The counts match the launch lists of V3 prefill (11 kernels) and
+    large prefill (9) in profiles/."""
+    assert bench.step_launches(4096, 256, 8, 0, 0, 7168) == 11   # split logits
+    assert bench.step_launches(32768, 256, 8, 0, 0, 7168) == 9   # fused selection
+    assert bench.step_launches(32768, 256, 8, 8, 4, 7168) == 9   # node-limited, 8 groups
+    assert bench.step_launches(32768, 256, 16, 0, 0, 7168) == 10  # K > 8: logits + top-K
+    assert bench.step_launches(512, 32, 8, 0, 0, 7168) == 10     # N = 32: 128 x 64 tiles
+    assert bench.step_launches(128, 256, 8, 0, 0, 7168) == 11
