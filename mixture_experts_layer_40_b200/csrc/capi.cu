@@ -1,5 +1,6 @@
 // C ABI entry points (declared in include/moe_capi.h): argument checks,
 // workspace layout, tensor maps, and the launch sequence of the forward.
+#include <algorithm>
 #include <mutex>
 
 #include "host_util.h"
@@ -59,7 +60,8 @@ void layout_of(const moe_shape& s, moe_ws_layout* L) {
   L->topk_ids = take((size_t)(T * K) * 4);
   L->topk_gates = take((size_t)(T * K) * 4);
   L->logits = take((size_t)(T * N) * 4);
-  L->a_q = take((size_t)L->rows_total * H);
+  // the router's partial logits live here until the rows are written
+  L->a_q = take(std::max((size_t)L->rows_total * H, router_splitk_bytes(T, (int)N, (int)H)));
   L->a_s = take((size_t)L->rows_total * (H / kTile) * 4);
   L->h_q = take((size_t)L->rows_total * I);
   L->h_s = take((size_t)L->rows_total * (I / kTile) * 4);
