@@ -117,6 +117,23 @@ def test_route_parity(capi, name):
     assert np.allclose(gates.sum(axis=1), 1.0, atol=GATE_TOL)
 
 
+@pytest.mark.parametrize("t,n,h", [(333, 512, 2048), (1, 256, 7168), (700, 256, 1024)])
+def test_route_parity_split_reduction(capi, t, n, h):
+    """Batches too small for whole-depth tiles to fill the GPU split the gate
+    GEMM's reduction into slices (8 for T=333 at N=512 over two 256-expert
+    column tiles, 28 for one token, 4 for T=700 at H=1024) and sum the
+    slices in order before the top-K."""
+    w = I.Workload("split", T=t, H=h, N=n, K=8, I=256, bias_range=0.05, seed=22)
+    xb = I.make_x(w)
+    gate_w, bias = I.make_gate_w(w), I.make_bias(w)
+    ids, gates, counts = _route(capi, w, xb, gate_w, bias)
+    r_ids, _, s, score = O.route(I.bf16_bits_to_f32(xb), gate_w, bias, w.K)
+    use_ids, _, _ = H.reconcile_ids(ids, r_ids, score, w.K)
+    assert np.array_equal(counts, O.expert_counts(use_ids, w.N))
+    sel = np.take_along_axis(s, ids.astype(np.int64), axis=1)
+    assert np.max(np.abs(gates - sel / sel.sum(axis=1, keepdims=True))) < GATE_TOL
+
+
 @pytest.mark.parametrize("k", [1, 4])
 def test_route_parity_wide_tiles_fewer_slots(capi, k):
     """The selection fused into the wide logits tiles keeps a sorted list of
