@@ -199,10 +199,11 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const __nv_bfloat16* __r
 }
 
 // Column tiles for the weight gradients: 128 GEMM rows x 1 channel. One CTA
-// per 128-row block and 32 channels: the values (computed on the fly from
-// the source, 0 on padding rows) go through shared memory, 8 threads reduce
-// each channel's amax over the 128 rows, and each writes 16 codes of the
-// channel's transposed row. A operands keep the scale ([C, R/128]); B
+// per 128-row block and 32 channels (128 channels for the bf16 sources): the
+// values (computed on the fly from the source with 16-byte loads, 0 on
+// padding rows) go through shared memory, 8 threads reduce each channel's
+// amax over the 128 rows, and each writes 16 codes of the channel's
+// transposed row. A operands keep the scale ([C, R/128]); B
 // operands store its inverse, block-major ([R/128, C]), for the per-column
 // promotion of the weight-gradient GEMM.
 enum ColSource { kColDy = 0, kColX = 1, kColH = 2, kColDgu = 3 };
@@ -245,17 +246,47 @@ MOE_DEV float col_value(const ColArgs& a, int64_t r, int c) {
   return j < 128 ? d * u * (sg * (1.0f + g * (1.0f - sg))) : d * (g * sg);
 }
 
+// The token of GEMM row r (-1 on padding rows).
+MOE_DEV int col_token(const ColArgs& a, int64_t r) {
+  const int64_t rs = r - a.routed_cap;
+  return r < a.routed_cap ? a.row_token[r] : (rs < a.T ? (int)rs : -1);
+}
+
+// The values of 4 consecutive channels c .. c+3 (one 128-channel block) of
+// GEMM row r from the fp32 sources, with 16-byte loads; same arithmetic as
+// col_value.
 template <int kSrc>
-__global__ void __launch_bounds__(256) quantize_cols_kernel(const ColArgs a) {
-  __shared__ float vals[kTile][33];
-  const int64_t rb = blockIdx.x;
-  const int c0 = blockIdx.y * 32;
-  for (int i = threadIdx.x; i < kTile * 32; i += blockDim.x) {
-    const int r = i >> 5, c = i & 31;
-    vals[r][c] = (c0 + c < a.C) ? col_value<kSrc>(a, rb * kTile + r, c0 + c) : 0.0f;
+MOE_DEV void col_values4(const ColArgs& a, int64_t r, int c, float (&v)[4]) {
+  if (kSrc == kColH) {
+    const float* row = a.gu + r * 2 * a.I + (int64_t)(c / 128) * 256 + c % 128;
+    const float4 g4 = *reinterpret_cast<const float4*>(row);
+    const float4 u4 = *reinterpret_cast<const float4*>(row + 128);
+    const float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float sg = __fdividef(1.0f, 1.0f + __expf(-g[j]));
+      v[j] = g[j] * sg * u[j];
+    }
+  } else {
+    const int jj = c % 256, ch = (c / 256) * 128 + (jj % 128);
+    const float* row = a.gu + r * 2 * a.I + (int64_t)(c / 256) * 256 + (jj % 128);
+    const float4 g4 = *reinterpret_cast<const float4*>(row);
+    const float4 u4 = *reinterpret_cast<const float4*>(row + 128);
+    const float4 d4 = *reinterpret_cast<const float4*>(a.dh + r * a.I + ch);
+    const float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w};
+    const float d[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float sg = __fdividef(1.0f, 1.0f + __expf(-g[j]));
+      v[j] = jj < 128 ? d[j] * u[j] * (sg * (1.0f + g[j] * (1.0f - sg))) : d[j] * (g[j] * sg);
+    }
   }
-  __syncthreads();
-  const int c = threadIdx.x >> 3, part = threadIdx.x & 7;  // 8 threads per channel
+}
+
+// Codes and scale of each of the 32 channels c0.. of one 128-row block from
+// vals (8 threads per channel: the amax over the 128 rows, then 16 codes each).
+MOE_DEV void quantize_col_block(const ColArgs& a, const float (*vals)[33], int64_t rb, int c0) {
+  const int c = threadIdx.x >> 3, part = threadIdx.x & 7;
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(vals[part * 16 + i][c]));
@@ -263,20 +294,86 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(const ColArgs a) {
   for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (c0 + c >= a.C) return;
   const float s = tile_scale(amax);
-  uint4 out;
   uint32_t w[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k)
     w[k] = e4m3x4(__fmul_rn(vals[part * 16 + 4 * k][c], s), __fmul_rn(vals[part * 16 + 4 * k + 1][c], s),
                   __fmul_rn(vals[part * 16 + 4 * k + 2][c], s), __fmul_rn(vals[part * 16 + 4 * k + 3][c], s));
-  out = make_uint4(w[0], w[1], w[2], w[3]);
-  reinterpret_cast<uint4*>(a.codes + (int64_t)(c0 + c) * a.R + rb * kTile)[part] = out;
+  reinterpret_cast<uint4*>(a.codes + (int64_t)(c0 + c) * a.R + rb * kTile)[part] =
+      make_uint4(w[0], w[1], w[2], w[3]);
   if (part == 0) {
     if (a.b_operand)
       a.scales[rb * a.C + c0 + c] = __fdiv_rn(1.0f, s);
     else
       a.scales[(int64_t)(c0 + c) * (a.R / kTile) + rb] = s;
   }
+}
+
+// bf16 sources (dY scaled by the row's gate, x): one CTA per 128-row block
+// and 128 channels, the four 32-channel blocks' 16-byte loads all issued
+// before the first is used.
+template <int kSrc>
+__global__ void __launch_bounds__(256) quantize_cols_bf16_kernel(const ColArgs a) {
+  __shared__ float vals[kTile][33];
+  const int64_t rb = blockIdx.x;
+  const int cb = blockIdx.y * 128;
+  const int q = threadIdx.x & 3;  // channels 8q .. 8q + 7 of each 32-channel block
+  uint4 u[2][4];
+  float gate[2];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int64_t gr = rb * kTile + half * 64 + (threadIdx.x >> 2);
+    const int t = col_token(a, gr);
+    gate[half] = (kSrc == kColDy && t >= 0) ? a.row_gate[gr] : 1.0f;
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk)
+      u[half][blk] = t >= 0 ? *reinterpret_cast<const uint4*>(a.src + (int64_t)t * a.C + cb +
+                                                              32 * blk + 8 * q)
+                            : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint4 v = u[half][blk];
+      const float b[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                          bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+      const int r = half * 64 + (threadIdx.x >> 2);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        vals[r][8 * q + j] = kSrc == kColDy ? __fmul_rn(gate[half], b[j]) : b[j];
+    }
+    __syncthreads();
+    quantize_col_block(a, vals, rb, cb + 32 * blk);
+    __syncthreads();
+  }
+}
+
+template <int kSrc>
+__global__ void __launch_bounds__(256) quantize_cols_kernel(const ColArgs a) {
+  __shared__ float vals[kTile][33];
+  const int64_t rb = blockIdx.x;
+  const int c0 = blockIdx.y * 32;
+  if ((kSrc == kColH || kSrc == kColDgu) && c0 + 32 <= a.C) {
+    // whole 32-channel block of an fp32 source: 16-byte loads (4 channels)
+    const int q = threadIdx.x & 7;  // channels c0 + 4q .. + 3
+#pragma unroll
+    for (int quarter = 0; quarter < 4; ++quarter) {
+      const int r = quarter * 32 + (threadIdx.x >> 3);
+      const int64_t gr = rb * kTile + r;
+      float f[4] = {0, 0, 0, 0};
+      if (col_token(a, gr) >= 0) col_values4<kSrc>(a, gr, c0 + 4 * q, f);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) vals[r][4 * q + j] = f[j];
+    }
+  } else {
+    for (int i = threadIdx.x; i < kTile * 32; i += blockDim.x) {
+      const int r = i >> 5, c = i & 31;
+      vals[r][c] = (c0 + c < a.C) ? col_value<kSrc>(a, rb * kTile + r, c0 + c) : 0.0f;
+    }
+  }
+  __syncthreads();
+  quantize_col_block(a, vals, rb, c0);
 }
 
 int grid_for(int64_t units, int per_cta, int sm_count) {
@@ -316,9 +413,17 @@ cudaError_t launch_quantize_cols(int source, const int32_t* row_token, int64_t r
   ColArgs a{row_token, routed_cap, T, row_gate, static_cast<const __nv_bfloat16*>(src), gu, dh,
             R, C, I, codes, scales, b_operand};
   dim3 grid((unsigned)(R / kTile), (unsigned)((C + 31) / 32));
+  const bool bf16_wide = (source == kColDy || source == kColX) && C % 128 == 0;
+  dim3 grid128((unsigned)(R / kTile), (unsigned)(C / 128));
   switch (source) {
-    case kColDy: quantize_cols_kernel<kColDy><<<grid, 256, 0, stream>>>(a); break;
-    case kColX: quantize_cols_kernel<kColX><<<grid, 256, 0, stream>>>(a); break;
+    case kColDy:
+      if (bf16_wide) quantize_cols_bf16_kernel<kColDy><<<grid128, 256, 0, stream>>>(a);
+      else quantize_cols_kernel<kColDy><<<grid, 256, 0, stream>>>(a);
+      break;
+    case kColX:
+      if (bf16_wide) quantize_cols_bf16_kernel<kColX><<<grid128, 256, 0, stream>>>(a);
+      else quantize_cols_kernel<kColX><<<grid, 256, 0, stream>>>(a);
+      break;
     case kColH: quantize_cols_kernel<kColH><<<grid, 256, 0, stream>>>(a); break;
     default: quantize_cols_kernel<kColDgu><<<grid, 256, 0, stream>>>(a); break;
   }
