@@ -41,31 +41,29 @@ __global__ void __launch_bounds__(128) combine_kernel(const Row* __restrict__ y_
   __shared__ float s_gate[kMaxK];
   __shared__ int s_n;
   const int t = blockIdx.x;
-  if (threadIdx.x == 0) {
-    int id[kMaxK];
-    int n = 0;
-    for (int k = 0; k < K; ++k) {
-      const int e = ids[(int64_t)t * K + k];
-      const int64_t r = token_row[(int64_t)t * K + k];
-      const float g = gates != nullptr ? gates[(int64_t)t * K + k] : 1.0f;
-      if (r < 0 || r >= routed_cap) {
-        flag_status(status, kStatusBounds);
-        continue;
-      }
-      // insertion by ascending expert id
-      int j = n;
-      while (j > 0 && id[j - 1] > e) {
-        id[j] = id[j - 1];
-        s_row[j] = s_row[j - 1];
-        s_gate[j] = s_gate[j - 1];
-        --j;
-      }
-      id[j] = e;
-      s_row[j] = r;
-      s_gate[j] = g;
-      ++n;
+  // slot k (thread k) goes to position = the number of its token's slots with
+  // a lower expert id (the K experts of a token are distinct); slots whose
+  // row is out of range are dropped and flagged
+  if (threadIdx.x < K) {
+    const int k = threadIdx.x;
+    const int e = ids[(int64_t)t * K + k];
+    const int64_t r = token_row[(int64_t)t * K + k];
+    const float g = gates != nullptr ? gates[(int64_t)t * K + k] : 1.0f;
+    const bool ok = r >= 0 && r < routed_cap;
+    if (!ok) flag_status(status, kStatusBounds);
+    const unsigned mask = (1u << K) - 1u;
+    int pos = 0;
+    for (int j = 0; j < K; ++j) {
+      const int ej = __shfl_sync(mask, e, j);
+      const bool okj = __shfl_sync(mask, ok, j);
+      pos += (okj && ej < e) ? 1 : 0;
     }
-    s_n = n;
+    const int n_ok = __popc(__ballot_sync(mask, ok));
+    if (ok) {
+      s_row[pos] = r;
+      s_gate[pos] = g;
+    }
+    if (k == 0) s_n = n_ok;
   }
   __syncthreads();
   const int n = s_n;
@@ -73,15 +71,33 @@ __global__ void __launch_bounds__(128) combine_kernel(const Row* __restrict__ y_
   if (shared_row >= rows_total) return;
   const Row* ys = y_rows + shared_row * H;
   uint4* out = reinterpret_cast<uint4*>(y + (int64_t)t * H);
+  int64_t rows[kMaxK];
+  float gk[kMaxK];
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) {
+    rows[k] = k < n ? s_row[k] * H : 0;
+    gk[k] = k < n ? s_gate[k] : 0.0f;
+  }
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
     float acc[8];
     load8(ys, c, acc);
-    for (int k = 0; k < n; ++k) {
-      float f[8];
-      load8(y_rows + s_row[k] * H, c, f);
-      const float g = s_gate[k];
+    if (n == 8) {
+      // the common case: all eight rows' loads in flight before the adds
+      float f[8][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, f[i], acc[i]);
+      for (int k = 0; k < 8; ++k) load8(y_rows + rows[k], c, f[k]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(gk[k], f[k][i], acc[i]);
+    } else {
+      for (int k = 0; k < n; ++k) {
+        float f[8];
+        load8(y_rows + s_row[k] * H, c, f);
+        const float g = s_gate[k];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, f[i], acc[i]);
+      }
     }
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]);

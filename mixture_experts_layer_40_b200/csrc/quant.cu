@@ -84,8 +84,8 @@ __global__ void __launch_bounds__(256) quantize_scatter_kernel(
     int64_t routed_cap, uint8_t* __restrict__ a_q, float* __restrict__ a_s,
     uint32_t* __restrict__ status) {
   // 8 threads per tile, 16 consecutive elements each (two 128-bit loads, one
-  // 128-bit store of codes per destination row); two tiles in flight
-  constexpr int kPerThread = 2;
+  // 128-bit store of codes per destination row); four tiles in flight
+  constexpr int kPerThread = 4;
   const int sub = threadIdx.x & 7;
   const int tiles_per_row = H / kTile;
   const int64_t n_tiles = (int64_t)T * tiles_per_row;
