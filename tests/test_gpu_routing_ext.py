@@ -81,10 +81,14 @@ def _reconcile_grouped(gpu_ids, o_ids, score, gscore, k, groups, top):
 
 
 @pytest.mark.parametrize("t_count,k,top", [(4096, 8, 4), (333, 8, 4), (16384, 8, 4),
-                                           (16384, 6, 3)])
+                                           (16384, 6, 3), (16384, 8, 1), (16384, 4, 4)])
 def test_node_limited_v3_shape(t_count, k, top):
     """T = 16384 takes the wide logits tiles, whose epilogue also makes the
-    selection (group scores, kept groups, top-K) for each of its tokens."""
+    selection (group scores, kept groups, top-K) for each of its tokens: a
+    group is scored by its K/M best scores, which the epilogue takes as the
+    pair of maxima for K/M = 2 (K = 8, M = 4; K = 6, M = 3), the single
+    maximum for K/M = 1 (K = 4, M = 4) and a sorted list of eight for larger
+    K/M (K = 8, M = 1)."""
     w = I.Workload("g", T=t_count, H=7168, N=256, K=k, I=2048, bias_range=0.05, seed=11)
     xb = I.make_x(w)
     x, gw, b = I.bf16_bits_to_f32(xb), I.make_gate_w(w), I.make_bias(w)
