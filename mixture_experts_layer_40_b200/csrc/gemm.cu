@@ -24,6 +24,9 @@
 // thread can hold 128 fp32 totals plus a 64-column partial chunk.
 // Tiles are (group, m-tile, n-tile) with n fastest: the n-tiles of one row
 // tile run on neighbouring CTAs at the same time and share its A rows in L2.
+// A group's last row tile with at most 64 rows runs M=64 MMAs (half the
+// tensor-core work on padding rows); its rows sit in TMEM lanes 0-15 of each
+// 32-lane sub-partition, and those tiles' rows are stored one by one.
 // Both operands load with the default L2 policy: with the weight stream
 // marked evict-first (and A evict-last) the HBM reads matched one full read
 // of an expert's weights per row tile, i.e. the expert's second row tile
@@ -46,6 +49,9 @@ constexpr int kThreads = 384;
 constexpr int kEpiThreads = 256;
 constexpr int kMaxGroups = 1025;
 constexpr uint32_t kIdesc = make_idesc(kBM, kBN, 0u, 0u);  // E4M3 x E4M3 -> fp32
+// a group's last row tile with at most 64 rows: M=64 MMAs, whose rows land in
+// TMEM lanes (r mod 16) + 32 (r / 16), i.e. lanes 0-15 of each sub-partition
+constexpr uint32_t kIdesc64 = make_idesc(kBM / 2, kBN, 0u, 0u);
 // down epilogue: each epilogue warp stages 32 rows x kYCols fp32 columns of
 // its output tile in shared memory (swizzled over the 128-byte box row), two
 // buffers so that one TMA store is in flight while the next chunk is written
@@ -111,6 +117,7 @@ struct alignas(8) GemmShared {
   int abort;
   int prefix[kMaxGroups + 1];
   float amax[2][2][kBM];   // [tile parity][epilogue group][row]
+  int stage_m64[kMaxStages];  // the producer's flag for the MMA: a 64-row tile
 };
 
 MOE_DEV void decode_tile(int tile, const int* prefix, int n_groups, int n_tiles, int& g, int& n,
@@ -210,10 +217,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         decode_tile(tile, sh.prefix, p.n_groups, p.n_tiles, g, n, m);
         const int a_row = p.group_start[g] + m * kBM;
         const int b_row = g * p.b_rows + n * kBN;
+        const int m64 = (p.group_rows[g] - m * kBM) <= kBM / 2 ? 1 : 0;
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % kSt;
           const uint32_t ph = (uint32_t)(it / kSt) & 1u;
           if (!mbar_wait(smem_u32(&sh.empty[s]), ph ^ 1u, abort, p.status)) { ok = false; break; }
+          sh.stage_m64[s] = m64;  // ordered before the MMA's read by the full barrier
           const uint32_t full = smem_u32(&sh.full[s]);
           mbar_arrive_expect_tx(full, kStageBytes);
           const uint32_t sa = ring + s * kStageBytes;
@@ -247,10 +256,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = ring + s * kStageBytes;
           const uint32_t d = tmem_base + (uint32_t)(buf * kBN);
           const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sa + kABytes);
+          const uint32_t idesc = *reinterpret_cast<volatile int*>(&sh.stage_m64[s]) ? kIdesc64 : kIdesc;
 #pragma unroll
           for (int k4 = 0; k4 < kBK / 32; ++k4) {
             // +32 bytes along K = +2 in the descriptor's 16-byte address field
-            mma_f8(d, da + (uint64_t)(2 * k4), db + (uint64_t)(2 * k4), kIdesc, k4 > 0 ? 1u : 0u);
+            mma_f8(d, da + (uint64_t)(2 * k4), db + (uint64_t)(2 * k4), idesc, k4 > 0 ? 1u : 0u);
           }
           mma_commit(smem_u32(&sh.tfull[buf]));
           mma_commit(smem_u32(&sh.empty[s]));
@@ -278,9 +288,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t acc2[64];  // the 128 fp32 totals as packed pairs
       int g, n, m;
       decode_tile(tile, sh.prefix, p.n_groups, p.n_tiles, g, n, m);
-      const int valid = p.group_rows[g] - m * kBM;
-      const int64_t grow = (int64_t)p.group_start[g] + m * kBM + row;
-      const bool live = row < valid;
+      const int valid_rows = p.group_rows[g] - m * kBM;
+      // a 64-row tile: lanes 0-15 of each sub-partition hold rows 16q + lane
+      const bool m64 = valid_rows <= kBM / 2;
+      const int r_in = m64 ? (lane < 16 ? 16 * quarter + lane : kBM) : row;
+      const int valid = m64 ? 0 : valid_rows;  // 64-row tiles store row by row
+      const int64_t grow = (int64_t)p.group_start[g] + m * kBM + r_in;
+      const bool live = r_in < valid_rows;
       const float* sa_ptr = p.a_s + (live ? grow : 0) * kb_n;
       const float* sb0 = p.b_s + ((int64_t)g * b_blocks + 2 * n + (kUp ? 0 : eg)) * kb_n;
       const float* sb1 = p.b_s + ((int64_t)g * b_blocks + 2 * n + 1) * kb_n;
