@@ -108,25 +108,42 @@ __global__ void __launch_bounds__(256) dy_rows_quantize_kernel(
 __global__ void __launch_bounds__(256) swiglu_backward_kernel(
     const float* __restrict__ gu, const float* __restrict__ dh, int64_t rows, int I,
     uint8_t* __restrict__ q, float* __restrict__ qs) {
+  // two units per thread per round: their six 16-byte loads each are issued
+  // before either is used
+  constexpr int kU = 2;
   const int sub = threadIdx.x & 15;
   const int blocks = I / kTile;
   const int64_t n_units = rows * blocks;
-  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_units; base += (int64_t)gridDim.x * 16) {
-    const int64_t unit = base + (threadIdx.x >> 4);
-    const bool live = unit < n_units;
-    const int64_t r = live ? unit / blocks : 0;
-    const int c = live ? (int)(unit - r * blocks) : 0;
-    float dg[8], du[8];
-    float ag = 0.0f, au = 0.0f;
-    if (live) {
+  const int64_t step = (int64_t)gridDim.x * 16;
+  for (int64_t base = (int64_t)blockIdx.x * 16; base < n_units; base += step * kU) {
+    float4 g0[kU], g1[kU], u0[kU], u1[kU], h0[kU], h1[kU];
+    int64_t unit[kU];
+#pragma unroll
+    for (int v = 0; v < kU; ++v) {
+      unit[v] = base + v * step + (threadIdx.x >> 4);
+      const bool live = unit[v] < n_units;
+      const int64_t r = live ? unit[v] / blocks : 0;
+      const int c = live ? (int)(unit[v] - r * blocks) : 0;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
       const float4* gp = reinterpret_cast<const float4*>(gu + r * 2 * I + (int64_t)c * 2 * kTile);
       const float4* hp = reinterpret_cast<const float4*>(dh + r * I + (int64_t)c * kTile);
-      const float4 g0 = __ldg(gp + 2 * sub), g1 = __ldg(gp + 2 * sub + 1);
-      const float4 u0 = __ldg(gp + 32 + 2 * sub), u1 = __ldg(gp + 32 + 2 * sub + 1);
-      const float4 h0 = __ldg(hp + 2 * sub), h1 = __ldg(hp + 2 * sub + 1);
-      const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-      const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+      g0[v] = live ? __ldg(gp + 2 * sub) : z;
+      g1[v] = live ? __ldg(gp + 2 * sub + 1) : z;
+      u0[v] = live ? __ldg(gp + 32 + 2 * sub) : z;
+      u1[v] = live ? __ldg(gp + 32 + 2 * sub + 1) : z;
+      h0[v] = live ? __ldg(hp + 2 * sub) : z;
+      h1[v] = live ? __ldg(hp + 2 * sub + 1) : z;
+    }
+#pragma unroll
+    for (int v = 0; v < kU; ++v) {
+      const bool live = unit[v] < n_units;
+      const int64_t r = live ? unit[v] / blocks : 0;
+      const int c = live ? (int)(unit[v] - r * blocks) : 0;
+      const float gv[8] = {g0[v].x, g0[v].y, g0[v].z, g0[v].w, g1[v].x, g1[v].y, g1[v].z, g1[v].w};
+      const float uv[8] = {u0[v].x, u0[v].y, u0[v].z, u0[v].w, u1[v].x, u1[v].y, u1[v].z, u1[v].w};
+      const float hv[8] = {h0[v].x, h0[v].y, h0[v].z, h0[v].w, h1[v].x, h1[v].y, h1[v].z, h1[v].w};
+      float dg[8], du[8];
+      float ag = 0.0f, au = 0.0f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         // sigmoid with the hardware exp2 and reciprocal, as the forward's SiLU
@@ -137,28 +154,25 @@ __global__ void __launch_bounds__(256) swiglu_backward_kernel(
         ag = fmaxf(ag, fabsf(dg[i]));
         au = fmaxf(au, fabsf(du[i]));
       }
-    } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dg[i] = du[i] = 0.0f;
-    }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) {
-      ag = fmaxf(ag, __shfl_xor_sync(0xffffffffu, ag, o));
-      au = fmaxf(au, __shfl_xor_sync(0xffffffffu, au, o));
-    }
-    if (!live) continue;
-    const float sg_ = tile_scale(ag), su = tile_scale(au);
-    uint2 og, ou;
-    og.x = e4m3x4(__fmul_rn(dg[0], sg_), __fmul_rn(dg[1], sg_), __fmul_rn(dg[2], sg_), __fmul_rn(dg[3], sg_));
-    og.y = e4m3x4(__fmul_rn(dg[4], sg_), __fmul_rn(dg[5], sg_), __fmul_rn(dg[6], sg_), __fmul_rn(dg[7], sg_));
-    ou.x = e4m3x4(__fmul_rn(du[0], su), __fmul_rn(du[1], su), __fmul_rn(du[2], su), __fmul_rn(du[3], su));
-    ou.y = e4m3x4(__fmul_rn(du[4], su), __fmul_rn(du[5], su), __fmul_rn(du[6], su), __fmul_rn(du[7], su));
-    uint8_t* row = q + r * 2 * I + (int64_t)c * 2 * kTile;
-    reinterpret_cast<uint2*>(row)[sub] = og;
-    reinterpret_cast<uint2*>(row + kTile)[sub] = ou;
-    if (sub == 0) {
-      qs[r * 2 * blocks + 2 * c] = sg_;
-      qs[r * 2 * blocks + 2 * c + 1] = su;
+      for (int o = 8; o > 0; o >>= 1) {
+        ag = fmaxf(ag, __shfl_xor_sync(0xffffffffu, ag, o));
+        au = fmaxf(au, __shfl_xor_sync(0xffffffffu, au, o));
+      }
+      if (!live) continue;
+      const float sg_ = tile_scale(ag), su = tile_scale(au);
+      uint2 og, ou;
+      og.x = e4m3x4(__fmul_rn(dg[0], sg_), __fmul_rn(dg[1], sg_), __fmul_rn(dg[2], sg_), __fmul_rn(dg[3], sg_));
+      og.y = e4m3x4(__fmul_rn(dg[4], sg_), __fmul_rn(dg[5], sg_), __fmul_rn(dg[6], sg_), __fmul_rn(dg[7], sg_));
+      ou.x = e4m3x4(__fmul_rn(du[0], su), __fmul_rn(du[1], su), __fmul_rn(du[2], su), __fmul_rn(du[3], su));
+      ou.y = e4m3x4(__fmul_rn(du[4], su), __fmul_rn(du[5], su), __fmul_rn(du[6], su), __fmul_rn(du[7], su));
+      uint8_t* row = q + r * 2 * I + (int64_t)c * 2 * kTile;
+      reinterpret_cast<uint2*>(row)[sub] = og;
+      reinterpret_cast<uint2*>(row + kTile)[sub] = ou;
+      if (sub == 0) {
+        qs[r * 2 * blocks + 2 * c] = sg_;
+        qs[r * 2 * blocks + 2 * c + 1] = su;
+      }
     }
   }
 }
