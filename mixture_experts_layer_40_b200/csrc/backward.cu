@@ -20,24 +20,48 @@ namespace moe {
 
 namespace {
 
-// One CTA per 128x128 block of one group: bytes through shared memory.
+// One CTA per 128x128 block of one group. The block comes in with 16-byte
+// loads as 32-bit words, each thread transposes 4x4-byte sub-blocks in
+// registers (byte permutes), and the transposed block goes out with 16-byte
+// stores; both shared-memory arrays are padded to 33 words a row.
 __global__ void __launch_bounds__(256) transpose_blocks_kernel(const uint8_t* __restrict__ w,
                                                                const float* __restrict__ s,
                                                                int64_t rows, int64_t cols,
                                                                uint8_t* __restrict__ wt,
                                                                float* __restrict__ st) {
-  __shared__ uint8_t tile[kTile][kTile + 4];
+  __shared__ uint32_t tin[kTile][kTile / 4 + 1];
+  __shared__ uint32_t tout[kTile][kTile / 4 + 1];
   const int64_t cb = blockIdx.x, rb = blockIdx.y, g = blockIdx.z;
   const uint8_t* src = w + g * rows * cols + rb * kTile * cols + cb * kTile;
-  for (int i = threadIdx.x; i < kTile * kTile; i += blockDim.x) {
-    const int r = i / kTile, c = i % kTile;
-    tile[r][c] = src[(int64_t)r * cols + c];
+  // 128 rows x 8 chunks of 16 bytes
+  for (int i = threadIdx.x; i < kTile * 8; i += blockDim.x) {
+    const int r = i >> 3, q = i & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(src + (int64_t)r * cols + 16 * q);
+    tin[r][4 * q + 0] = v.x;
+    tin[r][4 * q + 1] = v.y;
+    tin[r][4 * q + 2] = v.z;
+    tin[r][4 * q + 3] = v.w;
+  }
+  __syncthreads();
+  // 32 x 32 sub-blocks of 4x4 bytes: word bj of source rows 4bi..4bi+3 becomes
+  // word bi of destination rows 4bj..4bj+3
+  for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x) {
+    const int bi = i >> 5, bj = i & 31;
+    const uint32_t a0 = tin[4 * bi + 0][bj], a1 = tin[4 * bi + 1][bj];
+    const uint32_t a2 = tin[4 * bi + 2][bj], a3 = tin[4 * bi + 3][bj];
+    const uint32_t t0 = __byte_perm(a0, a1, 0x5140), t1 = __byte_perm(a2, a3, 0x5140);
+    const uint32_t t2 = __byte_perm(a0, a1, 0x7362), t3 = __byte_perm(a2, a3, 0x7362);
+    tout[4 * bj + 0][bi] = __byte_perm(t0, t1, 0x5410);
+    tout[4 * bj + 1][bi] = __byte_perm(t0, t1, 0x7632);
+    tout[4 * bj + 2][bi] = __byte_perm(t2, t3, 0x5410);
+    tout[4 * bj + 3][bi] = __byte_perm(t2, t3, 0x7632);
   }
   __syncthreads();
   uint8_t* dst = wt + g * rows * cols + cb * kTile * rows + rb * kTile;
-  for (int i = threadIdx.x; i < kTile * kTile; i += blockDim.x) {
-    const int r = i / kTile, c = i % kTile;  // destination row r (a source column)
-    dst[(int64_t)r * rows + c] = tile[c][r];
+  for (int i = threadIdx.x; i < kTile * 8; i += blockDim.x) {
+    const int r = i >> 3, q = i & 7;  // destination row r (a source column)
+    *reinterpret_cast<uint4*>(dst + (int64_t)r * rows + 16 * q) =
+        make_uint4(tout[r][4 * q + 0], tout[r][4 * q + 1], tout[r][4 * q + 2], tout[r][4 * q + 3]);
   }
   if (threadIdx.x == 0) {
     const int64_t rbn = rows / kTile, cbn = cols / kTile;
