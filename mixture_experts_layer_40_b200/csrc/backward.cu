@@ -93,6 +93,13 @@ __global__ void __launch_bounds__(256) dy_rows_quantize_kernel(
     }
     const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                         bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    // the tile's amax of |dy|, once: rounding is monotone, so the amax of the
+    // rounded products |fp32(g * dy)| is fp32(|g| * amax |dy|) for every gate
+    float amax_f = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax_f = fmaxf(amax_f, fabsf(f[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax_f = fmaxf(amax_f, __shfl_xor_sync(0xffffffffu, amax_f, o));
     for (int k = -1; k < K; ++k) {
       int64_t r = routed_cap + t;
       float g = 1.0f;
@@ -101,14 +108,9 @@ __global__ void __launch_bounds__(256) dy_rows_quantize_kernel(
         g = __shfl_sync(0xffffffffu, my_gate, k, 16);
       }
       float d[8];
-      float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        d[i] = __fmul_rn(g, f[i]);
-        amax = fmaxf(amax, fabsf(d[i]));
-      }
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      for (int i = 0; i < 8; ++i) d[i] = __fmul_rn(g, f[i]);
+      const float amax = __fmul_rn(fabsf(g), amax_f);
       if (!live) continue;
       if (k >= 0 && (r < 0 || r >= routed_cap)) {
         if (sub == 0) flag_status(status, kStatusBounds);
