@@ -133,7 +133,9 @@ typedef struct {
   size_t topk_ids;      /* int32 [T, K] (used when the caller passes none) */
   size_t topk_gates;    /* float [T, K] (used when the caller passes none) */
   size_t logits;        /* float [T, N] gate logits x . e_i */
-  size_t a_q;           /* E4M3 [rows_total, H]: GEMM1 input rows; x_q in the shared rows */
+  size_t a_q;           /* E4M3 [rows_total, H]: GEMM1 input rows; x_q in the shared rows
+                           (before the rows are written, the router's partial
+                           logits when it splits the gate GEMM's reduction) */
   size_t a_s;           /* float [rows_total, H/128] */
   size_t h_q;           /* E4M3 [rows_total, I]: SwiGLU output, 1x128 re-quantised */
   size_t h_s;           /* float [rows_total, I/128] */
