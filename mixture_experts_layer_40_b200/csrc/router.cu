@@ -3,8 +3,13 @@
 // Multi-Token Prediction, and FP8 Training at 671B Scale" (trishampatil.com),
 // section III, "The mechanism": the bias enters only the TopK comparison and
 // the gate is the unbiased affinity normalised over the K chosen. Gating stays
-// in fp32 ("DeepSeek-V3, explained", recipe step 7), so the logits come from an
-// fp32 FMA GEMM of the bf16 input and the fp32 centroids.
+// in fp32 ("DeepSeek-V3, explained", recipe step 7), so the logits are fp32
+// sums of the bf16 input times the fp32 centroids: either an fp32 FMA GEMM
+// (logits_kernel, the no-allocation route) or BF16 tensor-core MMAs against
+// the centroids split exactly into three bf16 terms with fp32 accumulation
+// (logits_tc_kernel, and logits_tc_wide_kernel whose 256 x 256 tiles either
+// cover the whole depth, then at N = 256 also make the selection in their
+// epilogue, or a slice of it that splitk_reduce_kernel sums).
 #include <algorithm>
 
 #include "kernels.cuh"
