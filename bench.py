@@ -526,6 +526,27 @@ def run_ours(args, w, rank, world, local_rank):
     stream.wait_event(ev_out[1])
     e_end.record(stream)
     barrier()
+    # ------------------------------------------------ the same step as a CUDA graph
+    # captured once and replayed (one graph launch per step instead of one
+    # call per kernel); one GPU only (the count all-reduce is not captured)
+    graph = None
+    if world == 1 and args.steps > 0:
+        gstep = layer.graphed_step(x, bias, y, gamma=w.gamma)
+        for _ in range(3):
+            gstep.replay()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            gstep.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        if layer.status() != 0:
+            raise RuntimeError("device status error in the graph replays")
+        g_ms = g0.elapsed_time(g1) / args.steps
+        graph = {"value": w.T / (g_ms * 1e-3), "unit": "tokens/s", "ms_per_step": g_ms,
+                 "note": "the timed step (forward + bias update, no stage events) captured "
+                         "once as a CUDA graph and replayed"}
+        del gstep
     # ------------------------------------------------ controller trace (untimed)
     # workloads with several steps (the skewed one: 50) replay forward + bias
     # update from the starting bias and record each step's max/mean load
@@ -630,6 +651,7 @@ def run_ours(args, w, rank, world, local_rank):
         "clocks": clk,
         "controller": trace,
         "backward": bwd,
+        "graph": graph,
         "balance_stats": {"ms": bal_ms, "seq_len": seq_len,
                           "note": "moe_balance_stats after the step, not part of it"},
     }

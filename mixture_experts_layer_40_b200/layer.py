@@ -157,6 +157,12 @@ class MoELayer:
     def update_bias(self, bias: torch.Tensor, gamma: float, stream=None) -> None:
         capi.moe_update_bias(bias, self.counts, self.N, self.T, self.K, gamma, stream)
 
+    def graphed_step(self, x: torch.Tensor, bias: torch.Tensor, y: torch.Tensor | None = None,
+                     gamma: float | None = None) -> "GraphedStep":
+        """The layer step on fixed buffers (x, bias, y) captured once as a CUDA
+        graph: forward, and with gamma also the bias update. See GraphedStep."""
+        return GraphedStep(self, x, bias, y, gamma)
+
     def status(self, stream=None) -> int:
         return capi.moe_get_status(self.ws, stream)
 
@@ -165,6 +171,40 @@ class MoELayer:
         off = getattr(self.layout, name)
         n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
         return self.ws[off:off + n].view(dtype).view(*shape)
+
+
+class GraphedStep:
+    """One layer step captured as a CUDA graph and replayed: the same kernels
+    with the same arguments as layer.forward (and layer.update_bias when gamma
+    is given), launched by one graph launch instead of one call per kernel.
+    The library allocates nothing and launches everything on the stream it
+    is given, so the capture holds the whole step; the tensor maps are
+    encoded at capture time and hold the buffers' addresses, so x, bias and y
+    must stay the same tensors (write new inputs into x in place). One
+    uncaptured forward runs first, so that the one-time set-up per device
+    (kernel attributes) happens outside the capture; it leaves the bias
+    untouched."""
+
+    def __init__(self, layer: MoELayer, x: torch.Tensor, bias: torch.Tensor,
+                 y: torch.Tensor | None = None, gamma: float | None = None):
+        self.layer, self.x, self.bias, self.gamma = layer, x, bias, gamma
+        self.y = y if y is not None else torch.empty((layer.T, layer.H), dtype=torch.bfloat16,
+                                                     device=layer.device)
+        side = torch.cuda.Stream(layer.device)
+        side.wait_stream(torch.cuda.current_stream(layer.device))
+        with torch.cuda.stream(side):
+            layer.forward(x, bias, self.y)
+        torch.cuda.current_stream(layer.device).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            layer.forward(x, bias, self.y)
+            if gamma is not None:
+                layer.update_bias(bias, gamma)
+
+    def replay(self) -> torch.Tensor:
+        """Runs the step on the current stream; returns y (the same tensor)."""
+        self.graph.replay()
+        return self.y
 
 
 # ---------------------------------------------------------------- controller state
