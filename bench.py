@@ -545,7 +545,8 @@ def run_ours(args, w, rank, world, local_rank):
         g_ms = g0.elapsed_time(g1) / args.steps
         graph = {"value": w.T / (g_ms * 1e-3), "unit": "tokens/s", "ms_per_step": g_ms,
                  "note": "the timed step (forward + bias update, no stage events) captured "
-                         "once as a CUDA graph and replayed"}
+                         "once as a CUDA graph and replayed; measured after the end-to-end "
+                         "run, on a warmer GPU under the power cap than the timed region"}
         del gstep
     # ------------------------------------------------ controller trace (untimed)
     # workloads with several steps (the skewed one: 50) replay forward + bias
