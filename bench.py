@@ -260,6 +260,16 @@ def step_launches(T: int, N: int, K: int, G: int, M: int, H: int) -> int:
     return router_launches(T, N, K, G, M, H) + 3 + 5
 
 
+def ep_step_launches(T: int, N: int, K: int, G: int, M: int, H: int) -> int:
+    """The library's kernels in one expert-parallel step on a rank that
+    receives rows (csrc/ep.cu; the centroids are split once at set-up): the
+    router's, then count, slot and pack (the send plan); the shared expert's
+    two GEMMs; on the receiver the index kernel, rank + scan + place, the row
+    gather, two GEMMs and the per-row reduction; the combine; the bias
+    update."""
+    return router_launches(T, N, K, G, M, H) + 3 + 2 + 1 + 3 + 1 + 2 + 1 + 1 + 1
+
+
 def oracle_sample_step(w, x, gate_w, bias, ew, step: int, sample_tokens: int = 512,
                        groups: int = 1, shared_rows: int = 64, node_limit: tuple = (0, 0)):
     """One bounded sample of the layer on the CPU oracle; returns its time
@@ -765,7 +775,8 @@ def run_ep(args, w, rank, world, local_rank):
                 "config": dict(run_config(args, w, world),
                                parallelism=f"ep{world} (routed experts sharded over ranks; own "
                                            f"batch per GPU)"),
-                "gpu_launches": 17 * args.steps,
+                "gpu_launches": ep_step_launches(w.T, w.N, w.K, args.groups, args.topk_groups,
+                                                 w.H) * args.steps,
                 "e2e": {"value": w.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                         "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2,
                         "copies": "pinned host buffers, on the compute stream"},

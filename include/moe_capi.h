@@ -438,8 +438,10 @@ int64_t moe_ep_row_bytes(moe_shape sh);
 size_t moe_ep_dispatch_workspace_size(moe_shape sh, int32_t W);
 
 /*
- * Step 1. gate_w: float [N, H]; x: bf16 [T, H]; bias: float [N]. Optional
- * outputs as in moe_forward (topk_ids and topk_gates [T, K] with global expert
+ * Step 1. gate_w: float [N, H]; gate_split_opt: NULL, or gate_w's three bf16
+ * terms [3, N, H] made by moe_split_gate (16-byte aligned; NULL: they are made
+ * on every call); x: bf16 [T, H]; bias: float [N]. Optional outputs as in
+ * moe_forward (topk_ids and topk_gates [T, K] with global expert
  * ids; counts [N] of this rank's tokens, for moe_update_bias after a sum over
  * ranks). send: uint8 [send_cap, moe_ep_row_bytes], 16-byte aligned
  * (T * min(W, K) rows always suffice; a row beyond send_cap is dropped and
@@ -447,7 +449,8 @@ size_t moe_ep_dispatch_workspace_size(moe_shape sh, int32_t W);
  * 256-byte aligned; it keeps the send slots and the shared-expert rows for
  * steps 1b and 5. T = 0 clears send_counts and counts only.
  */
-int moe_ep_dispatch(moe_shape sh, int32_t W, const float* gate_w, const void* x, const float* bias,
+int moe_ep_dispatch(moe_shape sh, int32_t W, const float* gate_w, const void* gate_split_opt,
+                    const void* x, const float* bias,
                     int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
                     uint8_t* send, int64_t send_cap, int32_t* send_counts, void* ws,
                     size_t ws_bytes, void* stream);
@@ -505,9 +508,9 @@ int moe_ep_combine(moe_shape sh, int32_t W, const float* ret, int64_t ret_rows, 
 size_t moe_ep_peer_expert_workspace_size(moe_shape sh, int32_t W, int32_t T_cap);
 
 int moe_ep_dispatch_peer(moe_shape sh, int32_t W, int32_t rank, int32_t T_cap,
-                         const float* gate_w, const void* x, const float* bias,
-                         int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
-                         uint8_t* const* peer_recv, int32_t* const* peer_counts,
+                         const float* gate_w, const void* gate_split_opt, const void* x,
+                         const float* bias, int32_t* topk_ids_opt, float* topk_gates_opt,
+                         int32_t* counts_opt, uint8_t* const* peer_recv, int32_t* const* peer_counts,
                          int32_t* send_counts_opt, void* ws, size_t ws_bytes, void* stream);
 
 /* recv, recv_counts: this rank's own buffers; peer_ret: device array [W] of

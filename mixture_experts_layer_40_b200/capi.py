@@ -79,8 +79,8 @@ SIGNATURES = {
                                             _P]),
     "moe_ep_row_bytes": (_I64, [moe_shape]),
     "moe_ep_dispatch_workspace_size": (_SZ, [moe_shape, _I32]),
-    "moe_ep_dispatch": (ctypes.c_int, [moe_shape, _I32, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P,
-                                       _SZ, _P]),
+    "moe_ep_dispatch": (ctypes.c_int, [moe_shape, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P,
+                                       _P, _SZ, _P]),
     "moe_ep_shared": (ctypes.c_int, [moe_shape, _I32, ctypes.POINTER(moe_weights), _P, _SZ, _P]),
     "moe_ep_expert_workspace_size": (_SZ, [moe_shape, _I32, _I64, _I64]),
     "moe_ep_experts": (ctypes.c_int, [moe_shape, _I32, ctypes.POINTER(moe_weights), _P, _I64,
@@ -88,7 +88,7 @@ SIGNATURES = {
     "moe_ep_combine": (ctypes.c_int, [moe_shape, _I32, _P, _I64, _P, _SZ, _P, _P]),
     "moe_ep_peer_expert_workspace_size": (_SZ, [moe_shape, _I32, _I32]),
     "moe_ep_dispatch_peer": (ctypes.c_int, [moe_shape, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P,
-                                            _P, _P, _P, _P, _SZ, _P]),
+                                            _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_ep_experts_peer": (ctypes.c_int, [moe_shape, _I32, _I32, _I32,
                                            ctypes.POINTER(moe_weights), _P, _P, _P, _P, _SZ, _P]),
     "moe_ep_combine_peer": (ctypes.c_int, [moe_shape, _I32, _I32, _P, _P, _SZ, _P, _P]),
@@ -301,10 +301,12 @@ def moe_ep_expert_workspace_size(sh: moe_shape, W: int, R: int, pairs: int) -> i
 
 
 def moe_ep_dispatch(sh: moe_shape, W: int, gate_w, x, bias, send, send_counts, ws,
-                    topk_ids=None, topk_gates=None, counts=None, stream=None):
-    """send: uint8 [send_cap, moe_ep_row_bytes(sh)]; send_counts: int32 [W, 2]."""
+                    topk_ids=None, topk_gates=None, counts=None, stream=None, gate_split=None):
+    """send: uint8 [send_cap, moe_ep_row_bytes(sh)]; send_counts: int32 [W, 2];
+    gate_split: None, or bf16 [3, N, H] from moe_split_gate."""
     _check("moe_ep_dispatch", LIB.moe_ep_dispatch(
-        sh, W, _ptr(gate_w, torch.float32, "gate_w"), _ptr(x, torch.bfloat16, "x"),
+        sh, W, _ptr(gate_w, torch.float32, "gate_w"),
+        _ptr(gate_split, torch.bfloat16, "gate_split"), _ptr(x, torch.bfloat16, "x"),
         _ptr(bias, torch.float32, "bias"), _ptr(topk_ids, torch.int32, "topk_ids"),
         _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
         _ptr(send, torch.uint8, "send"), send.shape[0] if send is not None else 0,
@@ -338,10 +340,12 @@ def moe_ep_peer_expert_workspace_size(sh: moe_shape, W: int, T_cap: int) -> int:
 
 def moe_ep_dispatch_peer(sh: moe_shape, W: int, rank: int, T_cap: int, gate_w, x, bias,
                          peer_recv, peer_counts, ws, topk_ids=None, topk_gates=None, counts=None,
-                         send_counts=None, stream=None):
-    """peer_recv, peer_counts: int64 device tensors [W] of device pointers."""
+                         send_counts=None, stream=None, gate_split=None):
+    """peer_recv, peer_counts: int64 device tensors [W] of device pointers;
+    gate_split as in moe_ep_dispatch."""
     _check("moe_ep_dispatch_peer", LIB.moe_ep_dispatch_peer(
-        sh, W, rank, T_cap, _ptr(gate_w, torch.float32, "gate_w"), _ptr(x, torch.bfloat16, "x"),
+        sh, W, rank, T_cap, _ptr(gate_w, torch.float32, "gate_w"),
+        _ptr(gate_split, torch.bfloat16, "gate_split"), _ptr(x, torch.bfloat16, "x"),
         _ptr(bias, torch.float32, "bias"), _ptr(topk_ids, torch.int32, "topk_ids"),
         _ptr(topk_gates, torch.float32, "topk_gates"), _ptr(counts, torch.int32, "counts"),
         _ptr(peer_recv, torch.int64, "peer_recv"), _ptr(peer_counts, torch.int64, "peer_counts"),

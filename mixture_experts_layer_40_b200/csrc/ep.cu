@@ -535,7 +535,8 @@ __global__ void ep_zero_counts_kernel(int32_t* const* peer_counts, int W, int ra
   __threadfence_system();
 }
 
-int dispatch_impl(const moe_shape& sh, int W, int rank, const float* gate_w, const void* x,
+int dispatch_impl(const moe_shape& sh, int W, int rank, const float* gate_w,
+                  const void* gate_split, const void* x,
                   const float* bias, int32_t* topk_ids_opt, float* topk_gates_opt,
                   int32_t* counts_opt, SendRows dst, int32_t* const* peer_counts,
                   int32_t* send_counts_opt, void* ws, size_t ws_bytes, cudaStream_t s) {
@@ -543,6 +544,7 @@ int dispatch_impl(const moe_shape& sh, int W, int rank, const float* gate_w, con
   if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
   const SourceLayout L = source_layout(sh, W);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (!aligned(gate_split, 16)) return MOE_ERR_ALIGN;
   uint32_t* status = at<uint32_t>(ws, L.status);
   int32_t* counts = counts_opt ? counts_opt : at<int32_t>(ws, L.counts);
   int32_t* send_counts = send_counts_opt ? send_counts_opt : at<int32_t>(ws, L.send_counts);
@@ -564,7 +566,8 @@ int dispatch_impl(const moe_shape& sh, int W, int rank, const float* gate_w, con
   float* gates = topk_gates_opt ? topk_gates_opt : at<float>(ws, L.topk_gates);
   e = launch_router_tc(x, gate_w, bias, sh.T, sh.H, sh.N, sh.K, sh.G, sh.M,
                        at<__nv_bfloat16>(ws, L.gate_split), at<float>(ws, L.logits), ids, gates,
-                       counts, status, s, sms, nullptr, at<float>(ws, L.splitk),
+                       counts, status, s, sms, static_cast<const __nv_bfloat16*>(gate_split),
+                       at<float>(ws, L.splitk),
                        router_splitk_bytes(sh.T, sh.N, sh.H));
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   int32_t* send_slot = at<int32_t>(ws, L.send_slot);
@@ -689,7 +692,8 @@ size_t moe_ep_expert_workspace_size(moe_shape sh, int32_t W, int64_t R, int64_t 
   return expert_layout(sh, W, R, pairs).total;
 }
 
-int moe_ep_dispatch(moe_shape sh, int32_t W, const float* gate_w, const void* x, const float* bias,
+int moe_ep_dispatch(moe_shape sh, int32_t W, const float* gate_w, const void* gate_split_opt,
+                    const void* x, const float* bias,
                     int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
                     uint8_t* send, int64_t send_cap, int32_t* send_counts, void* ws,
                     size_t ws_bytes, void* stream) {
@@ -698,8 +702,9 @@ int moe_ep_dispatch(moe_shape sh, int32_t W, const float* gate_w, const void* x,
   if (sh.T > 0 && !send) return MOE_ERR_NULL;
   if (!aligned(send, 16)) return MOE_ERR_ALIGN;
   SendRows dst{send, send_cap, nullptr, 0, row_bytes_of(sh)};
-  return dispatch_impl(sh, W, 0, gate_w, x, bias, topk_ids_opt, topk_gates_opt, counts_opt, dst,
-                       nullptr, send_counts, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+  return dispatch_impl(sh, W, 0, gate_w, gate_split_opt, x, bias, topk_ids_opt, topk_gates_opt,
+                       counts_opt, dst, nullptr, send_counts, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int moe_ep_shared(moe_shape sh, int32_t W, const moe_weights* w_local, void* ws, size_t ws_bytes,
@@ -753,15 +758,15 @@ size_t moe_ep_peer_expert_workspace_size(moe_shape sh, int32_t W, int32_t T_cap)
 }
 
 int moe_ep_dispatch_peer(moe_shape sh, int32_t W, int32_t rank, int32_t T_cap,
-                         const float* gate_w, const void* x, const float* bias,
-                         int32_t* topk_ids_opt, float* topk_gates_opt, int32_t* counts_opt,
-                         uint8_t* const* peer_recv, int32_t* const* peer_counts,
+                         const float* gate_w, const void* gate_split_opt, const void* x,
+                         const float* bias, int32_t* topk_ids_opt, float* topk_gates_opt,
+                         int32_t* counts_opt, uint8_t* const* peer_recv, int32_t* const* peer_counts,
                          int32_t* send_counts_opt, void* ws, size_t ws_bytes, void* stream) {
   if (!peer_ok(sh, W, rank, T_cap)) return MOE_ERR_SHAPE;
   if (!peer_recv || !peer_counts) return MOE_ERR_NULL;
   SendRows dst{nullptr, 0, peer_recv, (int64_t)rank * T_cap, row_bytes_of(sh)};
-  return dispatch_impl(sh, W, rank, gate_w, x, bias, topk_ids_opt, topk_gates_opt, counts_opt, dst,
-                       peer_counts, send_counts_opt, ws, ws_bytes,
+  return dispatch_impl(sh, W, rank, gate_w, gate_split_opt, x, bias, topk_ids_opt,
+                       topk_gates_opt, counts_opt, dst, peer_counts, send_counts_opt, ws, ws_bytes,
                        static_cast<cudaStream_t>(stream));
 }
 

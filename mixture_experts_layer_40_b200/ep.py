@@ -85,13 +85,15 @@ class ExpertParallelMoE:
     gate_w: float32 [N, H] (all experts); w13, s13, w2, s2: this rank's N/W + 1
     weight sets (see local_weights), on this rank's GPU. T is the number of
     tokens this rank routes per step (the batch may be smaller: forward takes
-    any T' <= T).
+    any T' <= T). With presplit_gate the centroids' three bf16 terms are made
+    once here (resplit_gate after changing gate_w); without them every
+    dispatch splits again.
     """
 
     def __init__(self, T: int, H: int, N: int, K: int, I: int, W: int, rank: int,
                  gate_w: torch.Tensor, w13: torch.Tensor, s13: torch.Tensor, w2: torch.Tensor,
                  s2: torch.Tensor, groups: int = 0, topk_groups: int = 0, group=None,
-                 peer: bool = False):
+                 peer: bool = False, presplit_gate: bool = True):
         self.T, self.H, self.N, self.K, self.I, self.W, self.rank = T, H, N, K, I, W, rank
         self.G, self.M = groups, topk_groups
         self.group = group
@@ -103,6 +105,10 @@ class ExpertParallelMoE:
         self.row_bytes = capi.moe_ep_row_bytes(sh)
         self._keep = (gate_w, w13, s13, w2, s2)
         self.gate_w = gate_w
+        self.gate_split = None
+        if presplit_gate:
+            self.gate_split = torch.empty((3, N, H), dtype=torch.bfloat16, device=dev)
+            capi.moe_split_gate(gate_w, self.gate_split)
         self.w_local = capi.make_weights(gate_w, w13, s13, w2, s2)
         self.send = torch.empty(max(T * min(W, K), 1), self.row_bytes, dtype=torch.uint8,
                                 device=dev)
@@ -168,7 +174,8 @@ class ExpertParallelMoE:
         if self.peer:
             return self._forward_peer(sh, x, bias)
         c.moe_ep_dispatch(sh, self.W, self.gate_w, x, bias, self.send, self.send_counts, self.ws,
-                          topk_ids=self.ids[:T], topk_gates=self.gates[:T], counts=self.counts)
+                          topk_ids=self.ids[:T], topk_gates=self.gates[:T], counts=self.counts,
+                          gate_split=self.gate_split)
         recv_counts = exchange_counts(self.send_counts, self.group)
         sc = self.send_counts.cpu()
         rc = recv_counts.cpu()
@@ -195,7 +202,7 @@ class ExpertParallelMoE:
         c.moe_ep_dispatch_peer(sh, self.W, self.rank, self.T, self.gate_w, x, bias, self.p_recv,
                                self.p_counts, self.ws, topk_ids=self.ids[:T],
                                topk_gates=self.gates[:T], counts=self.counts,
-                               send_counts=self.send_counts)
+                               send_counts=self.send_counts, gate_split=self.gate_split)
         self._barrier()          # every rank's rows are in place
         c.moe_ep_shared(sh, self.W, self.w_local, self.ws)
         c.moe_ep_experts_peer(sh, self.W, self.rank, self.T, self.w_local, self.recv,
@@ -204,6 +211,11 @@ class ExpertParallelMoE:
         y = torch.empty(T, self.H, dtype=torch.bfloat16, device=self.device)
         c.moe_ep_combine_peer(sh, self.W, self.T, self.ret, self.ws, y)
         return y
+
+    def resplit_gate(self, stream=None) -> None:
+        """Re-make the centroids' bf16 terms after gate_w changed."""
+        if self.gate_split is not None:
+            capi.moe_split_gate(self.gate_w, self.gate_split, stream)
 
     def batch_counts(self) -> torch.Tensor:
         """Per-expert counts of the last step summed over all ranks (the

@@ -114,3 +114,5 @@ def test_launch_count_follows_the_router_path():
     assert bench.step_launches(32768, 256, 16, 0, 0, 7168) == 10  # K > 8: logits + top-K
     assert bench.step_launches(512, 32, 8, 0, 0, 7168) == 10     # N = 32: 128 x 64 tiles
     assert bench.step_launches(128, 256, 8, 0, 0, 7168) == 11
+    # an expert-parallel step at V3 prefill: 18 kernels, as in its launch list
+    assert bench.ep_step_launches(4096, 256, 8, 0, 0, 7168) == 18

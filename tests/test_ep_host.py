@@ -186,12 +186,12 @@ def test_ep_calls_reject_bad_arguments_on_the_host(capi):
     null = ctypes.c_void_p(0)
     # W = 3 does not divide N; W = 4 leaves 8 experts per rank (< 16)
     for w_bad in (3, 4):
-        assert lib.moe_ep_dispatch(sh, w_bad, null, null, null, null, null, null, null, 0, null,
-                                   null, 0, null) == -1
+        assert lib.moe_ep_dispatch(sh, w_bad, null, null, null, null, null, null, null, null, 0,
+                                   null, null, 0, null) == -1
         assert lib.moe_ep_experts(sh, w_bad, None, null, 0, 0, null, null, 0, null) == -1
         assert lib.moe_ep_combine(sh, w_bad, null, 0, null, 0, null, null) == -1
-    assert lib.moe_ep_dispatch(sh, 2, null, null, null, null, null, null, null, 0, null, null, 0,
-                               null) == -2
+    assert lib.moe_ep_dispatch(sh, 2, null, null, null, null, null, null, null, null, 0, null,
+                               null, 0, null) == -2
     assert lib.moe_ep_experts(sh, 2, None, null, 10, 41, null, null, 0, null) == -1
     assert lib.moe_ep_experts(sh, 2, None, null, -1, 0, null, null, 0, null) == -1
     assert lib.moe_ep_combine(sh, 2, null, -1, null, 0, null, null) == -1
@@ -200,6 +200,14 @@ def test_ep_calls_reject_bad_arguments_on_the_host(capi):
     assert lib.moe_ep_shared(sh, 2, None, ctypes.c_void_p(addr), 256, null) == -6
     assert lib.moe_ep_combine(sh, 2, null, 0, ctypes.c_void_p(addr + 8), 1 << 40, null,
                               null) == -7
+    # a pre-split gate off its 16-byte alignment (checked before any CUDA call);
+    # the buffers are never dereferenced
+    ws_ok, split_bad = ctypes.c_void_p(addr), ctypes.c_void_p(addr + 8)
+    big = capi.moe_ep_dispatch_workspace_size(sh, 2)
+    assert lib.moe_ep_dispatch(sh, 2, null, split_bad, null, null, null, null, null, ws_ok, 1,
+                               ws_ok, ws_ok, big, null) == -7
+    assert lib.moe_ep_dispatch_peer(sh, 2, 0, 64, null, split_bad, null, null, null, null, null,
+                                    ws_ok, ws_ok, null, ws_ok, big, null) == -7
 
 
 def test_peer_mode_calls_reject_bad_arguments_on_the_host(capi):
@@ -211,13 +219,13 @@ def test_peer_mode_calls_reject_bad_arguments_on_the_host(capi):
     # rank outside [0, W), T above T_cap, T_cap < 1, W not dividing N into >= 16 experts
     for W, rank, T_cap in [(2, 2, 64), (2, -1, 64), (2, 0, 63), (2, 0, 0), (4, 0, 64)]:
         assert lib.moe_ep_dispatch_peer(sh, W, rank, T_cap, null, null, null, null, null, null,
-                                        fake, fake, null, null, 0, null) == -1
+                                        null, fake, fake, null, null, 0, null) == -1
         assert lib.moe_ep_experts_peer(sh, W, rank, T_cap, None, null, fake, fake, null, 0,
                                        null) == -1
     assert lib.moe_ep_combine_peer(sh, 2, 63, null, null, 0, null, null) == -1
     # missing pointer arrays
-    assert lib.moe_ep_dispatch_peer(sh, 2, 0, 64, null, null, null, null, null, null, null, fake,
-                                    null, null, 0, null) == -2
+    assert lib.moe_ep_dispatch_peer(sh, 2, 0, 64, null, null, null, null, null, null, null, null,
+                                    fake, null, null, 0, null) == -2
     assert lib.moe_ep_experts_peer(sh, 2, 1, 64, None, null, null, fake, null, 0, null) == -2
     assert lib.moe_ep_experts_peer(sh, 2, 1, 64, None, null, fake, null, null, 0, null) == -2
     # workspace sizes: W T_cap rows of min(K, N/W) slots each, growing with T_cap

@@ -55,6 +55,10 @@ def emulate(w: I.Workload, W: int, xs_bits, dw, bias: np.ndarray, G: int = 0, M:
     wl_t = [ep.local_weights(dw.w13, dw.s13, dw.w2, dw.s2, N, W, r) for r in range(W)]
     wl = [capi.make_weights(dw.gate_w, *t) for t in wl_t]
     rb = capi.moe_ep_row_bytes(capi.shape_of(1, Hd, N, K, w.I, G, M))
+    # odd ranks route with the centroids split once beforehand, even ranks
+    # split them in the call: both must route as moe_forward does
+    gs = torch.empty((3, N, Hd), dtype=torch.bfloat16, device="cuda")
+    capi.moe_split_gate(dw.gate_w, gs)
     ranks = []
     for r, xb in enumerate(xs_bits):
         T = xb.shape[0]
@@ -71,7 +75,8 @@ def emulate(w: I.Workload, W: int, xs_bits, dw, bias: np.ndarray, G: int = 0, M:
         st["counts"] = torch.full((N,), -1, dtype=torch.int32, device="cuda")
         capi.moe_ep_dispatch(sh, W, dw.gate_w, st["xd"], bd, st["send"], st["sc"], st["ws"],
                              topk_ids=st["ids"] if T else None,
-                             topk_gates=st["gates"] if T else None, counts=st["counts"])
+                             topk_gates=st["gates"] if T else None, counts=st["counts"],
+                             gate_split=gs if r % 2 else None)
         capi.moe_ep_shared(sh, W, wl[r], st["ws"])
         ranks.append(st)
     torch.cuda.synchronize()
@@ -328,13 +333,16 @@ def emulate_peer(w: I.Workload, W: int, T_cap: int, steps, dw, bias: np.ndarray,
                       device="cuda") for _ in range(W)]
     ews = [torch.empty(capi.moe_ep_peer_expert_workspace_size(sh_cap, W, T_cap),
                        dtype=torch.uint8, device="cuda") for _ in range(W)]
+    gs = torch.empty((3, N, Hd), dtype=torch.bfloat16, device="cuda")
+    capi.moe_split_gate(dw.gate_w, gs)
     outs = []
     for xs_bits in steps:
         shs = [capi.shape_of(xb.shape[0], Hd, N, K, w.I, G, M) for xb in xs_bits]
         for r, xb in enumerate(xs_bits):
             T = xb.shape[0]
             xd = H.x_to_device(xb) if T else torch.empty(0, Hd, dtype=torch.bfloat16, device="cuda")
-            capi.moe_ep_dispatch_peer(shs[r], W, r, T_cap, dw.gate_w, xd, bd, p_recv, p_cnt, ws[r])
+            capi.moe_ep_dispatch_peer(shs[r], W, r, T_cap, dw.gate_w, xd, bd, p_recv, p_cnt, ws[r],
+                                      gate_split=gs if r % 2 == 0 else None)
             capi.moe_ep_shared(shs[r], W, wl[r], ws[r])
         for d in range(W):
             capi.moe_ep_experts_peer(shs[d], W, d, T_cap, wl[d], recv[d], cnt[d], p_ret, ews[d])
