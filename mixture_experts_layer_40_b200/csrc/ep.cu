@@ -402,11 +402,20 @@ __global__ void __launch_bounds__(256) ep_gather_rows_kernel(
   }
 }
 
+// 8 consecutive bf16 row elements as fp32 (streamed: each is read once)
+MOE_DEV void load8_bf16(const __nv_bfloat16* p, int64_t c, float (&v)[8]) {
+  const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p) + c);
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+  v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+}
+
 // Per received row: the sum over its local slots, by ascending expert id, of
 // g * Y[row], fp32 (the rank's share of the token's combine). Written to
 // out[j] (all-to-all mode), or in peer mode straight into the source's
 // return buffer: row j = s seg_rows + i goes to peer_ret[s] at row
-// rank * seg_rows + i; rows without a slot are not written.
+// rank * seg_rows + i; rows without a slot are not written. Each thread
+// takes 8 columns at a time and puts up to four rows' loads in flight
+// before their adds, which keep the ascending order.
 __global__ void __launch_bounds__(128) ep_reduce_kernel(
     const __nv_bfloat16* __restrict__ y_rows, const int32_t* __restrict__ ids,
     const float* __restrict__ gates, const int32_t* __restrict__ token_row, int H, int K,
@@ -416,30 +425,34 @@ __global__ void __launch_bounds__(128) ep_reduce_kernel(
   __shared__ float s_gate[kMaxK];
   __shared__ int s_n;
   const int64_t j = blockIdx.x;
-  if (threadIdx.x == 0) {
-    int id[kMaxK];
-    int n = 0;
-    for (int k = 0; k < K; ++k) {
-      const int e = ids[j * K + k];
-      if (e < 0) continue;
-      const int64_t r = token_row[j * K + k];
-      if (r < 0 || r >= routed_cap) {
-        flag_status(status, kStatusBounds);
-        continue;
-      }
-      int m = n;  // insertion by ascending expert id
-      while (m > 0 && id[m - 1] > e) {
-        id[m] = id[m - 1];
-        s_row[m] = s_row[m - 1];
-        s_gate[m] = s_gate[m - 1];
-        --m;
-      }
-      id[m] = e;
-      s_row[m] = r;
-      s_gate[m] = gates[j * K + k];
-      ++n;
+  // slot k (thread k) goes to position = the number of the row's local slots
+  // with a lower expert id (a token's experts are distinct); slots of other
+  // ranks' experts (id < 0) are skipped, rows out of range dropped and flagged
+  if (threadIdx.x < K) {
+    const int k = threadIdx.x;
+    const int e = ids[j * K + k];
+    int64_t r = -1;
+    float g = 0.0f;
+    bool ok = false;
+    if (e >= 0) {
+      r = token_row[j * K + k];
+      ok = r >= 0 && r < routed_cap;
+      if (!ok) flag_status(status, kStatusBounds);
+      g = gates[j * K + k];
     }
-    s_n = n;
+    const unsigned mask = (1u << K) - 1u;
+    int pos = 0;
+    for (int i = 0; i < K; ++i) {
+      const int ei = __shfl_sync(mask, e, i);
+      const bool oki = __shfl_sync(mask, ok, i);
+      pos += (oki && ei < e) ? 1 : 0;
+    }
+    const int n_ok = __popc(__ballot_sync(mask, ok));
+    if (ok) {
+      s_row[pos] = r * H;
+      s_gate[pos] = g;
+    }
+    if (k == 0) s_n = n_ok;
   }
   __syncthreads();
   const int n = s_n;
@@ -450,17 +463,29 @@ __global__ void __launch_bounds__(128) ep_reduce_kernel(
     dst_row = peer_ret[s] + ((int64_t)rank * seg_rows + (j - s * seg_rows)) * H;
   }
   float4* o = reinterpret_cast<float4*>(dst_row);
-  for (int c = threadIdx.x; c < H / 4; c += blockDim.x) {
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int k = 0; k < n; ++k) {
-      const uint2 u = __ldcs(reinterpret_cast<const uint2*>(y_rows + s_row[k] * H) + c);
-      const float g = s_gate[k];
-      acc.x = fmaf(g, bf16_lo(u.x), acc.x);
-      acc.y = fmaf(g, bf16_hi(u.x), acc.y);
-      acc.z = fmaf(g, bf16_lo(u.y), acc.z);
-      acc.w = fmaf(g, bf16_hi(u.y), acc.w);
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    int k = 0;
+    for (; k + 4 <= n; k += 4) {
+      float f[4][8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) load8_bf16(y_rows + s_row[k + q], c, f[q]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float g = s_gate[k + q];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, f[q][i], acc[i]);
+      }
     }
-    o[c] = acc;
+    for (; k < n; ++k) {
+      float f[8];
+      load8_bf16(y_rows + s_row[k], c, f);
+      const float g = s_gate[k];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, f[i], acc[i]);
+    }
+    o[2 * c] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[2 * c + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
   if (peer_ret != nullptr) __threadfence_system();
 }
