@@ -785,8 +785,9 @@ size_t moe_ep_peer_expert_workspace_size(moe_shape sh, int32_t W, int32_t T_cap)
 int moe_ep_dispatch_peer(moe_shape sh, int32_t W, int32_t rank, int32_t T_cap,
                          const float* gate_w, const void* gate_split_opt, const void* x,
                          const float* bias, int32_t* topk_ids_opt, float* topk_gates_opt,
-                         int32_t* counts_opt, uint8_t* const* peer_recv, int32_t* const* peer_counts,
-                         int32_t* send_counts_opt, void* ws, size_t ws_bytes, void* stream) {
+                         int32_t* counts_opt, uint8_t* const* peer_recv,
+                         int32_t* const* peer_counts, int32_t* send_counts_opt, void* ws,
+                         size_t ws_bytes, void* stream) {
   if (!peer_ok(sh, W, rank, T_cap)) return MOE_ERR_SHAPE;
   if (!peer_recv || !peer_counts) return MOE_ERR_NULL;
   SendRows dst{nullptr, 0, peer_recv, (int64_t)rank * T_cap, row_bytes_of(sh)};
