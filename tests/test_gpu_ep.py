@@ -261,6 +261,18 @@ def test_expert_parallel_layer_one_rank_nccl():
         check_against_forward(w, st, dw, case.bias)
         total = layer.batch_counts()
         assert int(total.sum()) == 800
+        # new centroids: resplit_gate makes the layer route as one that splits
+        # them in every dispatch
+        ids0 = layer.ids[:200].clone()
+        dw.gate_w.mul_(-1.0)
+        layer.resplit_gate()
+        fresh = ep.ExpertParallelMoE(w.T, w.H, w.N, w.K, w.I, 1, 0, dw.gate_w, w13, s13, w2, s2,
+                                     presplit_gate=False)
+        ya, yb = layer.forward(xd, bd), fresh.forward(xd, bd)
+        torch.cuda.synchronize()
+        assert layer.status() == 0 and fresh.status() == 0
+        assert torch.equal(ya, yb) and torch.equal(layer.ids[:200], fresh.ids[:200])
+        assert not torch.equal(layer.ids[:200], ids0)   # the routing did change
     finally:
         dist.destroy_process_group()
 
