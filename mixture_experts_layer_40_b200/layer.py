@@ -108,6 +108,14 @@ class MoELayer:
         if self.gate_split is not None:
             capi.moe_split_gate(self.weights.gate_w, self.gate_split, stream)
 
+    def weights_changed(self, stream=None) -> None:
+        """After the weights were updated in place (gate_w, w13/s13, w2/s2):
+        re-make the centroids' bf16 terms and, once a backward has made them,
+        the transposed expert weights the backward reads."""
+        self.resplit_gate(stream)
+        if getattr(self, "_wt", None) is not None:
+            capi.moe_transpose_weights(self.shape, self._cw, *self._wt_bufs, stream)
+
     def route(self, x: torch.Tensor, bias: torch.Tensor, stream=None):
         capi.moe_route(self.shape, self.weights.gate_w, x, bias, self.ids, self.gates,
                        self.counts, self.ws, stream)

@@ -100,6 +100,36 @@ def test_transposed_weights_bit_exact():
     assert np.array_equal(w2t, w2.transpose(0, 2, 1)) and np.array_equal(s2t, s2.transpose(0, 2, 1))
 
 
+def test_weights_changed_matches_a_fresh_layer():
+    """After an in-place weight update, weights_changed re-makes the split
+    centroids and the transposed expert weights: forward and backward then
+    give the bits of a layer built on the new weights."""
+    w = I.Workload("bwc", T=160, H=512, N=16, K=4, I=256, bias_range=0.1, seed=58)
+    case = H.make_case(w)
+    dw = device_weights(w, case.pool, case.gate_w, "cuda")
+    x = H.x_to_device(case.x_bits)
+    bias = torch.from_numpy(case.bias).cuda()
+    dy = H.x_to_device(_dy(w, 4))
+    a = MoELayer(w.T, w.H, w.N, w.K, w.I, dw)
+    a.forward(x, bias)
+    a.backward(dy, x=x)                       # makes the transposed weights
+    # an update: new centroids, new scales, and one expert's codes reversed
+    dw.gate_w.mul_(-0.5)
+    dw.s13.mul_(2.0)
+    dw.s2.mul_(0.25)
+    dw.w13[3] = dw.w13[3].flip(0).clone()
+    a.weights_changed()
+    b = MoELayer(w.T, w.H, w.N, w.K, w.I, dw)
+    ya, yb = a.forward(x, bias), b.forward(x, bias)
+    ga, gb = a.backward(dy, x=x), b.backward(dy, x=x)
+    torch.cuda.synchronize()
+    assert a.status() == 0 and b.status() == 0
+    assert torch.equal(ya, yb) and torch.equal(a.ids, b.ids) and torch.equal(a.gates, b.gates)
+    for u, v in zip(ga, gb):
+        assert torch.equal(u, v)
+    assert all(torch.equal(u, v) for u, v in zip(a._wt_bufs, b._wt_bufs))
+
+
 @pytest.mark.parametrize("t", [300, 77])
 def test_backward_small(t):
     w = I.Workload(f"bw{t}", T=t, H=512, N=32, K=4, I=256, bias_range=0.1, seed=52 + t)
