@@ -225,8 +225,16 @@ def make_weights(gate_w, w13, s13, w2, s2, gate_split=None) -> moe_weights:
                                                             "gate_split"))
 
 
+def _check_split_size(gate_split, N: int, H: int) -> None:
+    # the three bf16 terms are written (moe_split_gate) or read whole
+    if gate_split is not None and gate_split.numel() < 3 * N * H:
+        raise ValueError(f"gate_split holds {gate_split.numel()} values; the three terms of "
+                         f"[{N}, {H}] centroids need {3 * N * H}")
+
+
 def moe_split_gate(gate_w, gate_split, stream=None):
     N, H = gate_w.shape
+    _check_split_size(gate_split, N, H)
     _check("moe_split_gate", LIB.moe_split_gate(
         _ptr(gate_w, torch.float32, "gate_w"), N, H, _ptr(gate_split, torch.bfloat16, "gate_split"),
         _stream(stream)))
@@ -304,6 +312,7 @@ def moe_ep_dispatch(sh: moe_shape, W: int, gate_w, x, bias, send, send_counts, w
                     topk_ids=None, topk_gates=None, counts=None, stream=None, gate_split=None):
     """send: uint8 [send_cap, moe_ep_row_bytes(sh)]; send_counts: int32 [W, 2];
     gate_split: None, or bf16 [3, N, H] from moe_split_gate."""
+    _check_split_size(gate_split, sh.N, sh.H)
     _check("moe_ep_dispatch", LIB.moe_ep_dispatch(
         sh, W, _ptr(gate_w, torch.float32, "gate_w"),
         _ptr(gate_split, torch.bfloat16, "gate_split"), _ptr(x, torch.bfloat16, "x"),
@@ -343,6 +352,7 @@ def moe_ep_dispatch_peer(sh: moe_shape, W: int, rank: int, T_cap: int, gate_w, x
                          send_counts=None, stream=None, gate_split=None):
     """peer_recv, peer_counts: int64 device tensors [W] of device pointers;
     gate_split as in moe_ep_dispatch."""
+    _check_split_size(gate_split, sh.N, sh.H)
     _check("moe_ep_dispatch_peer", LIB.moe_ep_dispatch_peer(
         sh, W, rank, T_cap, _ptr(gate_w, torch.float32, "gate_w"),
         _ptr(gate_split, torch.bfloat16, "gate_split"), _ptr(x, torch.bfloat16, "x"),

@@ -122,3 +122,17 @@ def test_split_gate_rejects_bad_arguments(capi):
     sh = capi.shape_of(64, 256, 16, 4, 128)
     w = capi.moe_weights(16, 16, 16, 16, 16, 8)
     assert lib.moe_forward(sh, ctypes.byref(w), 16, 16, 16, None, None, None, 256, 1 << 30, None) == -7
+
+
+def test_split_gate_buffer_size_checked_in_the_binding(capi):
+    import torch
+    gate_w = torch.zeros(16, 256)
+    small = torch.zeros(3 * 16 * 256 - 1, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="gate_split"):
+        capi.moe_split_gate(gate_w, small)
+    sh = capi.shape_of(64, 256, 16, 4, 128)
+    with pytest.raises(ValueError, match="gate_split"):
+        capi.moe_ep_dispatch(sh, 1, None, None, None, None, None, None, gate_split=small)
+    with pytest.raises(ValueError, match="gate_split"):
+        capi.moe_ep_dispatch_peer(sh, 1, 0, 64, None, None, None, None, None, None,
+                                  gate_split=small)
