@@ -316,3 +316,43 @@ def test_wgrad_up_uses_x_quantised_down_its_columns():
     assert np.max(np.abs(q["dwg"] - ref)) <= 1e-6 * np.max(np.abs(ref))
     wrong = O.dequantize_1x128(*O.quantize_1x128(x))
     assert np.max(np.abs(wrong - x_col)) > 1e-3 * np.max(np.abs(x))
+
+
+def test_dgrad_quantises_dy_and_dg_du_in_row_tiles():
+    """Where the Dgrad quantises, seen through scaled identity weights
+    (H = I = 128, one lossless 128x128 block each: W_gate = 2^-3 I,
+    W_up = 2^-4 I, W_down = 2^-2 I). Then dh = Q(dy) W_down = 2^-2 dy_hat,
+    and dx = Q(dG) W_gate + Q(dU) W_up = 2^-3 dG_hat + 2^-4 dU_hat, element
+    by element, with every hat the page's per-tile rule ("DeepSeek-V3
+    Technical Report" (deepforge), "Per-tile FP8 scaling") applied along the
+    rows. dG = dh U silu'(G) and dU = dh silu(G) use the forward's G and U
+    from the dequantised x (silu and silu' are pinned above: brute-force
+    loops and finite differences). Gaussian dy, x and activations are lossy
+    under the rule, so an oracle that fed the unquantised dy, dG or dU to a
+    Dgrad GEMM fails here."""
+    from tests.test_oracle_experts import _page_tile_1x128
+    rng = np.random.default_rng(55)
+    rows = 6
+    x = I.bf16_bits_to_f32(I.f32_to_bf16_bits(
+        (rng.standard_normal((rows, 128)) * 2.0).astype(np.float32)))
+    dy = (rng.standard_normal((rows, 128)) * 10.0 ** rng.uniform(-2, 2, (rows, 1))).astype(np.float32)
+    cg, cu, cd = 2.0 ** -3, 2.0 ** -4, 2.0 ** -2
+    wg, wu, wd = (O.dequantize_128x128(*O.quantize_128x128((np.eye(128) * c).astype(np.float32)))
+                  for c in (cg, cu, cd))
+    for m, c in ((wg, cg), (wu, cu), (wd, cd)):
+        assert np.array_equal(m, np.eye(128) * c)             # lossless blocks
+    xq, xs = O.quantize_1x128(x)
+    q = O.expert_ffn_backward_q(xq, xs, x, dy, wg, wu, wd)
+    dy_hat = _page_tile_1x128(dy)
+    assert np.max(np.abs(dy_hat - dy)) > 1e-3 * np.max(np.abs(dy))   # dy's quantisation shows
+    assert np.array_equal(q["dh"], cd * dy_hat)
+    x_hat = _page_tile_1x128(x)
+    g, u = cg * x_hat, cu * x_hat
+    dh = cd * dy_hat
+    d_g = dh * u * O.silu_grad(g)
+    d_u = dh * O.silu(g)
+    dg_hat, du_hat = _page_tile_1x128(d_g), _page_tile_1x128(d_u)
+    for a, b in ((d_g, dg_hat), (d_u, du_hat)):
+        assert np.max(np.abs(a - b)) > 1e-3 * np.max(np.abs(a))      # and dG's and dU's
+    expect = cg * dg_hat + cu * du_hat
+    assert np.max(np.abs(q["dx"] - expect)) <= 1e-12 * np.max(np.abs(expect))

@@ -199,3 +199,32 @@ def test_fp8_error_band_against_unquantised():
     yr = O.moe_forward(x, g, b, w.K, ew, mode="R")["y"]
     rel = np.sqrt(np.mean((yq - yr) ** 2)) / np.sqrt(np.mean(yr ** 2))
     assert 0.04 < rel < 0.09, rel
+
+
+def test_forced_routing_keeps_the_unbiased_gates():
+    """The near-tie rule re-runs the layer with another routing decision
+    (the GPU's ids). The gates then follow the pages' definition for those
+    ids ("DeepSeek-V3: Auxiliary-Loss-Free MoE Load Balancing, ...", section
+    III: g = s_i / sum of the chosen s, the bias only choosing): from the
+    unbiased affinities, whatever the bias. Handing the layer its own routing
+    back reproduces the unforced run exactly; a forced routing of the least
+    likely experts under a large bias gets gates from sigma(u . e_i), computed
+    here with plain loops, and the forward and backward agree on them."""
+    w, x, g, b, pool, ew = _tiny_all()
+    b = (np.sign(I.make_bias(w)) * 0.5).astype(np.float32)      # large bias
+    base = O.moe_forward(x, g, b, w.K, ew, mode="Q")
+    again = O.moe_forward(x, g, b, w.K, ew, mode="Q", ids=base["ids"])
+    assert np.array_equal(again["y"], base["y"]) and np.array_equal(again["gates"], base["gates"])
+    _, _, _, score = O.route(x, g, b, w.K)
+    forced = np.argsort(score, axis=1, kind="stable")[:, :w.K].astype(np.int32)
+    expect = np.empty(forced.shape)
+    for t in range(w.T):
+        s = [1.0 / (1.0 + math.exp(-sum(float(x[t, c]) * float(g[e, c]) for c in range(w.H))))
+             for e in forced[t]]
+        expect[t] = np.array(s) / sum(s)
+    fw = O.moe_forward(x, g, b, w.K, ew, mode="Q", ids=forced)
+    assert np.array_equal(fw["ids"], forced)
+    assert np.max(np.abs(fw["gates"] - expect)) < 1e-12
+    dy = np.random.default_rng(3).standard_normal((w.T, w.H)).astype(np.float32)
+    bw = O.moe_backward(x, g, b, w.K, ew, dy, mode="Q", ids=forced, tokens=[0, 5])
+    assert np.array_equal(bw["gates"], fw["gates"])
