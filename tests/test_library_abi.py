@@ -136,3 +136,44 @@ def test_split_gate_buffer_size_checked_in_the_binding(capi):
     with pytest.raises(ValueError, match="gate_split"):
         capi.moe_ep_dispatch_peer(sh, 1, 0, 64, None, None, None, None, None, None,
                                   gate_split=small)
+
+
+def _prototypes():
+    """name -> (return type, [parameter declarations]) of every function the
+    header declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    out = {}
+    for ret, name, params in re.findall(r"\b(int|size_t|int64_t|void)\s+(moe_[a-z0-9_]+)\s*"
+                                        r"\(([^)]*)\)\s*;", text):
+        ps = [p.strip() for p in params.split(",") if p.strip() and p.strip() != "void"]
+        out[name] = (ret, ps)
+    return out
+
+
+def test_binding_signatures_match_the_header(capi):
+    """Every prototype of include/moe_capi.h against the ctypes signature the
+    binding sets: the same number of parameters, and each of the same kind
+    (pointer, 32- or 64-bit integer, size, float, or the shape struct passed
+    by value), so no argument can land in another's place."""
+    protos = _prototypes()
+    assert set(protos) == set(declared_functions())
+    assert set(protos) == set(capi.SIGNATURES)
+    scalar = {"int32_t": ctypes.c_int32, "int": ctypes.c_int, "int64_t": ctypes.c_int64,
+              "size_t": ctypes.c_size_t, "float": ctypes.c_float, "moe_shape": capi.moe_shape}
+    rets = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "int64_t": ctypes.c_int64}
+    for name, (ret, params) in protos.items():
+        res, args = capi.SIGNATURES[name]
+        assert res is rets[ret], name
+        assert len(args) == len(params), f"{name}: {len(args)} argtypes, {len(params)} in the header"
+        for decl, arg in zip(params, args):
+            if "*" in decl:
+                # device or host pointers: void* in the binding, or a typed
+                # pointer to a struct or pointer array the binding builds
+                assert arg is ctypes.c_void_p or issubclass(arg, ctypes._Pointer), (name, decl)
+                if "moe_weights" in decl or "moe_ws_layout" in decl:
+                    assert issubclass(arg, ctypes._Pointer), (name, decl)
+            else:
+                ctype = decl.replace("const ", "").split()[0]
+                assert arg is scalar[ctype], (name, decl, arg)
