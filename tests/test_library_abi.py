@@ -177,3 +177,20 @@ def test_binding_signatures_match_the_header(capi):
             else:
                 ctype = decl.replace("const ", "").split()[0]
                 assert arg is scalar[ctype], (name, decl, arg)
+
+
+def test_product_fails_loudly_without_the_library(tmp_path):
+    """With libmoe_b200.so absent, importing the binding, the layer or the
+    expert-parallel driver raises ImportError naming the missing library:
+    there is no CPU fallback to run instead."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "mixture_experts_layer_40_b200")
+    shutil.copytree(pkg, tmp_path / "mixture_experts_layer_40_b200",
+                    ignore=shutil.ignore_patterns("*.so", "csrc", "__pycache__"))
+    for mod in ("capi", "layer", "ep"):
+        r = subprocess.run([sys.executable, "-c", f"import mixture_experts_layer_40_b200.{mod}"],
+                           cwd=tmp_path, capture_output=True, text=True, timeout=300)
+        assert r.returncode != 0, mod
+        assert "ImportError" in r.stderr and "no CPU fallback" in r.stderr, (mod, r.stderr[-500:])
