@@ -194,3 +194,42 @@ def test_product_fails_loudly_without_the_library(tmp_path):
                            cwd=tmp_path, capture_output=True, text=True, timeout=300)
         assert r.returncode != 0, mod
         assert "ImportError" in r.stderr and "no CPU fallback" in r.stderr, (mod, r.stderr[-500:])
+
+
+def _imports(path):
+    """Top-level module names imported anywhere in a Python file, with the
+    function each import sits in (None at module level)."""
+    import ast
+    tree = ast.parse(open(path).read())
+    found = []
+
+    def walk(node, fn):
+        for child in ast.iter_child_nodes(node):
+            name = child.name if isinstance(child, (ast.FunctionDef, ast.AsyncFunctionDef)) else fn
+            if isinstance(child, ast.Import):
+                found.extend((a.name.split(".")[0], fn) for a in child.names)
+            elif isinstance(child, ast.ImportFrom) and child.module and child.level == 0:
+                found.append((child.module.split(".")[0], fn))
+            walk(child, name)
+    walk(tree, None)
+    return found
+
+
+def test_oracle_and_product_are_independent():
+    """The product package never imports the oracle and the oracle never
+    imports the product; the CUDA sources do not name it. bench.py reaches
+    the oracle only from its CPU-baseline helpers (oracle_setup,
+    oracle_sample_step), which the reference arm and the cpu_baseline leg
+    call; the smoke check imports it inside smoke() only."""
+    import glob
+    pkg = os.path.join(ROOT, "mixture_experts_layer_40_b200")
+    for f in glob.glob(os.path.join(pkg, "*.py")):
+        assert all(m != "oracle" for m, _ in _imports(f)), f
+    for f in glob.glob(os.path.join(ROOT, "oracle", "*.py")):
+        assert all(m != "mixture_experts_layer_40_b200" for m, _ in _imports(f)), f
+    for f in glob.glob(os.path.join(pkg, "csrc", "*")) + glob.glob(os.path.join(ROOT, "include", "*")):
+        assert "oracle" not in open(f).read().lower(), f
+    users = {fn for m, fn in _imports(os.path.join(ROOT, "bench.py")) if m == "oracle"}
+    assert users == {"oracle_setup", "oracle_sample_step"}, users
+    users = {fn for m, fn in _imports(os.path.join(ROOT, "__graft_entry__.py")) if m == "oracle"}
+    assert users == {"smoke"}, users
