@@ -113,6 +113,47 @@ CASES = [
      "            dgates[rr, kk] = np.sum(dy[rr].astype(np.float64) * y_e, axis=1)",
      "            dgates[rr, kk] = gates[rr, kk] * np.sum(dy[rr].astype(np.float64) * y_e, axis=1)",
      "test_oracle_backward", "test_gate_gradients_are_dy_dot_expert_output"),
+    ("gate logits in float32",
+     "    return np.asarray(x, np.float64) @ np.asarray(gate_w, np.float64).T",
+     "    return (np.asarray(x, np.float32) @ np.asarray(gate_w, np.float32).T).astype(np.float64)",
+     "test_oracle_router", "test_logits_exact_on_small_case"),
+    ("counts off by one for expert 0",
+     "    return np.bincount(np.asarray(ids).ravel(), minlength=n_experts).astype(np.int32)",
+     "    return (np.bincount(np.asarray(ids).ravel(), minlength=n_experts) + (np.arange(n_experts) == 0)).astype(np.int32)",
+     "test_oracle_router", "test_route_invariants_tiny"),
+    ("bias update in float64", "    return (bias + step).astype(np.float32)",
+     "    return (bias.astype(np.float64) + float(gamma) * delta).astype(np.float32)",
+     "test_oracle_router", "test_bias_update_float32_rounding"),
+    ("negative zero loses its sign", "    codes = np.where(neg, mag | 0x80, mag).astype(np.uint8)",
+     "    codes = np.where(neg & (mag > 0), mag | 0x80, mag).astype(np.uint8)",
+     "test_oracle_codec", "test_roundtrip_all_codes"),
+    ("subnormal exponent off by one",
+     "            table[code] = sign * (man_field / 8.0) * 2.0 ** (1 - 7)",
+     "            table[code] = sign * (man_field / 8.0) * 2.0 ** (0 - 7)",
+     "test_oracle_codec", "test_decode_known_codes"),
+    ("weight blocks assembled transposed",
+     "        return m.transpose(0, 2, 1, 3).reshape(nb * TILE, kb * TILE)",
+     "        return m.transpose(0, 3, 1, 2).reshape(nb * TILE, kb * TILE)",
+     "test_oracle_experts", "test_assembly_places_pool_blocks"),
+    ("gate mass not normalised",
+     "        p[q] = np.sum(s[lo:hi] / np.sum(s[lo:hi], axis=1, keepdims=True), axis=0) / t_seq",
+     "        p[q] = np.sum(s[lo:hi], axis=0) / t_seq",
+     "test_oracle_routing_ext", "test_balance_stats_closed_forms"),
+    ("balance loss without alpha", "        loss[q] = alpha * np.sum(f[q] * p[q])",
+     "        loss[q] = np.sum(f[q] * p[q])",
+     "test_oracle_routing_ext", "test_balance_stats_closed_forms"),
+    ("dU from U instead of silu(G)", "    d_u = dh * silu(g)\n    dgq", "    d_u = dh * u\n    dgq",
+     "test_oracle_backward", "test_dgrad_quantises_dy_and_dg_du_in_row_tiles"),
+    ("dW_up from dG", "    dwu = q(d_u.astype(np.float32)).T @ q(x32)",
+     "    dwu = q(d_g.astype(np.float32)).T @ q(x32)",
+     "test_oracle_backward", "test_wgrad_up_uses_x_quantised_down_its_columns"),
+    ("128x1 tiles run along the columns",
+     "    return quantize_1x128(np.ascontiguousarray(pad.T))",
+     "    c2, s2 = quantize_1x128(np.ascontiguousarray(pad))\n    return quantize_1x128(np.ascontiguousarray(dequantize_1x128(c2, s2).astype(np.float32).T))",
+     "test_oracle_backward", "test_quantize_128x1_tiles_run_down_the_rows"),
+    ("backward without the shared expert", "    for e in list(np.unique(ids[keep])) + [n]:",
+     "    for e in list(np.unique(ids[keep])):",
+     "test_oracle_backward", "test_dx_matches_finite_differences"),
 ]
 
 

@@ -152,6 +152,12 @@ def test_bias_update_float32_rounding():
     # exact double result of a float32 add, then one rounding to float32
     assert nb[0] == np.float32(1.0 - g) and nb[1] == np.float32(1.0 + g)
     assert nb.dtype == np.float32
+    # biases where adding the float32 gamma and adding the float64 1e-3 round
+    # to different float32 values: the update is the float32 add (gamma = 1e-3f)
+    b = np.array([-4.167452425463125e-05, 0.004282602109014988], np.float32)
+    nb = O.update_bias(b, np.array([1, 3]), 2, 2, 1e-3)
+    assert nb[0] == np.float32(float(b[0]) + g) and nb[1] == np.float32(float(b[1]) - g)
+    assert nb[0] != np.float32(float(b[0]) + 1e-3) and nb[1] != np.float32(float(b[1]) - 1e-3)
 
 
 def test_gamma_zero_freezes_bias():
