@@ -1,7 +1,13 @@
 """Benchmark of the MoE layer forward (plus the per-step bias update) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3_prefill]
-                    [--impl ours|reference] [--no-cpu-baseline]
+                    [--impl ours|reference] [--no-cpu-baseline] [--backward]
+                    [--groups G --topk-groups M] [--ep [--peer]]
+
+`--backward` also times the FP8 backward of the expert path after the step;
+`--groups/--topk-groups` route node-limited; `--ep` runs the expert-parallel
+step instead (routed experts sharded over the ranks), `--peer` with the
+kernels storing rows into the other ranks' buffers.
 
 With --gpus N > 1 and no rank environment (RANK / WORLD_SIZE), bench.py
 starts the N ranks itself under torchrun on 127.0.0.1.
